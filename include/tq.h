@@ -1,0 +1,144 @@
+/*
+ * tq.h -- C ABI of libtq: ternary weight-only grouped linear layer on B200.
+ *
+ * The operations follow two pages:
+ *   "precisit/pack-unpack-run" (codec.py description and payload-rate
+ *   paragraph): per group of G input columns, a mean-absolute scale rounded to
+ *   fp16 (binary16), nearest-even ternary codes, five base-three digits per
+ *   byte, each group byte-aligned with zero-trit padding, bytes 243..255
+ *   invalid, a zero stored scale producing a zero group, decoding to bf16.
+ *   tiny-llm "Week 2 Day 3: Quantize the Model" ("Mathematical Formulation",
+ *   "Computation Flow"): C = A B^T with B reconstructed per group and the
+ *   products accumulated in float.
+ *
+ * Layout (all row-major, all buffers contiguous, no padding between rows):
+ *   W, W_out  bf16   [N][K]                      weights, nn.Linear "out x in"
+ *   codes     uint8  [N][K/G][B],  B = ceil(G/5) one byte-aligned run per group
+ *   scales    fp16   [N][K/G]                    one binary16 scale per group
+ *   X         bf16   [M][K]                      activations
+ *   Y         fp32 or bf16 [M][N]                Y = X . What^T
+ * Byte encoding: weight j of a group (0 <= j < G) is digit (j mod 5) of byte
+ * floor(j/5); digit d = t + 1 for trit t in {-1, 0, +1}; byte = sum_i d_i 3^i,
+ * the first weight being the least significant digit.  Positions j >= G in
+ * the last byte hold the padding digit 1 (the zero trit).
+ * Decoded weight: What = +0 if t == 0 or the scale is +0, else
+ * t * RNE_bf16(scale).  A group with an invalid byte, a padding digit other
+ * than 1, or a scale that is NaN, Inf or has its sign bit set, decodes to
+ * bf16 NaN, so every output that touches it is NaN.
+ *
+ * Calling convention: every pointer except the sizes is a DEVICE pointer
+ * owned by the caller; the library never allocates or frees device memory
+ * and never synchronizes.  Work is enqueued on `stream` (NULL = legacy
+ * default stream).  A call returns TQ_OK once its kernels are enqueued; a
+ * synchronous error code means nothing was launched.  Data errors found by
+ * the kernels are OR-ed into *d_err (a device word the caller zeroes; may be
+ * NULL) using the TQ_DERR_* bits.  No exceptions cross this boundary and
+ * there is no CPU fallback.  Calls are thread-safe.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *tq_stream_t;
+
+typedef enum {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1, /* null pointer, bad shape, G out of range, K % G != 0, overlap */
+    TQ_ERR_ALIGNMENT = 2,   /* a pointer misses the alignment stated for it */
+    TQ_ERR_UNSUPPORTED = 3, /* valid arguments this build cannot run (e.g. no sm_100 device) */
+    TQ_ERR_CUDA = 4         /* a CUDA launch or attribute call failed */
+} tq_status;
+
+typedef enum { TQ_OUT_F32 = 0, TQ_OUT_BF16 = 1 } tq_out_dtype;
+
+/* Asynchronous data-error bits written to *d_err. */
+#define TQ_DERR_BYTE     1u  /* a code byte >= 243 (decode, matmul)               */
+#define TQ_DERR_PADDING  2u  /* a padding digit other than 1 (decode, matmul)     */
+#define TQ_DERR_WEIGHT   4u  /* a NaN or Inf weight (quantize): group stored as 0 */
+#define TQ_DERR_SCALE    8u  /* a stored scale NaN, Inf or negative (decode, mm)  */
+#define TQ_DERR_OVERFLOW 16u /* a group mean that overflows binary16 (quantize)   */
+#define TQ_DERR_TIMEOUT  32u /* a bounded pipeline wait gave up (matmul)          */
+
+/* Largest supported group size. */
+#define TQ_MAX_G 4096
+
+/* Bytes of the codes buffer: N * (K/G) * ceil(G/5).  0 for invalid shapes. */
+TQ_API size_t tq_codes_bytes(int64_t N, int64_t K, int G);
+/* Bytes of the scales buffer: N * (K/G) * 2.  0 for invalid shapes. */
+TQ_API size_t tq_scales_bytes(int64_t N, int64_t K, int G);
+/* Bytes of device scratch tq_gemv / tq_gemm need for these shapes (may be 0). */
+TQ_API size_t tq_workspace_bytes(int64_t M, int64_t N, int64_t K, int G);
+
+/*
+ * Quantize and pack ("precisit/pack-unpack-run", codec.py: mean-absolute
+ * scale rounded to fp16, nearest-even ternary codes, base-3 packing).
+ * W_bf16: [N][K] bf16, 16-byte aligned.  codes: tq_codes_bytes() bytes.
+ * scales_f16: [N][K/G] binary16, 2-byte aligned.
+ * Scale = RNE_binary16(exact mean of |w| over the group); trit =
+ * clamp(round_half_even(w / scale), -1, 1), all zero when the scale is +0.
+ * A group with a NaN/Inf weight or a mean >= 65520 is stored as a zero group
+ * and flagged (TQ_DERR_WEIGHT / TQ_DERR_OVERFLOW).
+ * Errors: TQ_ERR_INVALID_ARG for N < 0, K < 0, G < 1, G > TQ_MAX_G, K % G,
+ * null pointers with nonzero sizes, or codes/scales overlapping W;
+ * TQ_ERR_ALIGNMENT; TQ_ERR_CUDA.
+ */
+TQ_API tq_status tq_quantize_pack(const void *W_bf16, int64_t N, int64_t K, int G, uint8_t *codes,
+                           void *scales_f16, uint32_t *d_err, tq_stream_t stream);
+
+/*
+ * Decode to bf16 ("precisit/pack-unpack-run", codec.py: decoding; bytes
+ * 243..255 invalid; weights restored as bf16).
+ * codes/scales as produced by tq_quantize_pack; W_bf16_out: [N][K] bf16,
+ * 16-byte aligned.  Rejected groups are written as bf16 NaN and flagged
+ * (TQ_DERR_BYTE, TQ_DERR_PADDING, TQ_DERR_SCALE).
+ */
+TQ_API tq_status tq_unpack_bf16(const uint8_t *codes, const void *scales_f16, int64_t N, int64_t K,
+                         int G, void *W_bf16_out, uint32_t *d_err, tq_stream_t stream);
+
+/*
+ * Fused unpack-and-scale matmul for decode (tiny-llm "Week 2 Day 3",
+ * "Computation Flow"; the scale is applied once per group as in its "SIMD
+ * Matvec" stage): Y[m][n] = sum_g RNE_bf16(s[n][g]) * sum_{j in g} t[n][j] X[m][j],
+ * accumulated in fp32, written as fp32 or RNE bf16.  Any M >= 1; tuned for
+ * M <= 16 (CUDA cores).  X: [M][K] bf16, 16-byte aligned; Y: [M][N]
+ * (fp32: 4-byte aligned, bf16: 2-byte aligned), must not overlap the inputs.
+ * workspace: at least tq_workspace_bytes(M, N, K, G) bytes of device scratch
+ * (NULL allowed when that is 0), 256-byte aligned.
+ */
+TQ_API tq_status tq_gemv(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
+                  int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,
+                  size_t ws_bytes, uint32_t *d_err, tq_stream_t stream);
+
+/*
+ * Fused unpack-and-scale matmul for prefill: same result definition as
+ * tq_gemv, computed on the tensor cores (tcgen05, fp32 accumulators in
+ * tensor memory) from bf16 weights decoded on chip: What = t * RNE_bf16(s).
+ * Same arguments and alignment rules as tq_gemv.
+ */
+TQ_API tq_status tq_gemm(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
+                  int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,
+                  size_t ws_bytes, uint32_t *d_err, tq_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+TQ_API const char *tq_status_string(tq_status s);
+/* Library version and build flags (static string). */
+TQ_API const char *tq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

@@ -345,16 +345,31 @@ uint32_t oracle_unpack_bf16(const uint8_t *codes, const uint16_t *scales, int64_
     return err;
 }
 
+/* Value of every bf16 bit pattern, filled once from oracle_bf16_value. */
+static double bf16_table[65536];
+static int bf16_table_ready = 0;
+
+static const double *bf16_values(void)
+{
+    if (!bf16_table_ready) {
+        for (uint32_t h = 0; h < 65536; h++)
+            bf16_table[h] = oracle_bf16_value((uint16_t)h);
+        bf16_table_ready = 1;
+    }
+    return bf16_table;
+}
+
 /*
  * [mm] Y[m][n] = sum_k X[m][k] * What[n][k] for the requested rows m in
- * rows[0..nrows) (all rows if rows == NULL), accumulated in binary64.  Each
- * product of two bf16 values is exact in binary64.
+ * rows[0..nrows) (all rows if rows == NULL), accumulated in binary64 in
+ * increasing k.  Each product of two bf16 values is exact in binary64.
  * Y: [nrows x N] binary64.
  */
 void oracle_matmul(const uint16_t *X, int64_t M, const int64_t *rows, int64_t nrows,
                    const uint16_t *What, int64_t N, int64_t K, double *Y)
 {
     (void)M;
+    const double *v = bf16_values();
     for (int64_t ri = 0; ri < nrows; ri++) {
         int64_t m = rows ? rows[ri] : ri;
         const uint16_t *x = X + m * K;
@@ -362,7 +377,7 @@ void oracle_matmul(const uint16_t *X, int64_t M, const int64_t *rows, int64_t nr
             const uint16_t *w = What + n * K;
             double acc = 0.0;
             for (int64_t k = 0; k < K; k++)
-                acc += oracle_bf16_value(x[k]) * oracle_bf16_value(w[k]);
+                acc += v[x[k]] * v[w[k]];
             Y[ri * N + n] = acc;
         }
     }
@@ -373,12 +388,13 @@ void oracle_matmul_points(const uint16_t *X, const uint16_t *What, int64_t K,
                           const int64_t *m_idx, const int64_t *n_idx, int64_t npts,
                           double *Y)
 {
+    const double *v = bf16_values();
     for (int64_t i = 0; i < npts; i++) {
         const uint16_t *x = X + m_idx[i] * K;
         const uint16_t *w = What + n_idx[i] * K;
         double acc = 0.0;
         for (int64_t k = 0; k < K; k++)
-            acc += oracle_bf16_value(x[k]) * oracle_bf16_value(w[k]);
+            acc += v[x[k]] * v[w[k]];
         Y[i] = acc;
     }
 }

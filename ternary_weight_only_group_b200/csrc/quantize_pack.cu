@@ -1,0 +1,189 @@
+// quantize_pack.cu -- per-group ternary quantizer and base-3 packer.
+//
+// "precisit/pack-unpack-run", codec.py description: mean-absolute scale
+// rounded to fp16, nearest-even ternary codes, five base-three digits per
+// byte, each group byte-aligned with zero-trit padding.
+//
+// The matrix is treated as a flat run of N*K/G groups (a group never crosses
+// a row because K % G == 0).  Fast path (G = 8 * 2^k, 8 <= G <= 256): a warp
+// covers 32*8/G consecutive groups, G/8 lanes per group, 8 weights per lane
+// from one 16-byte load; the group's max |w| and sum |w| are segmented warp
+// shuffle reductions.  The sum is exact: every |w| within 2^37 of the group
+// maximum fits, together with the total, in the 53-bit binary64 significand,
+// so the shuffle order cannot change it; dividing by G (a power of two) is
+// exact and cvt.rn.f16.f64 rounds once, ties to even.  A group holding a
+// nonzero |w| more than 2^37 below its maximum takes the multi-word exact
+// path instead.  Other G use one thread per group with the multi-word path.
+#include "tq_internal.cuh"
+
+namespace tq {
+
+template <int G>
+__global__ void __launch_bounds__(256) quantize_pack_pow2_kernel(
+    const uint16_t* __restrict__ W, int64_t num_groups, uint8_t* __restrict__ codes,
+    uint16_t* __restrict__ scales, uint32_t* __restrict__ d_err) {
+    constexpr int LPG = G / 8;     // lanes per group
+    constexpr int GPW = 32 / LPG;  // groups per warp pass
+    constexpr int B = bytes_per_group(G);
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % LPG;
+    const int p0 = 8 * sub;  // first weight of this lane inside its group
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    uint32_t err_acc = 0;
+
+    for (int64_t base = warp * GPW; base < num_groups; base += nwarps * GPW) {
+        const int64_t gi = base + lane / LPG;
+        const bool active = gi < num_groups;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (active) v = __ldcs(reinterpret_cast<const uint4*>(W + gi * G + p0));
+        const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+        uint32_t a[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            a[2 * i] = h[i] & 0x7FFFu;
+            a[2 * i + 1] = (h[i] >> 16) & 0x7FFFu;
+        }
+        uint32_t amax = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = max(amax, a[i]);
+        amax = seg_max_u32(amax, LPG);  // NaN/Inf patterns are the largest magnitudes
+
+        // All 32 lanes run every shuffle below; the per-group decisions come after.
+        const uint32_t emax = amax >> 7;
+        const uint32_t thr = emax > 37 ? (emax - 37) << 7 : 0;  // smallest pattern in the window
+        double sum = 0.0;
+        uint32_t outside = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (a[i] >= thr) sum += bf16_normal_mag_to_f64(a[i]);
+            else outside |= a[i];
+        }
+        sum = seg_sum_f64(sum, LPG);
+        outside = seg_or_u32(outside, LPG);
+
+        uint16_t s = 0;
+        uint32_t gerr = 0;
+        bool slow = false;
+        if (amax >= 0x7F80u) {
+            gerr = TQ_DERR_WEIGHT;
+        } else if (amax > kTinyMaxBits) {
+            if (outside) {
+                slow = true;
+            } else {
+                const uint16_t bits = __half_as_ushort(__double2half(sum * (1.0 / G)));
+                if (bits >= 0x7C00u) gerr = TQ_DERR_OVERFLOW;
+                else s = bits;
+            }
+        }
+        if (__any_sync(0xffffffffu, slow)) {
+            if (slow && sub == 0 && active) gerr = exact_group_scale(W + gi * G, G, &s);
+            const int leader = lane - sub;  // same value for every lane of a segment
+            s = (uint16_t)__shfl_sync(0xffffffffu, (uint32_t)s, leader, 32);
+            gerr = __shfl_sync(0xffffffffu, gerr, leader, 32);
+        }
+        if (gerr) s = 0;
+
+        // digits d = t + 1 of this lane's 8 weights, 2 bits each
+        const uint32_t th = trit_threshold(s);
+        uint32_t F = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint32_t hw = (h[i] >> (16 * k)) & 0xFFFFu;
+                const uint32_t d = (a[2 * i + k] > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
+                F |= d << (2 * (2 * i + k));
+            }
+        }
+        uint32_t Fn = __shfl_down_sync(0xffffffffu, F, 1);
+        if (sub == LPG - 1) Fn = 0x5555u;  // positions >= G: padding digit 1
+        const uint32_t D = F | (Fn << 16);  // digits of weights p0 .. p0+15
+
+        if (active) {
+            uint8_t* out = codes + gi * B;
+            for (int q = (p0 + 4) / 5; 5 * q < p0 + 8 && q < B; ++q) {
+                const uint32_t f = D >> (2 * (5 * q - p0));
+                const uint32_t byte = (f & 3u) + 3u * ((f >> 2) & 3u) + 9u * ((f >> 4) & 3u) +
+                                      27u * ((f >> 6) & 3u) + 81u * ((f >> 8) & 3u);
+                out[q] = (uint8_t)byte;
+            }
+            if (sub == 0) {
+                scales[gi] = s;
+                err_acc |= gerr;
+            }
+        }
+    }
+    if (err_acc && d_err) atomicOr(d_err, err_acc);
+}
+
+// Any G: one thread per group, multi-word exact scale.
+__global__ void __launch_bounds__(128) quantize_pack_generic_kernel(
+    const uint16_t* __restrict__ W, int64_t num_groups, int G, uint8_t* __restrict__ codes,
+    uint16_t* __restrict__ scales, uint32_t* __restrict__ d_err) {
+    const int B = bytes_per_group(G);
+    uint32_t err_acc = 0;
+    for (int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < num_groups;
+         gi += (int64_t)gridDim.x * blockDim.x) {
+        const uint16_t* w = W + gi * G;
+        uint16_t s;
+        const uint32_t gerr = exact_group_scale(w, G, &s);
+        err_acc |= gerr;
+        scales[gi] = s;
+        const uint32_t th = trit_threshold(s);
+        uint8_t* out = codes + gi * B;
+        for (int q = 0; q < B; ++q) {
+            uint32_t byte = 0, p3 = 1;
+            for (int i = 0; i < 5; ++i) {
+                const int j = 5 * q + i;
+                uint32_t d = 1;
+                if (j < G) {
+                    const uint32_t hw = w[j];
+                    d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
+                }
+                byte += d * p3;
+                p3 *= 3;
+            }
+            out[q] = (uint8_t)byte;
+        }
+    }
+    if (err_acc && d_err) atomicOr(d_err, err_acc);
+}
+
+static int grid_for(int64_t threads_needed, int block, int sm_count) {
+    int64_t blocks = (threads_needed + block - 1) / block;
+    const int64_t cap = (int64_t)sm_count * 16;
+    if (blocks > cap) blocks = cap;
+    return (int)(blocks < 1 ? 1 : blocks);
+}
+
+cudaError_t launch_quantize_pack(const uint16_t* W, int64_t N, int64_t K, int G, uint8_t* codes,
+                                 uint16_t* scales, uint32_t* d_err, cudaStream_t stream,
+                                 int sm_count) {
+    const int64_t num_groups = N * (K / G);
+    if (num_groups == 0) return cudaSuccess;
+    const int block = 256;
+#define TQ_QP_CASE(GG)                                                                           \
+    case GG: {                                                                                   \
+        const int64_t threads = (num_groups + (32 / (GG / 8)) - 1) / (32 / (GG / 8)) * 32;       \
+        quantize_pack_pow2_kernel<GG><<<grid_for(threads, block, sm_count), block, 0, stream>>>( \
+            W, num_groups, codes, scales, d_err);                                                \
+        return cudaGetLastError();                                                               \
+    }
+    switch (G) {
+        TQ_QP_CASE(8)
+        TQ_QP_CASE(16)
+        TQ_QP_CASE(32)
+        TQ_QP_CASE(64)
+        TQ_QP_CASE(128)
+        TQ_QP_CASE(256)
+        default:
+            break;
+    }
+#undef TQ_QP_CASE
+    quantize_pack_generic_kernel<<<grid_for(num_groups, 128, sm_count), 128, 0, stream>>>(
+        W, num_groups, G, codes, scales, d_err);
+    return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,220 @@
+// tq_abi.cu -- extern "C" entry points of libtq: argument validation and
+// kernel dispatch.  Every check here runs on the host before any launch; a
+// failed check returns a status and enqueues nothing.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "tq_internal.cuh"
+
+namespace tq {
+cudaError_t launch_quantize_pack(const uint16_t* W, int64_t N, int64_t K, int G, uint8_t* codes,
+                                 uint16_t* scales, uint32_t* d_err, cudaStream_t stream,
+                                 int sm_count);
+cudaError_t launch_unpack(const uint8_t* codes, const uint16_t* scales, int64_t N, int64_t K, int G,
+                          uint16_t* out, uint32_t* d_err, cudaStream_t stream, int sm_count);
+cudaError_t launch_gemv_rows(const uint16_t* X, int64_t M, const uint8_t* codes,
+                             const uint16_t* scales, int64_t N, int64_t K, int G, void* Y,
+                             int y_bf16, uint32_t* d_err, cudaStream_t stream, int sm_count,
+                             size_t smem_limit);
+cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes,
+                           const uint16_t* scales, int64_t N, int64_t K, int G, void* Y,
+                           int y_bf16, uint32_t* d_err, cudaStream_t stream, int sm_count,
+                           bool* handled);
+
+namespace {
+
+struct DeviceInfo {
+    int sm_count = 0;
+    int major = 0, minor = 0;
+    size_t smem_optin = 0;
+    bool ok = false;
+};
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_dev_once[kMaxDevices];
+DeviceInfo g_dev[kMaxDevices];
+
+tq_status device_info(const DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return TQ_ERR_CUDA;
+    }
+    std::call_once(g_dev_once[dev], [dev] {
+        DeviceInfo& d = g_dev[dev];
+        int smem = 0;
+        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess) {
+            d.smem_optin = (size_t)smem;
+            d.ok = true;
+        } else {
+            cudaGetLastError();
+        }
+    });
+    const DeviceInfo& d = g_dev[dev];
+    if (!d.ok) return TQ_ERR_CUDA;
+    // The kernels are built for sm_100a only.
+    if (d.major != 10 || d.minor != 0) return TQ_ERR_UNSUPPORTED;
+    *out = &d;
+    return TQ_OK;
+}
+
+bool shape_ok(int64_t N, int64_t K, int G) {
+    if (G < 1 || G > TQ_MAX_G) return false;
+    if (N < 0 || K < 0 || K % G != 0) return false;
+    if (N > 0 && K > (int64_t(1) << 62) / N) return false;
+    return true;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    if (!na || !nb) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+tq_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return TQ_OK;
+    cudaGetLastError();
+    return TQ_ERR_CUDA;
+}
+
+struct MatmulArgs {
+    const void* X;
+    int64_t M;
+    const uint8_t* codes;
+    const void* scales;
+    int64_t N, K;
+    int G;
+    void* Y;
+    tq_out_dtype yt;
+};
+
+tq_status check_matmul(const MatmulArgs& a) {
+    if (!shape_ok(a.N, a.K, a.G) || a.M < 0) return TQ_ERR_INVALID_ARG;
+    if (a.yt != TQ_OUT_F32 && a.yt != TQ_OUT_BF16) return TQ_ERR_INVALID_ARG;
+    if (a.M > 0 && a.K > (int64_t(1) << 62) / a.M) return TQ_ERR_INVALID_ARG;
+    if (a.M > 0 && a.N > (int64_t(1) << 62) / a.M) return TQ_ERR_INVALID_ARG;
+    const size_t cb = tq_codes_bytes(a.N, a.K, a.G), sb = tq_scales_bytes(a.N, a.K, a.G);
+    const size_t xb = (size_t)a.M * (size_t)a.K * 2;
+    const size_t yb = (size_t)a.M * (size_t)a.N * (a.yt == TQ_OUT_F32 ? 4 : 2);
+    if ((xb && !a.X) || (cb && !a.codes) || (sb && !a.scales) || (yb && !a.Y)) return TQ_ERR_INVALID_ARG;
+    if (overlap(a.Y, yb, a.X, xb) || overlap(a.Y, yb, a.codes, cb) || overlap(a.Y, yb, a.scales, sb))
+        return TQ_ERR_INVALID_ARG;
+    if (!aligned(a.X, 16) || !aligned(a.scales, 2) || !aligned(a.Y, a.yt == TQ_OUT_F32 ? 4 : 2))
+        return TQ_ERR_ALIGNMENT;
+    return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" {
+
+size_t tq_codes_bytes(int64_t N, int64_t K, int G) {
+    if (!shape_ok(N, K, G)) return 0;
+    return (size_t)N * (size_t)(K / G) * (size_t)bytes_per_group(G);
+}
+
+size_t tq_scales_bytes(int64_t N, int64_t K, int G) {
+    if (!shape_ok(N, K, G)) return 0;
+    return (size_t)N * (size_t)(K / G) * 2;
+}
+
+size_t tq_workspace_bytes(int64_t M, int64_t N, int64_t K, int G) {
+    (void)M; (void)N; (void)K; (void)G;
+    return 0;
+}
+
+tq_status tq_quantize_pack(const void* W, int64_t N, int64_t K, int G, uint8_t* codes, void* scales,
+                           uint32_t* d_err, tq_stream_t stream) {
+    if (!shape_ok(N, K, G)) return TQ_ERR_INVALID_ARG;
+    const size_t wb = (size_t)N * (size_t)K * 2;
+    const size_t cb = tq_codes_bytes(N, K, G), sb = tq_scales_bytes(N, K, G);
+    if ((wb && !W) || (cb && !codes) || (sb && !scales)) return TQ_ERR_INVALID_ARG;
+    if (overlap(codes, cb, W, wb) || overlap(scales, sb, W, wb) || overlap(codes, cb, scales, sb))
+        return TQ_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(scales, 2)) return TQ_ERR_ALIGNMENT;
+    if (wb == 0) return TQ_OK;
+    const DeviceInfo* d = nullptr;
+    if (tq_status st = device_info(&d)) return st;
+    return from_cuda(launch_quantize_pack(static_cast<const uint16_t*>(W), N, K, G, codes,
+                                          static_cast<uint16_t*>(scales), d_err,
+                                          (cudaStream_t)stream, d->sm_count));
+}
+
+tq_status tq_unpack_bf16(const uint8_t* codes, const void* scales, int64_t N, int64_t K, int G,
+                         void* W_out, uint32_t* d_err, tq_stream_t stream) {
+    if (!shape_ok(N, K, G)) return TQ_ERR_INVALID_ARG;
+    const size_t wb = (size_t)N * (size_t)K * 2;
+    const size_t cb = tq_codes_bytes(N, K, G), sb = tq_scales_bytes(N, K, G);
+    if ((wb && !W_out) || (cb && !codes) || (sb && !scales)) return TQ_ERR_INVALID_ARG;
+    if (overlap(W_out, wb, codes, cb) || overlap(W_out, wb, scales, sb)) return TQ_ERR_INVALID_ARG;
+    if (!aligned(W_out, 16) || !aligned(scales, 2)) return TQ_ERR_ALIGNMENT;
+    if (wb == 0) return TQ_OK;
+    const DeviceInfo* d = nullptr;
+    if (tq_status st = device_info(&d)) return st;
+    return from_cuda(launch_unpack(codes, static_cast<const uint16_t*>(scales), N, K, G,
+                                   static_cast<uint16_t*>(W_out), d_err, (cudaStream_t)stream,
+                                   d->sm_count));
+}
+
+tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* scales, int64_t N,
+                  int64_t K, int G, void* Y, tq_out_dtype yt, void* workspace, size_t ws_bytes,
+                  uint32_t* d_err, tq_stream_t stream) {
+    (void)workspace; (void)ws_bytes;
+    const MatmulArgs a{X, M, codes, scales, N, K, G, Y, yt};
+    if (tq_status st = check_matmul(a)) return st;
+    if (M == 0 || N == 0) return TQ_OK;
+    if (K == 0) return TQ_ERR_UNSUPPORTED;
+    const DeviceInfo* d = nullptr;
+    if (tq_status st = device_info(&d)) return st;
+    cudaError_t e = launch_gemv_rows(static_cast<const uint16_t*>(X), M, codes,
+                                     static_cast<const uint16_t*>(scales), N, K, G, Y,
+                                     yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count,
+                                     d->smem_optin);
+    if (e == cudaErrorInvalidValue) return TQ_ERR_UNSUPPORTED;
+    return from_cuda(e);
+}
+
+tq_status tq_gemm(const void* X, int64_t M, const uint8_t* codes, const void* scales, int64_t N,
+                  int64_t K, int G, void* Y, tq_out_dtype yt, void* workspace, size_t ws_bytes,
+                  uint32_t* d_err, tq_stream_t stream) {
+    (void)workspace; (void)ws_bytes;
+    const MatmulArgs a{X, M, codes, scales, N, K, G, Y, yt};
+    if (tq_status st = check_matmul(a)) return st;
+    if (M == 0 || N == 0) return TQ_OK;
+    if (K == 0) return TQ_ERR_UNSUPPORTED;
+    const DeviceInfo* d = nullptr;
+    if (tq_status st = device_info(&d)) return st;
+    bool handled = false;
+    cudaError_t e = launch_gemm_tc(static_cast<const uint16_t*>(X), M, codes,
+                                   static_cast<const uint16_t*>(scales), N, K, G, Y,
+                                   yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count,
+                                   &handled);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (!handled) return TQ_ERR_UNSUPPORTED;
+    return TQ_OK;
+}
+
+const char* tq_status_string(tq_status s) {
+    switch (s) {
+        case TQ_OK: return "TQ_OK";
+        case TQ_ERR_INVALID_ARG: return "TQ_ERR_INVALID_ARG";
+        case TQ_ERR_ALIGNMENT: return "TQ_ERR_ALIGNMENT";
+        case TQ_ERR_UNSUPPORTED: return "TQ_ERR_UNSUPPORTED";
+        case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+    }
+    return "TQ_ERR_UNKNOWN";
+}
+
+const char* tq_version(void) { return "libtq 0.1 sm_100a"; }
+
+}  // extern "C"

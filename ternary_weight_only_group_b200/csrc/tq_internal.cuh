@@ -1,0 +1,146 @@
+// tq_internal.cuh -- device helpers shared by the libtq kernels (CUDA side only).
+//
+// Format facts used here come from "precisit/pack-unpack-run" (codec.py
+// description): one binary16 scale per group of G columns, five base-3 digits
+// per byte, each group byte-aligned, digit d = t + 1, first weight = least
+// significant digit, padding digit 1, bytes >= 243 invalid.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+__host__ __device__ constexpr int bytes_per_group(int G) { return (G + 4) / 5; }
+
+// Byte of a group made only of zero trits: 1 + 3 + 9 + 27 + 81.
+constexpr uint32_t kZeroByte = 121;
+// bf16 bit pattern written for a rejected group.
+constexpr uint16_t kBf16NaN = 0x7FC0;
+// Largest bf16 magnitude pattern whose group mean is certain to round to +0:
+// max|w| <= 2^-25 implies mean <= 2^-25, the tie below the smallest binary16
+// subnormal, which rounds to even (+0).
+constexpr uint32_t kTinyMaxBits = 0x3300;  // bf16 2^-25
+// bf16 pattern of 2^32: a magnitude at or above it makes any group mean
+// (G <= 4096) exceed 65520 and overflow binary16.
+constexpr uint32_t kHugeBits = 0x4F80;
+
+__device__ __forceinline__ uint32_t seg_max_u32(uint32_t v, int width) {
+    for (int off = width >> 1; off > 0; off >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
+}
+__device__ __forceinline__ uint32_t seg_or_u32(uint32_t v, int width) {
+    for (int off = width >> 1; off > 0; off >>= 1) v |= __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+__device__ __forceinline__ double seg_sum_f64(double v, int width) {
+    for (int off = width >> 1; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+// Exact binary64 value of a normal bf16 magnitude pattern a (1 <= exponent <= 254):
+// same exponent, the 7 fraction bits moved to the top of the 52-bit fraction.
+__device__ __forceinline__ double bf16_normal_mag_to_f64(uint32_t a) {
+    return __hiloint2double((int)((a << 13) + 0x38000000u), 0);
+}
+
+// RNE bf16 of a binary16 scale, as the decoded magnitude of a nonzero trit.
+__device__ __forceinline__ uint16_t scale_to_bf16_bits(uint16_t s) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(__half2float(__ushort_as_half(s))));
+}
+
+// True for a stored scale the decoder must reject: sign bit set, or NaN/Inf.
+__device__ __forceinline__ bool scale_is_bad(uint32_t s) {
+    return (s & 0x8000u) != 0 || (s & 0x7C00u) == 0x7C00u;
+}
+
+// Trit threshold: |w| > s/2  <=>  (|w| bf16 pattern) > (binary32 pattern of s/2) >> 16.
+// Both sides are non-negative floats, whose order is the order of their bit
+// patterns; a bf16 pattern shifted left by 16 is the binary32 of the same value.
+// A zero scale gives a threshold no magnitude exceeds.
+__device__ __forceinline__ uint32_t trit_threshold(uint16_t s) {
+    if (s == 0) return 0xFFFFu;
+    float half_s = __half2float(__ushort_as_half(s)) * 0.5f;  // exact
+    return __float_as_uint(half_s) >> 16;
+}
+
+// ---------------------------------------------------------------------------
+// Exact group scale by multi-word integer arithmetic (any G <= TQ_MAX_G, any
+// exponent spread).  The sum of |w| is held exactly in units of 2^-133 (the
+// smallest bf16 subnormal); it is divided by G and rounded once to binary16,
+// ties to even.  Returns TQ_DERR_* bits; *s_out is +0 on error.
+// ---------------------------------------------------------------------------
+static __device__ __noinline__ uint32_t exact_group_scale(const uint16_t* __restrict__ w, int G,
+                                                    uint16_t* s_out) {
+    *s_out = 0;
+    uint32_t amax = 0;
+    for (int j = 0; j < G; ++j) amax = max(amax, (uint32_t)(w[j] & 0x7FFF));
+    if (amax >= 0x7F80u) return TQ_DERR_WEIGHT;
+    if (amax >= kHugeBits) return TQ_DERR_OVERFLOW;
+    if (amax <= kTinyMaxBits) return 0;
+    // Every magnitude is below 2^32 = 2^165 units; G <= 2^12 of them fit in 6 words.
+    uint32_t L[6] = {0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < G; ++j) {
+        uint32_t a = w[j] & 0x7FFF;
+        uint32_t e = a >> 7;
+        uint32_t m = (a & 0x7F) | (e ? 0x80u : 0u);
+        uint32_t sh = e ? e - 1 : 0;
+        uint32_t limb = sh >> 5, bit = sh & 31;
+        uint64_t v = (uint64_t)m << bit;
+        uint64_t carry = 0;
+        for (uint32_t i = limb; i < 6; ++i) {
+            uint64_t t = (uint64_t)L[i] + (v & 0xFFFFFFFFull) + carry;
+            L[i] = (uint32_t)t;
+            carry = t >> 32;
+            v >>= 32;
+            if (v == 0 && carry == 0) break;
+        }
+    }
+    uint32_t Q[6];
+    uint64_t r = 0;
+    for (int i = 5; i >= 0; --i) {
+        uint64_t cur = (r << 32) | L[i];
+        Q[i] = (uint32_t)(cur / (uint32_t)G);
+        r = cur % (uint32_t)G;
+    }
+    int P = -1;
+    for (int i = 5; i >= 0; --i)
+        if (Q[i]) { P = i * 32 + 31 - __clz(Q[i]); break; }
+    if (P < 0) return 0;
+    int E = P - 133;  // floor(log2(mean))
+    if (E > 15) return TQ_DERR_OVERFLOW;
+    int Eeff = E < -14 ? -14 : E;
+    int k = Eeff + 123;  // one binary16 ulp is 2^k units
+    auto bit_of = [&](int b) -> uint32_t { return (Q[b >> 5] >> (b & 31)) & 1u; };
+    uint32_t mant = 0;
+    for (int i = 0; i < 12; ++i) mant |= bit_of(k + i) << i;
+    uint32_t half = bit_of(k - 1);
+    bool rest = (r != 0);
+    for (int b = 0; b < k - 1 && !rest; ++b) rest = bit_of(b) != 0;
+    uint32_t up = half && (rest || (mant & 1u));
+    uint32_t bits = ((uint32_t)(Eeff + 14) << 10) + mant + up;
+    if (bits >= 0x7C00u) return TQ_DERR_OVERFLOW;
+    *s_out = (uint16_t)bits;
+    return 0;
+}
+
+// Decode table entry for a byte: its five digits, 2 bits each (digit i at
+// bits 2i..2i+1), with bit 15 set for an invalid byte (>= 243).
+__device__ __forceinline__ uint32_t byte_digit_pattern(uint32_t b) {
+    if (b >= 243) return 0x8000u;
+    uint32_t p = 0;
+    for (int i = 0; i < 5; ++i) {
+        p |= (b % 3) << (2 * i);
+        b /= 3;
+    }
+    return p;
+}
+
+// Digit pattern of a canonical last byte: digits >= `real` are all 1.
+__host__ __device__ constexpr uint32_t padding_mask(int real) { return 0x3FFu & ~((1u << (2 * real)) - 1u); }
+__host__ __device__ constexpr uint32_t padding_ones(int real) { return 0x155u & padding_mask(real); }
+
+}  // namespace tq

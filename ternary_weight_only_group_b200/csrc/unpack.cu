@@ -1,0 +1,154 @@
+// unpack.cu -- base-3 decoder to bf16.
+//
+// "precisit/pack-unpack-run", codec.py description: decoding; values 243
+// through 255 are invalid; the decoder restores the weights as bf16.  A zero
+// stored scale produces a zero group (the paragraph after it).
+//
+// Fast path (G = 8 * 2^k, 8 <= G <= 256): G/8 lanes per group, each lane
+// writes 8 consecutive bf16 with one 16-byte store.  The lanes of a group
+// validate the bytes that start in their range (the union is every byte of
+// the group), OR the verdict across the segment, and a rejected group is
+// written as bf16 NaN.  Digits come from a 256-entry shared-memory table.
+#include "tq_internal.cuh"
+
+namespace tq {
+
+template <int G>
+__global__ void __launch_bounds__(256) unpack_pow2_kernel(
+    const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales, int64_t num_groups,
+    uint16_t* __restrict__ out, uint32_t* __restrict__ d_err) {
+    constexpr int LPG = G / 8;
+    constexpr int GPW = 32 / LPG;
+    constexpr int B = bytes_per_group(G);
+    constexpr int REAL = G - 5 * (B - 1);  // real digits in the last byte (1..5)
+    __shared__ uint16_t lut[256];
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) lut[b] = (uint16_t)byte_digit_pattern(b);
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % LPG;
+    const int p0 = 8 * sub;
+    const int q_first = p0 / 5;      // byte holding weight p0
+    const int r_first = p0 - 5 * q_first;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    uint32_t err_acc = 0;
+
+    for (int64_t base = warp * GPW; base < num_groups; base += nwarps * GPW) {
+        const int64_t gi = base + lane / LPG;
+        const bool active = gi < num_groups;
+        // weights p0..p0+7 lie in bytes q_first .. q_first+2 (at most three)
+        uint32_t pat[3] = {0x155u, 0x155u, 0x155u};
+        uint32_t s = 0;
+        if (active) {
+            const uint8_t* in = codes + gi * B;
+#pragma unroll
+            for (int t = 0; t < 3; ++t)
+                if (q_first + t < B) pat[t] = lut[__ldcs(in + q_first + t)];
+            s = __ldg(scales + gi);
+        }
+        // validation of the bytes starting in [p0, p0+8)
+        uint32_t bad = 0;
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+            const int q = q_first + t;
+            if (5 * q >= p0 && 5 * q < p0 + 8 && q < B) {
+                if (pat[t] & 0x8000u) bad |= TQ_DERR_BYTE;
+                else if (q == B - 1 && (pat[t] & padding_mask(REAL)) != padding_ones(REAL))
+                    bad |= TQ_DERR_PADDING;
+            }
+        }
+        if (sub == 0 && scale_is_bad(s)) bad |= TQ_DERR_SCALE;
+        bad = seg_or_u32(bad, LPG);
+        if (!active) bad = 0;
+
+        const uint32_t mag = (s == 0) ? 0u : scale_to_bf16_bits((uint16_t)s);
+        uint32_t w[8];
+        int t = 0, r = r_first;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t d = (pat[t] >> (2 * r)) & 3u;
+            w[i] = (d == 1u || mag == 0u) ? 0u : (mag | (d == 0u ? 0x8000u : 0u));
+            if (++r == 5) { r = 0; ++t; }
+        }
+        if (bad) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = kBf16NaN;
+        }
+        if (active) {
+            uint4 o = make_uint4(w[0] | (w[1] << 16), w[2] | (w[3] << 16), w[4] | (w[5] << 16),
+                                 w[6] | (w[7] << 16));
+            __stcs(reinterpret_cast<uint4*>(out + gi * G + p0), o);
+            if (sub == 0) err_acc |= bad;
+        }
+    }
+    if (err_acc && d_err) atomicOr(d_err, err_acc);
+}
+
+// Any G: one thread per group.
+__global__ void __launch_bounds__(128) unpack_generic_kernel(
+    const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales, int64_t num_groups,
+    int G, uint16_t* __restrict__ out, uint32_t* __restrict__ d_err) {
+    const int B = bytes_per_group(G);
+    const int real = G - 5 * (B - 1);
+    uint32_t err_acc = 0;
+    for (int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < num_groups;
+         gi += (int64_t)gridDim.x * blockDim.x) {
+        const uint8_t* in = codes + gi * B;
+        const uint32_t s = scales[gi];
+        uint32_t bad = scale_is_bad(s) ? TQ_DERR_SCALE : 0u;
+        for (int q = 0; q < B; ++q) {
+            const uint32_t p = byte_digit_pattern(in[q]);
+            if (p & 0x8000u) bad |= TQ_DERR_BYTE;
+            else if (q == B - 1 && (p & padding_mask(real)) != padding_ones(real)) bad |= TQ_DERR_PADDING;
+        }
+        const uint32_t mag = (s == 0) ? 0u : scale_to_bf16_bits((uint16_t)s);
+        uint16_t* o = out + gi * G;
+        for (int j = 0; j < G; ++j) {
+            uint32_t v;
+            if (bad) {
+                v = kBf16NaN;
+            } else {
+                const uint32_t d = (byte_digit_pattern(in[j / 5]) >> (2 * (j % 5))) & 3u;
+                v = (d == 1u || mag == 0u) ? 0u : (mag | (d == 0u ? 0x8000u : 0u));
+            }
+            o[j] = (uint16_t)v;
+        }
+        err_acc |= bad;
+    }
+    if (err_acc && d_err) atomicOr(d_err, err_acc);
+}
+
+cudaError_t launch_unpack(const uint8_t* codes, const uint16_t* scales, int64_t N, int64_t K, int G,
+                          uint16_t* out, uint32_t* d_err, cudaStream_t stream, int sm_count) {
+    const int64_t num_groups = N * (K / G);
+    if (num_groups == 0) return cudaSuccess;
+    auto grid = [&](int64_t threads, int block) {
+        int64_t b = (threads + block - 1) / block;
+        const int64_t cap = (int64_t)sm_count * 16;
+        return (int)(b > cap ? cap : (b < 1 ? 1 : b));
+    };
+#define TQ_UP_CASE(GG)                                                                          \
+    case GG: {                                                                                  \
+        const int64_t threads = (num_groups + (32 / (GG / 8)) - 1) / (32 / (GG / 8)) * 32;      \
+        unpack_pow2_kernel<GG><<<grid(threads, 256), 256, 0, stream>>>(codes, scales, num_groups, \
+                                                                      out, d_err);              \
+        return cudaGetLastError();                                                              \
+    }
+    switch (G) {
+        TQ_UP_CASE(8)
+        TQ_UP_CASE(16)
+        TQ_UP_CASE(32)
+        TQ_UP_CASE(64)
+        TQ_UP_CASE(128)
+        TQ_UP_CASE(256)
+        default:
+            break;
+    }
+#undef TQ_UP_CASE
+    unpack_generic_kernel<<<grid(num_groups, 128), 128, 0, stream>>>(codes, scales, num_groups, G,
+                                                                      out, d_err);
+    return cudaGetLastError();
+}
+
+}  // namespace tq

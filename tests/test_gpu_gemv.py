@@ -1,0 +1,85 @@
+"""GPU parity of tq_gemv (decode matmul, CUDA cores) against the oracle.
+
+fp32 outputs: max_n |gpu - oracle| <= 1e-3 * max_n |oracle| per output row.
+bf16 outputs: |gpu - oracle| <= 2e-2 + 2e-2 |oracle|.  NaN rows (rejected
+groups) must coincide exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+import ternary_weight_only_group_b200 as tq
+from tests.parity import (assert_close_bf16, assert_rows_close_f32, to_dev_bf16, to_dev_f16,
+                          to_dev_u8, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def run(fn, X, codes, scales, N, K, G, out_dtype):
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Y = fn(to_dev_bf16(X), to_dev_u8(codes), to_dev_f16(scales), N, K, G, out_dtype=out_dtype, d_err=err)
+    torch.cuda.synchronize()
+    return to_f64(Y), int(err.item())
+
+
+def check(X, W, G, fn=tq.gemv, dtypes=(torch.float32, torch.bfloat16), codes=None, scales=None):
+    N, K = W.shape
+    if codes is None:
+        codes, scales, _ = oracle.quantize_pack(W, G)
+    ref = oracle.linear(X, codes, scales, N, K, G)
+    _, e_ref = oracle.unpack_bf16(codes, scales, N, K, G)
+    for dt in dtypes:
+        Y, e = run(fn, X, codes, scales, N, K, G, dt)
+        if dt == torch.float32:
+            assert_rows_close_f32(Y, ref)
+        else:
+            assert_close_bf16(Y, ref)
+        assert e == e_ref
+    return ref
+
+
+def test_tiny_workload():
+    W, X, G = synthetic.tiny_case()
+    ref = check(X, W, G)
+    assert np.all(ref[:, :4] == 0)
+
+
+@pytest.mark.parametrize("G", [64, 128])
+@pytest.mark.parametrize("name", ["gate", "up", "down"])
+def test_ffn_decode_full_size(name, G):
+    W = synthetic.ffn_matrix(name)
+    X = synthetic.activations(1, W.shape[1])
+    check(X, W, G)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 8, 9, 16, 33, 64])
+@pytest.mark.parametrize("name", ["q", "gate", "down"])
+def test_msweep_shapes(name, M):
+    W = synthetic.msweep_matrix(name)
+    X = synthetic.activations(M, W.shape[1])
+    check(X, W, 128, dtypes=(torch.float32,))
+
+
+@pytest.mark.parametrize("G", [1, 5, 8, 40, 64, 100, 128, 256, 4096])
+def test_group_sizes_and_ragged_rows(G):
+    K = G * max(2, 1024 // G)
+    N = 77
+    W = synthetic.weights(N, K, index=G + 50, outlier_frac=1e-3)
+    X = synthetic.activations(3, K)
+    check(X, W, G)
+
+
+def test_rejected_groups_give_nan_rows():
+    G, N, K = 64, 40, 512
+    W = synthetic.weights(N, K, index=12)
+    codes, scales, _ = oracle.quantize_pack(W, G)
+    codes[3, 2, 4] = 250          # invalid byte
+    codes[7, 1, 12] = 0           # padding digit 0
+    scales[11, 5] = 0x7C00        # Inf scale
+    scales[13, 0] = 0x8001        # negative scale
+    scales[17, 3] = 0             # zero group: finite result
+    X = synthetic.activations(2, K)
+    ref = check(X, W, G, codes=codes, scales=scales)
+    assert np.all(np.isnan(ref[:, [3, 7, 11, 13]])) and np.all(np.isfinite(ref[:, 17]))
