@@ -1,0 +1,525 @@
+#!/usr/bin/env python
+"""Benchmark of the ternary weight-only grouped linear layer on B200.
+
+Headline (`value`): decode GEMV throughput in GB/s of algorithmic HBM bytes
+(packed codes + fp16 scales + bf16 activations + bf16 outputs) on the
+Qwen3.5-0.8B-shaped FFN projections (gate/up 3584 x 1024, down 1024 x 3584),
+G in {64, 128}, M = 1.  One step = a decode token through a 48-layer stack of
+those three projections for both group sizes (288 tq_gemv launches replayed
+from one CUDA graph).  The stack's working set (232 MB) exceeds the 126 MB L2,
+so no step finds its weights in cache.
+
+The other rows of the hot path are measured in the same run and reported in
+their own keys: bulk quantize+pack and unpack over the 72-matrix, 24-layer FFN
+stack (packed-byte GB/s both ways), a single large streaming GEMV, and the
+tensor-core prefill GEMM (M=4096, 4096->14336 and 14336->4096, TFLOP/s).
+
+Multi-GPU: one process per GPU (torchrun), every rank runs its own replica
+(weak scaling, no data-path collective); time = max over ranks.
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ternary x bf16 GEMV HBM GB/s (% of peak); prefill GEMM TFLOP/s; pack GB/s"
+FFN = {"gate": (3584, 1024), "up": (3584, 1024), "down": (1024, 3584)}
+GROUPS = (64, 128)
+LAYERS = 48
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def packed_bytes(N, K, G):
+    return N * (K // G) * ((G + 4) // 5) + N * (K // G) * 2
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- helpers
+
+def dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(fn, steps, warmup, world, stream=None):
+    """W untimed + K timed calls of fn, barrier + synchronize on both sides,
+    CUDA events on the launching stream; returns max-over-ranks ms."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    s = stream or torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed")
+    e0.record(s)
+    for _ in range(steps):
+        fn()
+    e1.record(s)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    return max_over_ranks(ms, world)
+
+
+def device_weights(N, K, seed, outliers=True):
+    """Seeded synthetic bf16 weights ~ N(0, 0.02), 0.1% of entries x10, made on the device."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    w = torch.randn((N, K), generator=g, device="cuda", dtype=torch.float32) * 0.02
+    if outliers:
+        mask = torch.rand((N, K), generator=g, device="cuda") < 1e-3
+        w = torch.where(mask, w * 10.0, w)
+    return w.to(torch.bfloat16)
+
+
+def device_acts(M, K, seed):
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    return torch.randn((M, K), generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)
+
+
+# --------------------------------------------------------------------- our arm
+
+def build_decode_stack(tq, layers):
+    """Packed weights of `layers` x (gate, up, down) for each G, plus one X
+    buffer and one Y buffer sliced per launch (so a whole step's inputs and
+    outputs are single contiguous transfers for the end-to-end measurement)."""
+    import torch
+    calls = []
+    x_elems = y_elems = 0
+    for G in GROUPS:
+        for l in range(layers):
+            for name, (N, K) in FFN.items():
+                calls.append((G, l, name, N, K, x_elems, y_elems))
+                x_elems += K
+                y_elems += N
+    packs = {}
+    for G in GROUPS:
+        for l in range(layers):
+            for i, (name, (N, K)) in enumerate(FFN.items()):
+                W = device_weights(N, K, seed=1000 + 3 * l + i)
+                packs[(G, l, name)] = tq.quantize_pack(W, G)
+                del W
+    X = device_acts(1, x_elems, seed=2001).view(-1)
+    Y = torch.empty(y_elems, dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    return calls, packs, X, Y
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import ternary_weight_only_group_b200 as tq
+    from ternary_weight_only_group_b200 import _build
+    if not _build.up_to_date():
+        raise RuntimeError("libtq.so is missing or stale; run __graft_entry__.build() first")
+    torch.cuda.set_device(local)
+    peaks = load_peaks()
+    K_steps, W_steps = args.steps, args.warmup
+
+    calls, packs, X, Y = build_decode_stack(tq, LAYERS)
+    step_bytes = 0
+    for (G, l, name, N, K, xo, yo) in calls:
+        step_bytes += packed_bytes(N, K, G) + 2 * K + 2 * N
+
+    def step_kernels():
+        for (G, l, name, N, K, xo, yo) in calls:
+            codes, scales = packs[(G, l, name)]
+            tq.gemv(X[xo:xo + K].view(1, K), codes, scales, N, K, G,
+                    out=Y[yo:yo + N].view(1, N))
+
+    # warm once outside capture (sets kernel attributes), then capture one step
+    step_kernels()
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=cap, capture_error_mode="relaxed"):
+        step_kernels()
+    torch.cuda.synchronize()
+
+    # end-to-end variant: pinned host X in, kernels, pinned host Y out
+    X_host = torch.empty(X.numel(), dtype=torch.bfloat16, pin_memory=True)
+    X_host.copy_(X.cpu())
+    Y_host = torch.empty(Y.numel(), dtype=torch.bfloat16, pin_memory=True)
+    graph_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_e2e, stream=cap, capture_error_mode="relaxed"):
+        X.copy_(X_host, non_blocking=True)
+        step_kernels()
+        Y_host.copy_(Y, non_blocking=True)
+    torch.cuda.synchronize()
+
+    launches_per_step = len(calls)
+    results = {}
+    with ClockSampler(local) as clocks:
+        ms = timed(graph.replay, K_steps, W_steps, world)
+        ms_e2e = timed(graph_e2e.replay, K_steps, W_steps, world)
+        results["stream"] = bench_gemv_stream(tq, args, world, peaks)
+        results["pack"], results["unpack"] = bench_bulk_codec(tq, args, world, peaks)
+        results["prefill"] = bench_prefill(tq, args, world, peaks)
+    clk = clocks.summary()
+
+    ms_step = ms / K_steps
+    value = world * step_bytes * K_steps / (ms * 1e-3) / 1e9
+    e2e = world * step_bytes * K_steps / (ms_e2e * 1e-3) / 1e9
+    per_launch_us = ms_step * 1e3 / launches_per_step
+    avg_bytes = step_bytes / launches_per_step
+    achieved = avg_bytes / (per_launch_us * 1e-6) / 1e9
+    if rank != 0:
+        return
+    cpu = cpu_baseline(args)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K_steps,
+        "warmup": W_steps,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": "decode GEMV, M=1, Qwen3.5-0.8B-shaped FFN gate/up 3584x1024 and "
+                        "down 1024x3584, G in {64,128}; one step = 48 layers x 3 projections "
+                        "x 2 group sizes = 288 tq_gemv launches from one CUDA graph",
+            "layers": LAYERS, "group_sizes": list(GROUPS), "M": 1, "out_dtype": "bf16",
+            "l2": f"inputs larger than L2: {step_bytes / 1e6:.1f} MB per step vs 126 MB L2",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "gemv_row_kernel<1>",
+            "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "peak_source": peaks["source"],
+            "per_launch_us": round(per_launch_us, 3),
+            "bytes_per_launch": round(avg_bytes, 1),
+            "traffic": None,
+        },
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2},
+        "gpu_launches": launches_per_step * K_steps * 2 + sum(
+            r.get("launches", 0) for r in results.values() if isinstance(r, dict)),
+        "clocks": clk,
+        "gemv_stream": results["stream"],
+        "pack": results["pack"],
+        "unpack": results["unpack"],
+        "prefill_gemm": results["prefill"],
+    }
+    print(json.dumps(line), flush=True)
+
+
+def bench_gemv_stream(tq, args, world, peaks):
+    """One GEMV over the 24-layer gate/up stack as a single [172032 x 1024]
+    matrix (G=128, M=1): the kernel's streaming rate without launch gaps."""
+    import torch
+    N, K, G = 48 * 3584, 1024, 128
+    W = device_weights(N, K, seed=77)
+    codes, scales = tq.quantize_pack(W, G)
+    del W
+    X = device_acts(1, K, seed=78)
+    Y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+    reps = max(5, args.steps)
+    ms = timed(lambda: tq.gemv(X, codes, scales, N, K, G, out=Y), reps, max(3, args.warmup), world)
+    byts = packed_bytes(N, K, G) + 2 * K + 2 * N
+    gbs = byts * reps / (ms * 1e-3) / 1e9
+    return {"shape": [N, K], "G": G, "us": round(ms * 1e3 / reps, 2), "GB/s": round(gbs, 1),
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": reps,
+            "note": "same kernel as the headline on one large matrix (inputs 36 MB, L2-resident "
+                    "after the first pass; upper bound on the per-launch rate)"}
+
+
+def bench_bulk_codec(tq, args, world, peaks):
+    """Quantize+pack and unpack over the 72-matrix FFN stack (24 layers), as two
+    launches per direction: gate/up stacked [172032 x 1024] and downs [24576 x 3584]."""
+    import torch
+    shapes = [(48 * 3584, 1024), (24 * 1024, 3584)]
+    out_pack, out_unpack = {}, {}
+    for G in GROUPS:
+        mats = [device_weights(N, K, seed=500 + i, outliers=False) for i, (N, K) in enumerate(shapes)]
+        packed = [tq.quantize_pack(W, G) for W in mats]
+        outs = [torch.empty_like(W) for W in mats]
+        reps = max(3, args.steps // 4)
+
+        def do_pack():  # into preallocated outputs, through the C ABI
+            st = torch.cuda.current_stream().cuda_stream
+            for W, (c, s) in zip(mats, packed):
+                rc = tq.lib().tq_quantize_pack(W.data_ptr(), W.shape[0], W.shape[1], G,
+                                               c.data_ptr(), s.data_ptr(), None, st)
+                if rc != tq.TQ_OK:
+                    raise tq.TQError(rc, "tq_quantize_pack")
+
+        def do_unpack():
+            for (c, s), o in zip(packed, outs):
+                tq.unpack_bf16(c, s, o.shape[0], o.shape[1], G, out=o)
+
+        ms_p = timed(do_pack, reps, max(3, args.warmup), world)
+        ms_u = timed(do_unpack, reps, max(3, args.warmup), world)
+        wbytes = sum(2 * N * K for N, K in shapes)
+        pbytes = sum(packed_bytes(N, K, G) for N, K in shapes)
+        for d, ms in ((out_pack, ms_p), (out_unpack, ms_u)):
+            sec = ms * 1e-3 / reps
+            d[f"G{G}"] = {"us": round(sec * 1e6, 1),
+                          "packed_GB/s": round(pbytes / sec / 1e9, 1),
+                          "total_GB/s": round((wbytes + pbytes) / sec / 1e9, 1),
+                          "frac": round((wbytes + pbytes) / sec / 1e9 / peaks["hbm_gbs"], 4),
+                          "launches": 2 * reps}
+        del mats, packed, outs
+        torch.cuda.empty_cache()
+    return out_pack, out_unpack
+
+
+def bench_prefill(tq, args, world, peaks):
+    import torch
+    M, G = 4096, 128
+    res = {}
+    for name, (N, K) in (("up", (14336, 4096)), ("down", (4096, 14336))):
+        W = device_weights(N, K, seed=900 + len(res), outliers=False)
+        codes, scales = tq.quantize_pack(W, G)
+        del W
+        X = device_acts(M, K, seed=950 + len(res))
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        try:
+            tq.gemm(X, codes, scales, N, K, G, out=Y)
+        except tq.TQError as e:
+            res[name] = {"unavailable": str(e)}
+            continue
+        reps = max(3, args.steps // 4)
+        ms = timed(lambda: tq.gemm(X, codes, scales, N, K, G, out=Y), reps, max(3, args.warmup), world)
+        tflops = 2.0 * M * N * K * reps / (ms * 1e-3) / 1e12
+        res[name] = {"M": M, "N": N, "K": K, "G": G, "us": round(ms * 1e3 / reps, 1),
+                     "TFLOP/s": round(tflops, 1), "frac": round(tflops / peaks["bf16_tflops"], 4),
+                     "launches": reps}
+    return res
+
+
+# --------------------------------------------------------------------- oracle (CPU)
+
+_ORACLE_MATS = None
+
+
+def oracle_mats():
+    """Layer-0 gate, up and down projections packed by the oracle for G=64
+    and G=128, with their M=1 activations (prepared outside any timing)."""
+    global _ORACLE_MATS
+    if _ORACLE_MATS is None:
+        import oracle
+        import synthetic
+        mats = []
+        for G in GROUPS:
+            for name in ("gate", "up", "down"):
+                W = synthetic.ffn_matrix(name)
+                N, K = W.shape
+                codes, scales, _ = oracle.quantize_pack(W, G)
+                mats.append((synthetic.activations(1, K), codes, scales, N, K, G))
+        _ORACLE_MATS = mats
+    return _ORACLE_MATS
+
+
+def oracle_sample_step():
+    """One bounded sample of the decode workload on the CPU oracle: decode
+    GEMV (decode to bf16 + binary64 matmul) of the layer-0 gate, up and down
+    projections for G=64 and G=128 at M=1.  Returns the algorithmic bytes."""
+    import oracle
+    nbytes = 0
+    for X, codes, scales, N, K, G in oracle_mats():
+        oracle.linear(X, codes, scales, N, K, G)
+        nbytes += packed_bytes(N, K, G) + 2 * K + 2 * N
+    return nbytes
+
+
+def cpu_baseline(args, budget_s=10.0):
+    """The oracle as it stands, single-threaded C, timed on this host on a
+    bounded sample: repeated decode GEMVs of the layer-0 projections."""
+    oracle_mats()
+    t0 = time.perf_counter()
+    nbytes = reps = 0
+    while True:
+        nbytes += oracle_sample_step()
+        reps += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    sec = time.perf_counter() - t0
+    return {"value": round(nbytes / sec / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} passes of the decode GEMV (decode to bf16 + binary64 matmul) over "
+                      f"layer-0 gate/up/down for G=64 and G=128, M=1, {sec:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    t = []
+    nbytes = 0
+    oracle_mats()
+    for _ in range(args.warmup):
+        oracle_sample_step()
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        nbytes = oracle_sample_step()
+        t.append(time.perf_counter() - t0)
+    total = sum(t)
+    value = nbytes * len(t) / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / len(t), 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "decode GEMV, M=1, Qwen3.5-0.8B-shaped FFN gate/up 3584x1024 and "
+                               "down 1024x3584, G in {64,128}; each step a bounded sample: layer 0's "
+                               "three projections for both G (decode to bf16 + binary64 matmul)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "layer-0 gate/up/down, G=64 and 128, M=1, per step"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    ap.add_argument("--only", choices=["stream", "codec", "prefill"], default=None,
+                    help="run one sub-benchmark alone and print its result (profiling aid)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":  # CPU only: rank 0 runs, the others exit without work
+        run_reference(args, int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    rank, world, local = dist_setup(args)
+    try:
+        if args.only:
+            import torch
+            import ternary_weight_only_group_b200 as tq
+            torch.cuda.set_device(local)
+            peaks = load_peaks()
+            fn = {"stream": bench_gemv_stream, "codec": bench_bulk_codec, "prefill": bench_prefill}
+            res = fn[args.only](tq, args, world, peaks)
+            if rank == 0:
+                print(json.dumps({"only": args.only, "result": res}), flush=True)
+            return
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

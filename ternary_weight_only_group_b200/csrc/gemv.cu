@@ -10,6 +10,8 @@
 // l, l+32, ...; each byte contributes its five trits against the activations
 // staged in shared memory as bf16.  A row whose codes or scales fail
 // validation produces NaN.
+#include <atomic>
+
 #include "tq_internal.cuh"
 
 namespace tq {
@@ -94,6 +96,22 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_row_kernel(
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
+// Raises a kernel's dynamic shared memory limit only when a launch needs more
+// than any earlier one, so steady-state launches (and stream capture) make no
+// attribute calls.  The slot is per process; all devices here are B200s.
+static std::atomic<int> smem_attr_slot[kGemvMaxMT + 1];
+
+static cudaError_t ensure_smem_attr(const void* fn, std::atomic<int>& slot, size_t smem) {
+    if ((int)smem <= 48 * 1024 || (int)smem <= slot.load(std::memory_order_acquire)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) {
+        int cur = slot.load();
+        while ((int)smem > cur && !slot.compare_exchange_weak(cur, (int)smem)) {
+        }
+    }
+    return e;
+}
+
 size_t gemv_row_smem_bytes(int mt, int64_t K) { return (size_t)mt * (size_t)(K + 8) * 2; }
 
 cudaError_t launch_gemv_rows(const uint16_t* X, int64_t M, const uint8_t* codes,
@@ -111,8 +129,7 @@ cudaError_t launch_gemv_rows(const uint16_t* X, int64_t M, const uint8_t* codes,
 #define TQ_GEMV_CASE(T)                                                                         \
     case T: {                                                                                   \
         auto k = gemv_row_kernel<T>;                                                            \
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
-                                             (int)smem);                                        \
+        cudaError_t e = ensure_smem_attr((const void*)k, smem_attr_slot[T], smem);              \
         if (e != cudaSuccess) return e;                                                         \
         k<<<grid, block, smem, stream>>>(X, (int)M, codes, scales, N, (int)K, G, Y, y_bf16,     \
                                          d_err);                                                \

@@ -83,3 +83,26 @@ def test_rejected_groups_give_nan_rows():
     X = synthetic.activations(2, K)
     ref = check(X, W, G, codes=codes, scales=scales)
     assert np.all(np.isnan(ref[:, [3, 7, 11, 13]])) and np.all(np.isfinite(ref[:, 17]))
+
+
+def test_unaligned_codes_pointer():
+    """Codes starting at an odd address are still served (the 16-bit code
+    loads are not used then)."""
+    G, N, K = 128, 300, 1024
+    W = synthetic.weights(N, K, index=21)
+    codes, scales, _ = oracle.quantize_pack(W, G)
+    X = synthetic.activations(1, K)
+    ref = oracle.linear(X, codes, scales, N, K, G)
+    buf = torch.zeros(codes.size + 1, dtype=torch.uint8, device="cuda")
+    buf[1:] = to_dev_u8(codes.reshape(-1))
+    Y = tq.gemv(to_dev_bf16(X), buf[1:], to_dev_f16(scales), N, K, G, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert_rows_close_f32(to_f64(Y), ref)
+
+
+@pytest.mark.parametrize("N", [1, 7, 33, 3584 * 6])
+def test_row_counts(N):
+    G, K = 64, 1024
+    W = synthetic.weights(N, K, index=N)
+    X = synthetic.activations(1, K)
+    check(X, W, G, dtypes=(torch.float32,))
