@@ -299,7 +299,7 @@ def run_ours(args, rank, world, local):
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
-            "bound": "hbm", "kernel": "gemv_row_kernel<1>",
+            "bound": "hbm", "kernel": "gemv_lut_kernel (tq_gemv, M=1)",
             "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4),
             "peak_source": peaks["source"],
@@ -339,6 +339,38 @@ def bench_gemv_stream(tq, args, world, peaks):
             "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": reps,
             "note": "same kernel as the headline on one large matrix (inputs 36 MB, L2-resident "
                     "after the first pass; upper bound on the per-launch rate)"}
+
+
+def bench_gemv_shapes(tq, args, world, peaks):
+    """Each decode projection alone (M=1, both G): per-launch time over 48
+    weight copies replayed from a CUDA graph (inputs larger than L2)."""
+    import torch
+    res = {}
+    for G in GROUPS:
+        for name, (N, K) in FFN.items():
+            if name == "up":
+                continue
+            packs = []
+            for c in range(48):
+                W = device_weights(N, K, seed=7000 + c)
+                packs.append(tq.quantize_pack(W, G))
+                del W
+            X = device_acts(1, K, seed=7100)
+            Y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+            for c, s in packs[:3]:
+                tq.gemv(X, c, s, N, K, G, out=Y)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+                for c, s in packs:
+                    tq.gemv(X, c, s, N, K, G, out=Y)
+            ms = timed(graph.replay, max(3, args.steps), max(3, args.warmup), world)
+            us = ms * 1e3 / (max(3, args.steps) * len(packs))
+            byts = packed_bytes(N, K, G) + 2 * K + 2 * N
+            res[f"{name}{N}x{K}_G{G}"] = {"us": round(us, 2), "GB/s": round(byts / us / 1e3, 1),
+                                           "launches": max(3, args.steps) * len(packs)}
+            del packs
+    return res
 
 
 def bench_bulk_codec(tq, args, world, peaks):
@@ -493,7 +525,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
-    ap.add_argument("--only", choices=["stream", "codec", "prefill"], default=None,
+    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv"], default=None,
                     help="run one sub-benchmark alone and print its result (profiling aid)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -508,7 +540,8 @@ def main():
             import ternary_weight_only_group_b200 as tq
             torch.cuda.set_device(local)
             peaks = load_peaks()
-            fn = {"stream": bench_gemv_stream, "codec": bench_bulk_codec, "prefill": bench_prefill}
+            fn = {"stream": bench_gemv_stream, "codec": bench_bulk_codec, "prefill": bench_prefill,
+                  "gemv": bench_gemv_shapes}
             res = fn[args.only](tq, args, world, peaks)
             if rank == 0:
                 print(json.dumps({"only": args.only, "result": res}), flush=True)
