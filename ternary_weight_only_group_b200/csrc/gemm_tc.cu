@@ -38,19 +38,23 @@ namespace tq {
 
 namespace gemm {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3;
+constexpr int UM = 128;                     // rows of X per MMA (two MMAs per k-step)
 constexpr int kThreads = 384;
 constexpr int kDecodeWarp0 = 4, kDecodeWarps = 8;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t A_STAGE = BM * BK * 2;  // 16 KB
-constexpr uint32_t B_STAGE = BN * BK * 2;  // 32 KB
+constexpr uint32_t kTmemCols = 512;         // two 128 x 256 fp32 accumulators
+constexpr uint32_t A_SUB = UM * BK * 2;     // 16 KB: one 128-row X subtile
+constexpr uint32_t B_STAGE = BN * BK * 2;   // 32 KB: decoded W tile
+constexpr uint32_t C_ROW = 32;              // code bytes fetched per W row and stage
+constexpr uint32_t C_STAGE = BN * C_ROW;    // 8 KB
 constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s
 
 struct Smem {
-    uint8_t a[STAGES][A_STAGE];      // X tiles, 1024-byte aligned
+    uint8_t a[STAGES][2][A_SUB];     // X subtiles, 1024-byte aligned
     uint8_t b[STAGES][B_STAGE];      // decoded W tiles
+    uint8_t c[STAGES][C_STAGE];      // packed code bytes of the stage (TMA mode)
     uint2 lut[256];                  // byte -> PRMT selectors of its five weights
-    uint64_t full_a[STAGES], full_b[STAGES], empty[STAGES], done;
+    uint64_t full_a[STAGES], full_c[STAGES], full_b[STAGES], empty[STAGES], done;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -204,7 +208,40 @@ struct Params {
     int y_vec;  // Y rows allow 16-byte vector stores (base aligned, N a multiple of 16 bytes)
 };
 
+// Code bytes q_lo .. q_lo+13 of one row for a stage, read from the staged
+// 32-byte window (TMA mode): the window starts at the 16-byte-aligned byte at
+// or below the first needed one, `off` bytes earlier.
+__device__ __forceinline__ void window_bytes(const uint8_t* row32, int off, uint32_t (&bytes)[14]) {
+    const uint4 lo = *reinterpret_cast<const uint4*>(row32);
+    const uint4 hi = *reinterpret_cast<const uint4*>(row32 + 16);
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    const uint32_t sh = (uint32_t)(off & 3) * 8u;
+    uint32_t o[4];
+    switch (off >> 2) {
+        case 0:
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = __funnelshift_r(w[i], w[i + 1], sh);
+            break;
+        case 1:
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = __funnelshift_r(w[i + 1], w[i + 2], sh);
+            break;
+        case 2:
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = __funnelshift_r(w[i + 2], w[i + 3], sh);
+            break;
+        default:
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = __funnelshift_r(w[i + 3], w[i + 4], sh);
+            break;
+    }
+#pragma unroll
+    for (int i = 0; i < 14; ++i) bytes[i] = (o[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+}
+
+template <bool CODES_TMA>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                                                              const __grid_constant__ CUtensorMap tmap_c,
                                                               const Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>(smem_raw + ((1024 - (s32(smem_raw) & 1023)) & 1023));
@@ -216,24 +253,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 
     // selector table: byte -> selector bytes of digits 0..4 (bytes 5..7 unused)
     for (int b = threadIdx.x; b < 256; b += kThreads) {
-        uint32_t s[5];
+        uint32_t sv[5];
         if (b >= 243) {
-            for (int i = 0; i < 5; ++i) s[i] = kSelNaN;
+            for (int i = 0; i < 5; ++i) sv[i] = kSelNaN;
         } else {
             uint32_t v = b;
             for (int i = 0; i < 5; ++i) {
                 const uint32_t d = v % 3;
                 v /= 3;
-                s[i] = d == 0 ? kSelNeg : (d == 1 ? kSelZero : kSelPos);
+                sv[i] = d == 0 ? kSelNeg : (d == 1 ? kSelZero : kSelPos);
             }
         }
-        sm.lut[b] = make_uint2(s[0] | (s[1] << 8) | (s[2] << 16) | (s[3] << 24), s[4]);
+        sm.lut[b] = make_uint2(sv[0] | (sv[1] << 8) | (sv[2] << 16) | (sv[3] << 24), sv[4]);
     }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&sm.full_a[s], 1);
-            mbar_init(&sm.full_b[s], kDecodeWarps);
-            mbar_init(&sm.empty[s], 1);
+        for (int st = 0; st < STAGES; ++st) {
+            mbar_init(&sm.full_a[st], 1);
+            mbar_init(&sm.full_c[st], 1);
+            mbar_init(&sm.full_b[st], kDecodeWarps);
+            mbar_init(&sm.empty[st], 1);
         }
         mbar_init(&sm.done, 1);
         sm.abort_flag = 0;
@@ -250,43 +288,66 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+
+    // first code byte of stage kb inside its row, and the 16-byte-aligned TMA window start
+    auto stage_geom = [&](int kb, int& g, int& c0, int& q_lo) {
+        const int k0 = kb * BK;
+        g = k0 / p.G;
+        c0 = k0 - g * p.G;
+        q_lo = c0 / 5;
+    };
+
     if (warp == 0) {
-        // ---------------- TMA producer (X)
+        // ---------------- TMA producer: X subtiles (and the stage's code window)
         int issued = 0;
         if (lane == 0) {
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % STAGES, use = kb / STAGES;
-                if (use > 0 && !mbar_wait(&sm.empty[s], (use - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&sm.full_a[s], A_STAGE);
-                tma_load_2d(sm.a[s], &tmap_x, kb * BK, (int)m0, &sm.full_a[s]);
+                const int st = kb % STAGES, use = kb / STAGES;
+                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
+                mbar_arrive_expect_tx(&sm.full_a[st], 2 * A_SUB);
+                tma_load_2d(sm.a[st][0], &tmap_x, kb * BK, (int)m0, &sm.full_a[st]);
+                tma_load_2d(sm.a[st][1], &tmap_x, kb * BK, (int)(m0 + UM), &sm.full_a[st]);
+                if (CODES_TMA) {
+                    int g, c0, q_lo;
+                    stage_geom(kb, g, c0, q_lo);
+                    const int gb = g * p.B + q_lo;
+                    mbar_arrive_expect_tx(&sm.full_c[st], C_STAGE);
+                    tma_load_2d(sm.c[st], &tmap_c, gb & ~15, (int)n0, &sm.full_c[st]);
+                }
                 ++issued;
             }
             // Drain: every issued load must land before the CTA can exit.
             for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb) {
-                const int s = kb % STAGES, use = kb / STAGES;
+                const int st = kb % STAGES, use = kb / STAGES;
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(&sm.full_a[s], use & 1) && globaltimer() - t0 < kTimeoutNs) {
+                while (!mbar_try_wait(&sm.full_a[st], use & 1) && globaltimer() - t0 < kTimeoutNs) {
                 }
+                if (CODES_TMA)
+                    while (!mbar_try_wait(&sm.full_c[st], use & 1) && globaltimer() - t0 < kTimeoutNs) {
+                    }
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer: two 128 x 256 x 16 MMAs per k-step
         if (lane == 0) {
-            const uint32_t idesc = instr_desc(BM, BN);
-            int kb = 0;
-            for (; kb < nk; ++kb) {
-                const int s = kb % STAGES, use = kb / STAGES;
-                if (!mbar_wait(&sm.full_a[s], use & 1, abort_flag)) break;
-                if (!mbar_wait(&sm.full_b[s], use & 1, abort_flag)) break;
+            const uint32_t idesc = instr_desc(UM, BN);
+            for (int kb = 0; kb < nk; ++kb) {
+                const int st = kb % STAGES, use = kb / STAGES;
+                if (!mbar_wait(&sm.full_a[st], use & 1, abort_flag)) break;
+                if (!mbar_wait(&sm.full_b[st], use & 1, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t a0 = s32(sm.a[s]), b0 = s32(sm.b[s]);
+                const uint32_t b0 = s32(sm.b[st]);
 #pragma unroll
-                for (int k = 0; k < BK / 16; ++k)
-                    mma_bf16(tmem, smem_desc_sw128(a0 + 32 * k), smem_desc_sw128(b0 + 32 * k), idesc,
-                             (kb > 0 || k > 0) ? 1u : 0u);
-                mma_commit(&sm.empty[s]);  // stage free once these MMAs have read it
+                for (int sub = 0; sub < 2; ++sub) {
+                    const uint32_t a0 = s32(sm.a[st][sub]);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        mma_bf16(tmem + (uint32_t)(sub * BN), smem_desc_sw128(a0 + 32 * k),
+                                 smem_desc_sw128(b0 + 32 * k), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                }
+                mma_commit(&sm.empty[st]);  // stage free once these MMAs have read it
             }
-            mma_commit(&sm.done);  // all issued MMAs complete -> accumulator ready
+            mma_commit(&sm.done);  // all issued MMAs complete -> accumulators ready
         }
     } else if (warp >= kDecodeWarp0) {
         // ---------------- decoders: thread -> one W row of the tile
@@ -298,15 +359,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         const int real = p.G - 5 * (p.B - 1);
         const uint32_t pm = padding_mask(real), po = padding_ones(real);
         for (int kb = 0; kb < nk; ++kb) {
-            const int s = kb % STAGES, use = kb / STAGES;
-            if (use > 0 && !mbar_wait(&sm.empty[s], (use - 1) & 1, abort_flag)) break;
-            const int k0 = kb * BK;
-            const int g = k0 / p.G, c0 = k0 - g * p.G;
-            const int q_lo = c0 / 5;
+            const int st = kb % STAGES, use = kb / STAGES;
+            int g, c0, q_lo;
+            stage_geom(kb, g, c0, q_lo);
             uint32_t bytes[14];
-            const uint8_t* cb = crow + (int64_t)g * p.B;
+            if (CODES_TMA) {
+                if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag)) break;
+                const int gb = g * p.B + q_lo;
+                window_bytes(sm.c[st] + t * C_ROW, gb & 15, bytes);
 #pragma unroll
-            for (int i = 0; i < 14; ++i) bytes[i] = (q_lo + i < p.B) ? (uint32_t)__ldg(cb + q_lo + i) : kZeroByte;
+                for (int i = 0; i < 14; ++i)
+                    if (q_lo + i >= p.B) bytes[i] = kZeroByte;
+            } else {
+                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
+                const uint8_t* cb = crow + (int64_t)g * p.B;
+#pragma unroll
+                for (int i = 0; i < 14; ++i)
+                    bytes[i] = (q_lo + i < p.B) ? (uint32_t)__ldg(cb + q_lo + i) : kZeroByte;
+            }
             // a group's last byte with a padding digit other than 1 decodes to NaN
             const int ql = p.B - 1 - q_lo;
 #pragma unroll
@@ -326,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 V = mag | ((mag ? (mag | 0x8000u) : 0u) << 16);  // {+s, -s}
                 Z = 0x7FC00000u;                                // {0, NaN}
             }
-            uint8_t* row = sm.b[s] + t * 128;
+            uint8_t* row = sm.b[st] + t * 128;
             const int rin = t & 7;
             switch (c0 % 5) {
                 case 0: decode_row<0>(sm.lut, bytes, V, Z, row, rin); break;
@@ -337,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor core
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.full_b[s]);
+            if (lane == 0) mbar_arrive(&sm.full_b[st]);
         }
         // ---------------- epilogue: warps 4..7 read their accumulator quadrant
         if (warp < kDecodeWarp0 + 4) {
@@ -345,40 +415,47 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             const bool ok = mbar_wait(&sm.done, 0, abort_flag);
             tc_fence_after();
             if (ok) {
-                const int64_t m = m0 + 32 * q + lane;
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(32 * c), r);
-                    const int64_t nb = n0 + 32 * c;
-                    if (m < p.M && nb < p.N) {
-                        const int cnt = (int)(p.N - nb < 32 ? p.N - nb : 32);
-                        if (p.y_bf16) {
-                            __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.Y) + m * p.N + nb;
-                            if (cnt == 32 && p.y_vec) {
+                for (int sub = 0; sub < 2; ++sub) {
+                    const int64_t m = m0 + sub * UM + 32 * q + lane;
+                    for (int c = 0; c < BN / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(sub * BN + 32 * c), r);
+                        const int64_t nb = n0 + 32 * c;
+                        if (m < p.M && nb < p.N) {
+                            const int cnt = (int)(p.N - nb < 32 ? p.N - nb : 32);
+                            if (p.y_bf16) {
+                                __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.Y) + m * p.N + nb;
+                                if (cnt == 32 && p.y_vec) {
 #pragma unroll
-                                for (int v = 0; v < 4; ++v) {
-                                    uint32_t w[4];
+                                    for (int v = 0; v < 4; ++v) {
+                                        uint32_t w[4];
 #pragma unroll
-                                    for (int h = 0; h < 4; ++h) {
-                                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                                            __uint_as_float(r[8 * v + 2 * h]), __uint_as_float(r[8 * v + 2 * h + 1]));
-                                        w[h] = *reinterpret_cast<const uint32_t*>(&b2);
+                                        for (int h = 0; h < 4; ++h) {
+                                            const __nv_bfloat162 b2 =
+                                                __floats2bfloat162_rn(__uint_as_float(r[8 * v + 2 * h]),
+                                                                      __uint_as_float(r[8 * v + 2 * h + 1]));
+                                            w[h] = *reinterpret_cast<const uint32_t*>(&b2);
+                                        }
+                                        reinterpret_cast<uint4*>(y)[v] = make_uint4(w[0], w[1], w[2], w[3]);
                                     }
-                                    reinterpret_cast<uint4*>(y)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                                } else {
+#pragma unroll
+                                    for (int j = 0; j < 32; ++j)
+                                        if (j < cnt) y[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
                                 }
                             } else {
-                                for (int j = 0; j < cnt; ++j) y[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
-                            }
-                        } else {
-                            float* y = reinterpret_cast<float*>(p.Y) + m * p.N + nb;
-                            if (cnt == 32 && p.y_vec) {
+                                float* y = reinterpret_cast<float*>(p.Y) + m * p.N + nb;
+                                if (cnt == 32 && p.y_vec) {
 #pragma unroll
-                                for (int v = 0; v < 8; ++v)
-                                    reinterpret_cast<float4*>(y)[v] =
-                                        make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                                    __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-                            } else {
-                                for (int j = 0; j < cnt; ++j) y[j] = __uint_as_float(r[j]);
+                                    for (int v = 0; v < 8; ++v)
+                                        reinterpret_cast<float4*>(y)[v] =
+                                            make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                        __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+                                } else {
+#pragma unroll
+                                    for (int j = 0; j < 32; ++j)
+                                        if (j < cnt) y[j] = __uint_as_float(r[j]);
+                                }
                             }
                         }
                     }
@@ -433,21 +510,38 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
     (void)sm_count;
     *handled = false;
     // Shapes this kernel covers: K a multiple of the 64-column stage, G a
-    // multiple of 64 (a stage never crosses a group), rows of X 16-byte aligned.
+    // multiple of 64 (a stage never crosses a group).
     if (K % BK != 0 || G % 64 != 0 || M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (1 << 30))
         return cudaSuccess;
     PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    CUtensorMap tmap;
-    std::memset(&tmap, 0, sizeof(tmap));
-    const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
-    const cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {BK, BM};
-    const cuuint32_t estride[2] = {1, 1};
-    CUresult r = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), gdim, gstride, box,
-                     estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    const int B = bytes_per_group(G);
+    const int64_t row_bytes = (int64_t)(K / G) * B;
+    CUtensorMap tmap_x, tmap_c;
+    std::memset(&tmap_x, 0, sizeof(tmap_x));
+    std::memset(&tmap_c, 0, sizeof(tmap_c));
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)K * 2};
+        const cuuint32_t box[2] = {BK, UM};
+        const cuuint32_t estride[2] = {1, 1};
+        CUresult r = enc(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), gdim, gstride, box,
+                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
+    // Codes by TMA when their rows are 16-byte multiples and the base is 16-byte aligned.
+    const bool codes_tma = (row_bytes % 16 == 0) && ((reinterpret_cast<uintptr_t>(codes) & 15) == 0);
+    if (codes_tma) {
+        const cuuint64_t gdim[2] = {(cuuint64_t)row_bytes, (cuuint64_t)N};
+        const cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
+        const cuuint32_t box[2] = {C_ROW, BN};
+        const cuuint32_t estride[2] = {1, 1};
+        CUresult r = enc(&tmap_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), gdim, gstride, box,
+                         estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
     Params p{};
     p.codes = codes;
     p.scales = scales;
@@ -457,9 +551,9 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
     p.N = N;
     p.K = (int)K;
     p.G = G;
-    p.B = bytes_per_group(G);
+    p.B = B;
     p.ng = (int)(K / G);
-    p.row_bytes = (int64_t)p.ng * p.B;
+    p.row_bytes = row_bytes;
     p.n_tiles = (int)((N + BN - 1) / BN);
     p.y_bf16 = y_bf16;
     p.y_vec = ((reinterpret_cast<uintptr_t>(Y) & 15) == 0) && ((N * (y_bf16 ? 2 : 4)) % 16 == 0);
@@ -467,13 +561,15 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
     const int64_t grid = m_tiles * p.n_tiles;
     if (grid > 0x7FFFFFFF) return cudaSuccess;
     const size_t smem = gemm_smem_bytes();
-    static std::atomic<int> smem_set{0};
-    if ((int)smem > smem_set.load()) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = codes_tma ? gemm_tc_kernel<true> : gemm_tc_kernel<false>;
+    static std::atomic<int> smem_set[2];
+    std::atomic<int>& slot = smem_set[codes_tma ? 1 : 0];
+    if ((int)smem > slot.load()) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        smem_set.store((int)smem);
+        slot.store((int)smem);
     }
-    gemm_tc_kernel<<<(unsigned)grid, kThreads, smem, stream>>>(tmap, p);
+    kern<<<(unsigned)grid, kThreads, smem, stream>>>(tmap_x, tmap_c, p);
     *handled = true;
     return cudaGetLastError();
 }
