@@ -1,0 +1,355 @@
+// gemm_small.cu -- small-M fused matmul on the tensor cores (tcgen05, sm_100a).
+//
+// Same result as the decode GEMV and the prefill GEMM (tiny-llm "Week 2 Day
+// 3: Quantize the Model", "Mathematical Formulation": C = A B^T with B
+// reconstructed per group, float accumulation; "Tune the SIMD Schedule":
+// the decode and matrix schedules are chosen by M), for 5 <= M <= 64 tokens.
+// The roles of the operands are swapped so the tensor core's 128-row side is
+// filled by weights:  D^T[128 W rows x NT tokens] += What[128 x 16] . X[NT x 16]^T
+// with What decoded on chip into the 128-byte-swizzled K-major layout (as in
+// the prefill GEMM) and X tiles (NT = 16, 32 or 64 rows, zero-filled past M)
+// loaded by TMA.  K is split across the CTAs of a thread-block cluster; each
+// CTA pushes its fp32 partial tile into the shared memory of the rank that
+// owns those rows (distributed shared memory), one cluster barrier, and the
+// owner adds the partials in rank order (deterministic) and writes Y.
+//   warp 0  TMA producer (X tile and the stage's code-byte window)
+//   warp 1  MMA issuer (tcgen05.mma kind::f16, M=128, N=NT, fp32 in TMEM)
+//   warp 2  tensor-memory allocation
+//   warps 4-7  decoders (one W row per thread), then the epilogue
+// All mbarrier waits are bounded (globaltimer deadline -> TQ_DERR_TIMEOUT).
+#include <cooperative_groups.h>
+
+#include <atomic>
+#include <cstring>
+
+#include "tc_common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace tq {
+namespace small {
+
+using namespace tc;
+
+constexpr int WM = 128;  // W rows per CTA (UMMA M)
+constexpr int BK = 64;
+constexpr int STAGES = 6;
+constexpr int kThreads = 256;
+constexpr int kDecodeWarp0 = 4, kDecodeWarps = 4;
+constexpr uint32_t W_STAGE = WM * BK * 2;  // 16 KB
+constexpr uint32_t C_ROW = 32;
+constexpr uint32_t C_STAGE = WM * C_ROW;   // 4 KB
+constexpr int kMaxCS = 8;
+
+template <int NT>
+struct Smem {
+    uint8_t w[STAGES][W_STAGE];   // decoded W tiles (UMMA A), 1024-byte aligned
+    uint8_t x[STAGES][NT * 128];  // X tiles (UMMA B): NT rows of 128 bytes
+    uint8_t c[STAGES][C_STAGE];   // code-byte windows
+    float red[WM * NT];           // partials pushed by the cluster: [rank][row of owner][token]
+    uint2 lut[256];
+    uint64_t full_x[STAGES], full_c[STAGES], full_w[STAGES], empty[STAGES], done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct Params {
+    const uint8_t* codes;
+    int64_t row_bytes;
+    const uint16_t* scales;
+    void* Y;
+    uint32_t* d_err;
+    int64_t M, N;
+    int K, G, B, ng;
+    int CS;  // cluster size = split of K
+    int y_bf16;
+};
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <int NT, bool CODES_TMA>
+__global__ void __launch_bounds__(kThreads, 1) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                                                                 const __grid_constant__ CUtensorMap tmap_c,
+                                                                 const Params p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    Smem<NT>& sm = *reinterpret_cast<Smem<NT>*>(smem_raw + ((1024 - (s32(smem_raw) & 1023)) & 1023));
+    cg::cluster_group cluster = cg::this_cluster();
+    const int crank = (int)cluster.block_rank();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n0 = (int64_t)(blockIdx.x / p.CS) * WM;
+    const int nk = p.K / BK;
+    const int kb_lo = (int)((int64_t)nk * crank / p.CS), kb_hi = (int)((int64_t)nk * (crank + 1) / p.CS);
+    const int nkl = kb_hi - kb_lo;  // stages of this CTA (>= 1)
+    constexpr uint32_t kCols = NT < 32 ? 32 : NT;
+    volatile int* abort_flag = &sm.abort_flag;
+
+    init_selector_lut(sm.lut, threadIdx.x, kThreads);
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < STAGES; ++st) {
+            mbar_init(&sm.full_x[st], 1);
+            mbar_init(&sm.full_c[st], 1);
+            mbar_init(&sm.full_w[st], kDecodeWarps);
+            mbar_init(&sm.empty[st], 1);
+        }
+        mbar_init(&sm.done, 1);
+        sm.abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(s32(&sm.tmem_base)),
+                     "r"(kCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    auto stage_geom = [&](int kb, int& g, int& c0, int& q_lo) {
+        const int k0 = kb * BK;
+        g = k0 / p.G;
+        c0 = k0 - g * p.G;
+        q_lo = c0 / 5;
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < nkl; ++i) {
+                const int kb = kb_lo + i, st = i % STAGES, use = i / STAGES;
+                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
+                int g, c0, q_lo;
+                stage_geom(kb, g, c0, q_lo);
+                mbar_arrive_expect_tx(&sm.full_x[st], NT * 128);
+                tma_load_2d(sm.x[st], &tmap_x, kb * BK, 0, &sm.full_x[st]);
+                if (CODES_TMA) {
+                    mbar_arrive_expect_tx(&sm.full_c[st], C_STAGE);
+                    tma_load_2d(sm.c[st], &tmap_c, (g * p.B + q_lo) & ~15, (int)n0, &sm.full_c[st]);
+                }
+                ++issued;
+            }
+            for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
+                const int st = i % STAGES, use = i / STAGES;
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait(&sm.full_x[st], use & 1) && globaltimer() - t0 < kTimeoutNs) {
+                }
+                if (CODES_TMA)
+                    while (!mbar_try_wait(&sm.full_c[st], use & 1) && globaltimer() - t0 < kTimeoutNs) {
+                    }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = instr_desc(WM, NT);
+            for (int i = 0; i < nkl; ++i) {
+                const int st = i % STAGES, use = i / STAGES;
+                if (!mbar_wait(&sm.full_x[st], use & 1, abort_flag)) break;
+                if (!mbar_wait(&sm.full_w[st], use & 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t a0 = s32(sm.w[st]), b0 = s32(sm.x[st]);
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k)
+                    mma_bf16(tmem, smem_desc_sw128(a0 + 32 * k), smem_desc_sw128(b0 + 32 * k), idesc,
+                             (i > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&sm.empty[st]);
+            }
+            mma_commit(&sm.done);
+        }
+    } else if (warp >= kDecodeWarp0) {
+        const int t = threadIdx.x - kDecodeWarp0 * 32;  // W row of the tile
+        const int64_t n = n0 + t;
+        const uint16_t* srow = p.scales + (n < p.N ? n : 0) * p.ng;
+        const int real = p.G - 5 * (p.B - 1);
+        const uint32_t pm = padding_mask(real), po = padding_ones(real);
+        const uint8_t* crow = p.codes + (n < p.N ? n : 0) * p.row_bytes;
+        auto load_global = [&](int kb, uint32_t (&bytes)[14]) {
+            int g, c0, q_lo;
+            stage_geom(kb, g, c0, q_lo);
+            const uint8_t* cb = crow + (int64_t)g * p.B;
+#pragma unroll
+            for (int j = 0; j < 14; ++j) bytes[j] = (q_lo + j < p.B) ? (uint32_t)__ldg(cb + q_lo + j) : kZeroByte;
+        };
+        uint32_t cur[14], nxt[14];
+        if (!CODES_TMA && nkl > 0) load_global(kb_lo, cur);
+        for (int i = 0; i < nkl; ++i) {
+            const int kb = kb_lo + i, st = i % STAGES, use = i / STAGES;
+            int g, c0, q_lo;
+            stage_geom(kb, g, c0, q_lo);
+            uint32_t bytes[14];
+            if (CODES_TMA) {
+                if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag)) break;
+                window_bytes(sm.c[st] + t * C_ROW, (g * p.B + q_lo) & 15, bytes);
+            } else {
+                if (i + 1 < nkl) load_global(kb + 1, nxt);  // next stage's bytes in flight
+                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
+#pragma unroll
+                for (int j = 0; j < 14; ++j) bytes[j] = cur[j];
+            }
+            decode_stage_row(sm.lut, bytes, c0, q_lo, p.B, pm, po, __ldg(srow + g), sm.w[st] + t * 128, t & 7);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.full_w[st]);
+            if (!CODES_TMA) {
+#pragma unroll
+                for (int j = 0; j < 14; ++j) cur[j] = nxt[j];
+            }
+        }
+    }
+
+    // ---------------- epilogue: partial tile -> owner ranks -> Y
+    const int RPQ = WM / p.CS;  // rows owned by each rank
+    if (warp >= kDecodeWarp0) {
+        const int q = warp - kDecodeWarp0;
+        const int r = 32 * q + lane;  // W row of the tile = TMEM lane
+        const bool ok = mbar_wait(&sm.done, 0, abort_flag);
+        tc_fence_after();
+        uint32_t v[NT];
+        if (NT == 16) {
+            uint32_t (&v16)[16] = reinterpret_cast<uint32_t (&)[16]>(v);
+            tmem_ld16(tmem + ((uint32_t)(32 * q) << 16), v16);
+        } else {
+#pragma unroll
+            for (int h = 0; h < NT / 32; ++h) {
+                uint32_t (&v32)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[32 * h]);
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 32u * h, v32);
+            }
+        }
+        if (!ok) {
+#pragma unroll
+            for (int j = 0; j < NT; ++j) v[j] = 0x7FC00000u;
+        }
+        const int owner = r / RPQ;
+        float* dst = cluster.map_shared_rank(sm.red, owner) + ((crank * RPQ) + (r - owner * RPQ)) * NT;
+#pragma unroll
+        for (int j = 0; j < NT; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                                              __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+    }
+    tc_fence_before();
+    cluster.sync();
+    tc_fence_after();
+    // owner: rows [crank*RPQ, (crank+1)*RPQ) of the tile, all tokens
+    const int64_t Mv = p.M < NT ? p.M : NT;
+    for (int i = threadIdx.x; i < RPQ * Mv; i += kThreads) {
+        const int m = i / RPQ, rr = i - m * RPQ;
+        float acc = 0.f;
+        for (int qr = 0; qr < p.CS; ++qr) acc += sm.red[(qr * RPQ + rr) * NT + m];
+        const int64_t n = n0 + crank * RPQ + rr;
+        if (n < p.N) {
+            const int64_t o = (int64_t)m * p.N + n;
+            if (p.y_bf16) reinterpret_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(acc);
+            else reinterpret_cast<float*>(p.Y)[o] = acc;
+        }
+    }
+
+    // ---------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1 && lane == 0 && *abort_flag) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(&sm.done, 0) && globaltimer() - t0 < kTimeoutNs) {
+        }
+    }
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols) : "memory");
+    if (threadIdx.x == 0 && *abort_flag && p.d_err) atomicOr(p.d_err, TQ_DERR_TIMEOUT);
+}
+
+template <int NT, bool CT>
+static cudaError_t launch_nt(const CUtensorMap& tx, const CUtensorMap& tc_, const Params& p, int tiles,
+                             cudaStream_t stream) {
+    auto kern = gemm_small_kernel<NT, CT>;
+    const size_t smem = sizeof(Smem<NT>) + 1024;
+    static std::atomic<int> smem_set{0};
+    if ((int)smem > smem_set.load()) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        smem_set.store((int)smem);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles * p.CS));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.CS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tx, tc_, p);
+}
+
+}  // namespace small
+
+// Covered shapes: 1 <= M <= 64, K % 64 == 0, G % 64 == 0, code rows a
+// multiple of 16 bytes with a 16-byte aligned base.  Otherwise *handled is
+// left false and nothing is launched.
+cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
+                              int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
+                              cudaStream_t stream, int sm_count, bool* handled) {
+    using namespace small;
+    *handled = false;
+    const int B = bytes_per_group(G);
+    const int64_t row_bytes = (int64_t)(K / G) * B;
+    if (M < 1 || M > 64 || K % BK != 0 || G % 64 != 0 || N > (int64_t(1) << 31) || K > (1 << 30))
+        return cudaSuccess;
+    // code bytes by TMA when their rows are 16-byte multiples with an aligned base, else by loads
+    const bool codes_tma = row_bytes % 16 == 0 && (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
+    const int NT = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    CUtensorMap tx, tcm;
+    if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<uint16_t*>(X), (uint64_t)K, (uint64_t)M,
+                        (uint64_t)K * 2, BK, (uint32_t)NT, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    std::memset(&tcm, 0, sizeof(tcm));
+    if (codes_tma && !encode_tmap_2d(&tcm, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<uint8_t*>(codes),
+                                     (uint64_t)row_bytes, (uint64_t)N, (uint64_t)row_bytes, C_ROW, WM,
+                                     CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    const int nk = (int)(K / BK);
+    const int64_t tiles = (N + WM - 1) / WM;
+    if (tiles * kMaxCS > 0x7FFFFFFF) return cudaSuccess;
+    // split K so the grid covers the SMs, keeping at least two stages per CTA
+    int CS = 1;
+    while (CS < kMaxCS && tiles * CS * 2 <= sm_count && nk / (CS * 2) >= 2) CS *= 2;
+    Params p{};
+    p.codes = codes;
+    p.row_bytes = row_bytes;
+    p.scales = scales;
+    p.Y = Y;
+    p.d_err = d_err;
+    p.M = M;
+    p.N = N;
+    p.K = (int)K;
+    p.G = G;
+    p.B = B;
+    p.ng = (int)(K / G);
+    p.CS = CS;
+    p.y_bf16 = y_bf16;
+    cudaError_t e;
+    if (codes_tma) {
+        if (NT == 16) e = launch_nt<16, true>(tx, tcm, p, (int)tiles, stream);
+        else if (NT == 32) e = launch_nt<32, true>(tx, tcm, p, (int)tiles, stream);
+        else e = launch_nt<64, true>(tx, tcm, p, (int)tiles, stream);
+    } else {
+        if (NT == 16) e = launch_nt<16, false>(tx, tcm, p, (int)tiles, stream);
+        else if (NT == 32) e = launch_nt<32, false>(tx, tcm, p, (int)tiles, stream);
+        else e = launch_nt<64, false>(tx, tcm, p, (int)tiles, stream);
+    }
+    if (e == cudaSuccess) *handled = true;
+    return e;
+}
+
+}  // namespace tq

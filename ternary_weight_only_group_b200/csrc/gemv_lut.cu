@@ -38,7 +38,7 @@ namespace cg = cooperative_groups;
 
 namespace tq {
 
-constexpr int kLutThreads = 512;
+constexpr int kLutThreads = 256;
 constexpr int kLutWarps = kLutThreads / 32;
 constexpr int kRB = 8;                 // rows per warp batch
 constexpr int kLPG = 13;               // lanes per group
@@ -196,7 +196,7 @@ __device__ __forceinline__ void build_part(const LutArgs& a, float* tab, int sl,
 }
 
 template <int B, int MT, int NS>
-__global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const LutArgs a) {
+__global__ void __launch_bounds__(kLutThreads, 2) gemv_lut_kernel(const LutArgs a) {
     constexpr int BPL = B / kLPG;
     constexpr int SLICE_BYTES = kGPS * B;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -385,7 +385,7 @@ static bool make_plan(int64_t N, int K, int G, int MT, int sm_count, size_t smem
         for (int ns = 1; ns <= per_cta && ns <= ns_max; ++ns) {
             if (per_cta % ns || ns == 3) continue;
             const size_t tbytes = table_per_slice * ns;
-            if (tbytes > 160 * 1024) continue;
+            if (tbytes > 96 * 1024) continue;
             int rb = sm_count / cs;
             if (rb < 1) rb = 1;
             int64_t R = (N + rb - 1) / rb;
@@ -397,7 +397,8 @@ static bool make_plan(int64_t N, int K, int G, int MT, int sm_count, size_t smem
             const size_t off_acc = off_scale + (size_t)ns * kGPS * RP * 4;
             const size_t off_red = off_acc + (size_t)MT * RP * 4;
             const size_t smem = off_red + (size_t)cs * MT * PER * 4;
-            if (smem > smem_limit) continue;
+            // two CTAs per SM, so a dependent launch's CTAs can start beside this one's
+            if (smem > smem_limit || smem > 112 * 1024) continue;
             // estimated cycles per CTA: table writes (one wavefront per 26 entries),
             // lookups (~1/20 cycle per byte per row), row reductions, cluster overhead
             const int passes = per_cta / ns;

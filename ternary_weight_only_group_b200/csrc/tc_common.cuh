@@ -1,0 +1,242 @@
+// tc_common.cuh -- device helpers shared by the tensor-core kernels (sm_100a):
+// mbarriers with bounded waits, TMA loads, UMMA descriptors, tcgen05 MMA /
+// commit / fences / TMEM loads, and the on-chip ternary decoder that writes
+// bf16 weights into the 128-byte-swizzled K-major layout.
+#pragma once
+
+#include <cuda.h>
+
+#include "tq_internal.cuh"
+
+namespace tq {
+namespace tc {
+
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // bound of every mbarrier wait: 2 s
+
+__device__ __forceinline__ uint32_t s32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(s32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(s32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(s32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(s32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: false when the deadline passed or another role gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            s32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(s32(bar))
+        : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major operand with 128-byte swizzle:
+// rows of 128 bytes, 8-row atoms 1024 bytes apart (SBO), version 1.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFF);
+    d |= (uint64_t)1 << 16;             // leading byte offset (16 B; unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset: 1024 B between 8-row groups
+    d |= (uint64_t)1 << 46;             // descriptor version
+    d |= (uint64_t)2 << 61;             // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor: kind::f16, bf16 A and B (K-major), fp32 D, M x N.
+__host__ __device__ constexpr uint32_t instr_desc(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(s32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+        "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// PRMT selector byte of one weight: two nibbles naming the bytes of its bf16
+// value inside the 8-byte pair (V = {+s, -s}, Z = {0, NaN}).
+constexpr uint32_t kSelPos = 0x10, kSelNeg = 0x32, kSelZero = 0x54, kSelNaN = 0x76;
+
+// Decode one row's 64 weights of a stage (columns c0..c0+63 of group g, c0 % 5 == R0)
+// into the swizzled tile row.  bytes[] holds code bytes q_lo .. q_lo+13.
+template <int R0>
+__device__ __forceinline__ void decode_row(const uint2* lut, const uint32_t (&bytes)[14], uint32_t V, uint32_t Z,
+                                           uint8_t* tile_row, int row_in_atom) {
+    // selector bytes of the 64 columns: column j uses digit (R0 + j) % 5 of byte (R0 + j) / 5
+    uint2 e[14];
+#pragma unroll
+    for (int t = 0; t < 14; ++t) e[t] = lut[bytes[t]];
+#pragma unroll
+    for (int chunk = 0; chunk < 8; ++chunk) {
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const int j0 = chunk * 8 + 2 * h, j1 = j0 + 1;
+            const int q0 = (R0 + j0) / 5, i0 = (R0 + j0) % 5;
+            const int q1 = (R0 + j1) / 5, i1 = (R0 + j1) % 5;
+            // selector bytes live in byte i of the 8-byte entry {lo, hi}
+            uint32_t sel;
+            if (q0 == q1) {
+                const uint32_t lo = e[q0].x, hi = e[q0].y;
+                sel = prmt(lo, hi, (uint32_t)i0 | ((uint32_t)i1 << 4));
+            } else {  // pair straddles two bytes: digit 4 of one, digit 0 of the next
+                sel = prmt(e[q0].y, e[q1].x, 0u | (4u << 4));
+            }
+            // sel bytes: [s0, s1, ...]; value selector = s0 | s1 << 8 (PRMT uses the low 16 bits)
+            w[h] = prmt(V, Z, sel);
+        }
+        const int phys = chunk ^ row_in_atom;  // 128-byte swizzle: 16-byte chunk index XOR (row % 8)
+        *reinterpret_cast<uint4*>(tile_row + phys * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// Code bytes q_lo .. q_lo+13 of one row for a stage, read from the staged
+// 32-byte window (TMA mode): the window starts at the 16-byte-aligned byte at
+// or below the first needed one, `off` bytes earlier.
+__device__ __forceinline__ void window_bytes(const uint8_t* row32, int off, uint32_t (&bytes)[14]) {
+    const uint4 lo = *reinterpret_cast<const uint4*>(row32);
+    const uint4 hi = *reinterpret_cast<const uint4*>(row32 + 16);
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    const uint32_t sh = (uint32_t)(off & 3) * 8u;
+    uint32_t o[4];
+    switch (off >> 2) {
+        case 0:
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = __funnelshift_r(w[i], w[i + 1], sh);
+            break;
+        case 1:
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = __funnelshift_r(w[i + 1], w[i + 2], sh);
+            break;
+        case 2:
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = __funnelshift_r(w[i + 2], w[i + 3], sh);
+            break;
+        default:
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = __funnelshift_r(w[i + 3], w[i + 4], sh);
+            break;
+    }
+#pragma unroll
+    for (int i = 0; i < 14; ++i) bytes[i] = (o[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+}
+
+
+// Selector table: byte -> PRMT selector bytes of its five weights (digits
+// 0..4 in bytes 0..4 of the 8-byte entry); bytes >= 243 select NaN.
+__device__ __forceinline__ void init_selector_lut(uint2* lut, int tid, int nthreads) {
+    for (int b = tid; b < 256; b += nthreads) {
+        uint32_t sv[5];
+        if (b >= 243) {
+            for (int i = 0; i < 5; ++i) sv[i] = kSelNaN;
+        } else {
+            uint32_t v = b;
+            for (int i = 0; i < 5; ++i) {
+                const uint32_t d = v % 3;
+                v /= 3;
+                sv[i] = d == 0 ? kSelNeg : (d == 1 ? kSelZero : kSelPos);
+            }
+        }
+        lut[b] = make_uint2(sv[0] | (sv[1] << 8) | (sv[2] << 16) | (sv[3] << 24), sv[4]);
+    }
+}
+
+// Decodes the 64 weights of one W row for a stage (columns c0 .. c0+63 of
+// group g, code bytes q_lo .. q_lo+13 in bytes[]) into a 128-byte swizzled
+// tile row.  A group's last byte with a padding digit other than 1, and a
+// scale that is NaN, Inf or negative, decode to NaN.
+__device__ __forceinline__ void decode_stage_row(const uint2* lut, uint32_t (&bytes)[14], int c0, int q_lo, int B,
+                                                 uint32_t pm, uint32_t po, uint32_t scale_bits, uint8_t* tile_row,
+                                                 int row_in_atom) {
+    const int ql = B - 1 - q_lo;
+#pragma unroll
+    for (int i = 0; i < 14; ++i) {
+        if (q_lo + i >= B) bytes[i] = kZeroByte;
+        if (i == ql) {
+            const uint32_t dp = byte_digit_pattern(bytes[i]);
+            if ((dp & 0x8000u) == 0 && (dp & pm) != po) bytes[i] = 255;
+        }
+    }
+    uint32_t V, Z;
+    if (scale_is_bad(scale_bits)) {
+        V = 0x7FC07FC0u;
+        Z = 0x7FC07FC0u;
+    } else {
+        const uint32_t mag = scale_bits == 0 ? 0u : scale_to_bf16_bits((uint16_t)scale_bits);
+        V = mag | ((mag ? (mag | 0x8000u) : 0u) << 16);  // {+s, -s}
+        Z = 0x7FC00000u;                                // {0, NaN}
+    }
+    switch (c0 % 5) {
+        case 0: decode_row<0>(lut, bytes, V, Z, tile_row, row_in_atom); break;
+        case 1: decode_row<1>(lut, bytes, V, Z, tile_row, row_in_atom); break;
+        case 2: decode_row<2>(lut, bytes, V, Z, tile_row, row_in_atom); break;
+        case 3: decode_row<3>(lut, bytes, V, Z, tile_row, row_in_atom); break;
+        default: decode_row<4>(lut, bytes, V, Z, tile_row, row_in_atom); break;
+    }
+}
+
+// Encoder of 2-D TMA descriptors (driver entry point, no libcuda link).
+bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, void* base, uint64_t dim0, uint64_t dim1,
+                    uint64_t stride1_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle swizzle);
+
+}  // namespace tc
+}  // namespace tq

@@ -21,6 +21,9 @@ cudaError_t launch_gemv_rows(const uint16_t* X, int64_t M, const uint8_t* codes,
 cudaError_t launch_gemv_lut(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                             int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                             cudaStream_t stream, int sm_count, size_t smem_limit);
+cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
+                              int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
+                              cudaStream_t stream, int sm_count, bool* handled);
 cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes,
                            const uint16_t* scales, int64_t N, int64_t K, int G, void* Y,
                            int y_bf16, uint32_t* d_err, cudaStream_t stream, int sm_count,
@@ -185,10 +188,17 @@ tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* sc
                                     d->smem_optin);
     if (e != cudaErrorNotSupported) return from_cuda(e);
     cudaGetLastError();
+    if (M > 4) {  // 5..64 tokens: the tensor-core small-M kernel
+        bool handled = false;
+        e = launch_gemm_small(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales), N,
+                              K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, &handled);
+        if (e != cudaSuccess) return from_cuda(e);
+        if (handled) return TQ_OK;
+    }
     e = launch_gemv_rows(static_cast<const uint16_t*>(X), M, codes,
-                                     static_cast<const uint16_t*>(scales), N, K, G, Y,
-                                     yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count,
-                                     d->smem_optin);
+                         static_cast<const uint16_t*>(scales), N, K, G, Y,
+                         yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count,
+                         d->smem_optin);
     if (e == cudaErrorInvalidValue) return TQ_ERR_UNSUPPORTED;
     return from_cuda(e);
 }
@@ -204,10 +214,15 @@ tq_status tq_gemm(const void* X, int64_t M, const uint8_t* codes, const void* sc
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
     bool handled = false;
-    cudaError_t e = launch_gemm_tc(static_cast<const uint16_t*>(X), M, codes,
-                                   static_cast<const uint16_t*>(scales), N, K, G, Y,
-                                   yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count,
-                                   &handled);
+    cudaError_t e = cudaSuccess;
+    if (M <= 64)
+        e = launch_gemm_small(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales), N,
+                              K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, &handled);
+    if (e == cudaSuccess && !handled)
+        e = launch_gemm_tc(static_cast<const uint16_t*>(X), M, codes,
+                           static_cast<const uint16_t*>(scales), N, K, G, Y,
+                           yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count,
+                           &handled);
     if (e != cudaSuccess) return from_cuda(e);
     if (!handled) return TQ_ERR_UNSUPPORTED;
     return TQ_OK;

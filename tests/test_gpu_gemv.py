@@ -106,3 +106,13 @@ def test_row_counts(N):
     W = synthetic.weights(N, K, index=N)
     X = synthetic.activations(1, K)
     check(X, W, G, dtypes=(torch.float32,))
+
+
+@pytest.mark.parametrize("M", [5, 15, 16, 17, 31, 32, 48, 64])
+@pytest.mark.parametrize("N,K,G", [(300, 1024, 128), (1536, 4096, 128), (257, 128, 64)])
+def test_small_m_tensor_path(M, N, K, G):
+    """5..64 tokens take the tensor-core small-M kernel (token tiles of 16, 32
+    or 64, K split across a cluster)."""
+    W = synthetic.weights(N, K, index=M * 7 + N)
+    X = synthetic.activations(M, K)
+    check(X, W, G)
