@@ -38,8 +38,8 @@ namespace cg = cooperative_groups;
 
 namespace tq {
 
-constexpr int kLutThreads = 256;
-constexpr int kLutWarps = kLutThreads / 32;
+// CTA size: 256 threads (two CTAs per SM, so a dependent launch can start
+// beside the running one) for small matrices, 512 for large ones.
 constexpr int kRB = 8;                 // rows per warp batch
 constexpr int kLPG = 13;               // lanes per group
 constexpr int kGPS = 2;                // groups per slice
@@ -56,6 +56,7 @@ struct LutPlan {
     int RB;       // row blocks (grid = RB * CS)
     int MT;       // tokens per launch
     int PER;      // rows reduced by each cluster rank = ceil(R / CS)
+    int THREADS;  // 256 (small matrices, two CTAs per SM) or 512
     size_t smem;
     size_t off_scale, off_acc, off_red;
 };
@@ -195,8 +196,9 @@ __device__ __forceinline__ void build_part(const LutArgs& a, float* tab, int sl,
         for (int k = 0; k < 9; ++k) c4[(9 * i + k) * 32] = P[k] + Q[i];
 }
 
-template <int B, int MT, int NS>
-__global__ void __launch_bounds__(kLutThreads, 2) gemv_lut_kernel(const LutArgs a) {
+template <int B, int MT, int NS, int kLutThreads>
+__global__ void __launch_bounds__(kLutThreads, 512 / kLutThreads) gemv_lut_kernel(const LutArgs a) {
+    constexpr int kLutWarps = kLutThreads / 32;
     constexpr int BPL = B / kLPG;
     constexpr int SLICE_BYTES = kGPS * B;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -377,6 +379,10 @@ static bool make_plan(int64_t N, int K, int G, int MT, int sm_count, size_t smem
     const int S = ng / kGPS;
     const size_t table_per_slice = (size_t)MT * BPL * kTableWords * 4;
     const int ns_max = MT == 4 ? 1 : (MT == 2 ? 2 : 4);
+    // Small matrices are latency-bound: keep two CTAs per SM.  Large ones
+    // amortize bigger resident tables with one 512-thread CTA per SM.
+    const bool big = (double)N * K > 16.0 * 1024 * 1024;
+    const size_t smem_cap = big ? smem_limit : (size_t)112 * 1024;
     double best_cost = -1;
     LutPlan best{};
     for (int cs = 1; cs <= 8; ++cs) {
@@ -385,7 +391,7 @@ static bool make_plan(int64_t N, int K, int G, int MT, int sm_count, size_t smem
         for (int ns = 1; ns <= per_cta && ns <= ns_max; ++ns) {
             if (per_cta % ns || ns == 3) continue;
             const size_t tbytes = table_per_slice * ns;
-            if (tbytes > 96 * 1024) continue;
+            if (tbytes > (big ? (size_t)160 * 1024 : (size_t)96 * 1024)) continue;
             int rb = sm_count / cs;
             if (rb < 1) rb = 1;
             int64_t R = (N + rb - 1) / rb;
@@ -398,7 +404,7 @@ static bool make_plan(int64_t N, int K, int G, int MT, int sm_count, size_t smem
             const size_t off_red = off_acc + (size_t)MT * RP * 4;
             const size_t smem = off_red + (size_t)cs * MT * PER * 4;
             // two CTAs per SM, so a dependent launch's CTAs can start beside this one's
-            if (smem > smem_limit || smem > 112 * 1024) continue;
+            if (smem > smem_cap) continue;
             // estimated cycles per CTA: table writes (one wavefront per 26 entries),
             // lookups (~1/20 cycle per byte per row), row reductions, cluster overhead
             const int passes = per_cta / ns;
@@ -425,13 +431,14 @@ static bool make_plan(int64_t N, int K, int G, int MT, int sm_count, size_t smem
         }
     }
     if (best_cost < 0) return false;
+    best.THREADS = big ? 512 : 256;
     *out = best;
     return true;
 }
 
-template <int B, int MT, int NS>
+template <int B, int MT, int NS, int T>
 static cudaError_t launch_lut(const LutArgs& a, cudaStream_t stream) {
-    auto kern = gemv_lut_kernel<B, MT, NS>;
+    auto kern = gemv_lut_kernel<B, MT, NS, T>;
     static std::atomic<int> smem_set{0};
     if ((int)a.p.smem > smem_set.load()) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)a.p.smem);
@@ -440,7 +447,7 @@ static cudaError_t launch_lut(const LutArgs& a, cudaStream_t stream) {
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.p.RB * a.p.CS));
-    cfg.blockDim = dim3(kLutThreads);
+    cfg.blockDim = dim3(T);
     cfg.dynamicSmemBytes = a.p.smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -455,15 +462,15 @@ static cudaError_t launch_lut(const LutArgs& a, cudaStream_t stream) {
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int B>
+template <int B, int T>
 static cudaError_t launch_lut_sel(const LutArgs& a, cudaStream_t stream) {
     const int ns = a.p.NS;
     switch (a.p.MT) {
-        case 4: return launch_lut<B, 4, 1>(a, stream);
-        case 2: return ns == 1 ? launch_lut<B, 2, 1>(a, stream) : launch_lut<B, 2, 2>(a, stream);
+        case 4: return launch_lut<B, 4, 1, T>(a, stream);
+        case 2: return ns == 1 ? launch_lut<B, 2, 1, T>(a, stream) : launch_lut<B, 2, 2, T>(a, stream);
         default:
-            return ns == 1 ? launch_lut<B, 1, 1>(a, stream)
-                           : (ns == 2 ? launch_lut<B, 1, 2>(a, stream) : launch_lut<B, 1, 4>(a, stream));
+            return ns == 1 ? launch_lut<B, 1, 1, T>(a, stream)
+                           : (ns == 2 ? launch_lut<B, 1, 2, T>(a, stream) : launch_lut<B, 1, 4, T>(a, stream));
     }
 }
 
@@ -480,9 +487,9 @@ cudaError_t launch_gemv_lut(const uint16_t* X, int64_t M, const uint8_t* codes, 
     if (B == 26 && (reinterpret_cast<uintptr_t>(codes) & 1)) return cudaErrorNotSupported;
     static const bool debug = getenv("TQ_DEBUG_PLAN") != nullptr;
     if (debug)
-        fprintf(stderr, "tq gemv_lut N=%lld K=%lld G=%d M=%lld: S=%d CS=%d NS=%d P=%d R=%d RB=%d smem=%zu\n",
+        fprintf(stderr, "tq gemv_lut N=%lld K=%lld G=%d M=%lld: S=%d CS=%d NS=%d P=%d R=%d RB=%d T=%d smem=%zu\n",
                 (long long)N, (long long)K, G, (long long)M, a.p.S, a.p.CS, a.p.NS, a.p.P, a.p.R, a.p.RB,
-                a.p.smem);
+                a.p.THREADS, a.p.smem);
     a.X = X;
     a.M = (int)M;
     a.m0 = 0;
@@ -496,7 +503,8 @@ cudaError_t launch_gemv_lut(const uint16_t* X, int64_t M, const uint8_t* codes, 
     a.Y = Y;
     a.y_bf16 = y_bf16;
     a.d_err = d_err;
-    return B == 26 ? launch_lut_sel<26>(a, stream) : launch_lut_sel<13>(a, stream);
+    if (a.p.THREADS == 512) return B == 26 ? launch_lut_sel<26, 512>(a, stream) : launch_lut_sel<13, 512>(a, stream);
+    return B == 26 ? launch_lut_sel<26, 256>(a, stream) : launch_lut_sel<13, 256>(a, stream);
 }
 
 }  // namespace tq
