@@ -13,6 +13,17 @@
 
 namespace tq {
 
+// PRMT selector byte of a digit d: the bf16 value of a weight is picked from
+// the 8 bytes {V, Z} = {-s, 0, +s, NaN}; digit d (d = t + 1) selects bytes
+// 2d and 2d+1, i.e. selector 0x10 + 0x22 d, and d = 3 (invalid) selects NaN.
+__device__ __forceinline__ uint32_t digit_selector(uint32_t d) { return 0x10u + 0x22u * d; }
+
+__device__ __forceinline__ uint32_t prmt32(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
 template <int G>
 __global__ void __launch_bounds__(256) unpack_pow2_kernel(
     const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales, int64_t num_groups,
@@ -21,8 +32,17 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
     constexpr int GPW = 32 / LPG;
     constexpr int B = bytes_per_group(G);
     constexpr int REAL = G - 5 * (B - 1);  // real digits in the last byte (1..5)
-    __shared__ uint16_t lut[256];
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) lut[b] = (uint16_t)byte_digit_pattern(b);
+    // byte -> selector bytes of its five digits (digit i in byte i of the entry)
+    __shared__ uint2 sel_lut[256];
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+        uint32_t sv[5];
+        uint32_t v = b;
+        for (int i = 0; i < 5; ++i) {
+            sv[i] = digit_selector(b >= 243 ? 3u : v % 3);
+            v /= 3;
+        }
+        sel_lut[b] = make_uint2(sv[0] | (sv[1] << 8) | (sv[2] << 16) | (sv[3] << 24), sv[4]);
+    }
     __syncthreads();
 
     const int lane = threadIdx.x & 31;
@@ -30,6 +50,7 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
     const int p0 = 8 * sub;
     const int q_first = p0 / 5;      // byte holding weight p0
     const int r_first = p0 - 5 * q_first;
+    const uint32_t shift = 8u * (uint32_t)r_first;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     uint32_t err_acc = 0;
@@ -37,14 +58,14 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
     for (int64_t base = warp * GPW; base < num_groups; base += nwarps * GPW) {
         const int64_t gi = base + lane / LPG;
         const bool active = gi < num_groups;
-        // weights p0..p0+7 lie in bytes q_first .. q_first+2 (at most three)
-        uint32_t pat[3] = {0x155u, 0x155u, 0x155u};
+        // weights p0..p0+7 lie in bytes q_first .. q_first+2 (the third only for its first digits)
+        uint32_t bv[3] = {kZeroByte, kZeroByte, kZeroByte};
         uint32_t s = 0;
         if (active) {
             const uint8_t* in = codes + gi * B;
 #pragma unroll
             for (int t = 0; t < 3; ++t)
-                if (q_first + t < B) pat[t] = lut[__ldcs(in + q_first + t)];
+                if (q_first + t < B) bv[t] = __ldcs(in + q_first + t);
             s = __ldg(scales + gi);
         }
         // validation of the bytes starting in [p0, p0+8)
@@ -53,8 +74,9 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
         for (int t = 0; t < 3; ++t) {
             const int q = q_first + t;
             if (5 * q >= p0 && 5 * q < p0 + 8 && q < B) {
-                if (pat[t] & 0x8000u) bad |= TQ_DERR_BYTE;
-                else if (q == B - 1 && (pat[t] & padding_mask(REAL)) != padding_ones(REAL))
+                if (bv[t] >= 243) bad |= TQ_DERR_BYTE;
+                else if (q == B - 1 && REAL < 5 &&
+                         (byte_digit_pattern(bv[t]) & padding_mask(REAL)) != padding_ones(REAL))
                     bad |= TQ_DERR_PADDING;
             }
         }
@@ -62,22 +84,25 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
         bad = seg_or_u32(bad, LPG);
         if (!active) bad = 0;
 
-        const uint32_t mag = (s == 0) ? 0u : scale_to_bf16_bits((uint16_t)s);
-        uint32_t w[8];
-        int t = 0, r = r_first;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t d = (pat[t] >> (2 * r)) & 3u;
-            w[i] = (d == 1u || mag == 0u) ? 0u : (mag | (d == 0u ? 0x8000u : 0u));
-            if (++r == 5) { r = 0; ++t; }
-        }
+        // selector bytes of the lane's 8 digits: stream s0.. = digits of bv[0], bv[1], bv[2]
+        const uint2 e0 = sel_lut[bv[0]], e1 = sel_lut[bv[1]], e2 = sel_lut[bv[2]];
+        const uint32_t w0 = e0.x;                                          // s0..s3
+        const uint32_t w1 = prmt32(e0.y, e1.x, 0x6540u);                   // s4..s7
+        const uint32_t w2 = prmt32(prmt32(e1.x, e1.y, 0x4343u), e2.x, 0x5410u);  // s8..s11
+        const uint32_t o0 = __funnelshift_rc(w0, w1, shift);               // selectors of weights 0..3
+        const uint32_t o1 = __funnelshift_rc(w1, w2, shift);               // weights 4..7
+
+        uint32_t V, Z;  // {-s, 0} and {+s, NaN}
         if (bad) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) w[i] = kBf16NaN;
+            V = Z = 0x7FC07FC0u;
+        } else {
+            const uint32_t mag = (s == 0) ? 0u : scale_to_bf16_bits((uint16_t)s);
+            V = mag ? (mag | 0x8000u) : 0u;
+            Z = mag | 0x7FC00000u;
         }
         if (active) {
-            uint4 o = make_uint4(w[0] | (w[1] << 16), w[2] | (w[3] << 16), w[4] | (w[5] << 16),
-                                 w[6] | (w[7] << 16));
+            const uint4 o = make_uint4(prmt32(V, Z, o0), prmt32(V, Z, o0 >> 16), prmt32(V, Z, o1),
+                                       prmt32(V, Z, o1 >> 16));
             __stcs(reinterpret_cast<uint4*>(out + gi * G + p0), o);
             if (sub == 0) err_acc |= bad;
         }
