@@ -117,6 +117,12 @@ TQ_API tq_status tq_unpack_bf16(const uint8_t *codes, const void *scales_f16, in
  * (fp32: 4-byte aligned, bf16: 2-byte aligned), must not overlap the inputs.
  * workspace: at least tq_workspace_bytes(M, N, K, G) bytes of device scratch
  * (NULL allowed when that is 0), 256-byte aligned.
+ * Ordering: the kernels are launched as programmatic dependents of the work
+ * before them on `stream`.  X is read only after that work has completed;
+ * codes and scales (the weights) may be read while it is still finishing, so
+ * they must not be written by the kernel launched immediately before this
+ * call on the same stream (write them earlier, or on another stream and
+ * join with an event).
  */
 TQ_API tq_status tq_gemv(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
                   int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,

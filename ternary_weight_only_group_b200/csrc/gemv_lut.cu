@@ -123,22 +123,6 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[RB]) {
     return v[0];
 }
 
-// Row rescan for the error bits of a NaN output row (rare path).
-__device__ uint32_t scan_row_errors(const uint8_t* crow, const uint16_t* srow, int ng, int G, int B) {
-    const int real = G - 5 * (B - 1);
-    const uint32_t pm = padding_mask(real), po = padding_ones(real);
-    uint32_t bad = 0;
-    for (int g = 0; g < ng; ++g) {
-        if (scale_is_bad(srow[g])) bad |= TQ_DERR_SCALE;
-        for (int q = 0; q < B; ++q) {
-            const uint32_t p = byte_digit_pattern(crow[g * B + q]);
-            if (p & 0x8000u) bad |= TQ_DERR_BYTE;
-            else if (q == B - 1 && (p & pm) != po) bad |= TQ_DERR_PADDING;
-        }
-    }
-    return bad;
-}
-
 // Writes the entries b = 81*d4 + [0, 81) of this lane's chunk table (d4 =
 // part), or the 13 entries 243..255 (part == 3, always NaN).  With
 // b = d0 + 3 d1 + 9 d2 + 27 d3 + 81 d4, entry(b) = P[d0 + 3 d1] + Q[d2 + 3 d3]
@@ -166,7 +150,7 @@ __device__ __forceinline__ void build_part(const LutArgs& a, float* tab, int sl,
     const int real = min(5, a.G - 5 * q);
 #pragma unroll
     for (int i = 0; i < 5; ++i)
-        if (i < real) x[i] = bf16_bits_to_f32(__ldg(xr + i));
+        if (i < real) x[i] = bf16_bits_to_f32(__ldcg(xr + i));  // written by the preceding kernel: bypass L1
     const int d4 = part;
     const bool bad4 = (4 >= real) && d4 != 1;
     const float h4 = (float)(d4 - 1) * x[4];
@@ -286,14 +270,24 @@ __global__ void __launch_bounds__(kLutThreads, 512 / kLutThreads) gemv_lut_kerne
                 }
                 const float tot = transpose_reduce<kRB>(acc[m]);
                 if (lane < kRB && r0 + lane < nrows) {
-                    float* dst = acc_s + m * p.RP + r0 + lane;
-                    *dst = (pass == 0) ? tot : *dst + tot;
+                    const int r = r0 + lane;
+                    if (p.P == 1) {  // single pass: straight to the owner rank (no block barrier)
+                        const int q = r / p.PER;
+                        float* dst = cluster.map_shared_rank(red, q);
+                        dst[(crank * MT + m) * p.PER + (r - q * p.PER)] = tot;
+                    } else {
+                        float* dst = acc_s + m * p.RP + r;
+                        *dst = (pass == 0) ? tot : *dst + tot;
+                    }
                 }
             }
         };
 
         uint32_t cwA[NS][kRB], cwB[NS][kRB];
-        if (warp < nbatch) load_batch(warp, cwA);  // code bytes do not depend on earlier kernels
+        // Code bytes do not depend on earlier kernels: request this warp's first
+        // two batches before waiting for the activations.
+        if (warp < nbatch) load_batch(warp, cwA);
+        if (warp + kLutWarps < nbatch) load_batch(warp + kLutWarps, cwB);
 
         // decoded scales of this pass: ssc[gl][r]
         for (int r = threadIdx.x; r < p.RP; r += kLutThreads) {
@@ -332,12 +326,13 @@ __global__ void __launch_bounds__(kLutThreads, 512 / kLutThreads) gemv_lut_kerne
         int bt = warp;
         while (bt < nbatch) {
             const int b1 = bt + kLutWarps;
-            if (b1 < nbatch) load_batch(b1, cwB);
-            run_batch(bt, cwA);
+            run_batch(bt, cwA);  // cwB (batch b1) is already in flight
             if (b1 >= nbatch) break;
             const int b2 = b1 + kLutWarps;
             if (b2 < nbatch) load_batch(b2, cwA);
             run_batch(b1, cwB);
+            const int b3 = b2 + kLutWarps;
+            if (b3 < nbatch) load_batch(b3, cwB);
             bt = b2;
         }
     }
@@ -345,12 +340,14 @@ __global__ void __launch_bounds__(kLutThreads, 512 / kLutThreads) gemv_lut_kerne
     // Cluster reduction: every rank pushes its partial rows into the owner
     // rank's buffer (rows [q*PER, (q+1)*PER) belong to rank q), one cluster
     // barrier, then each owner adds the CS partials in rank order.
-    __syncthreads();
-    for (int i = threadIdx.x; i < nrows * MT; i += kLutThreads) {
-        const int m = i / nrows, r = i - m * nrows;
-        const int q = r / p.PER;
-        float* dst = cluster.map_shared_rank(red, q);
-        dst[(crank * MT + m) * p.PER + (r - q * p.PER)] = acc_s[m * p.RP + r];
+    if (p.P > 1) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < nrows * MT; i += kLutThreads) {
+            const int m = i / nrows, r = i - m * nrows;
+            const int q = r / p.PER;
+            float* dst = cluster.map_shared_rank(red, q);
+            dst[(crank * MT + m) * p.PER + (r - q * p.PER)] = acc_s[m * p.RP + r];
+        }
     }
     cluster.sync();
     const int rlo = crank * p.PER, rhi = min(nrows, rlo + p.PER);

@@ -21,6 +21,9 @@ cudaError_t launch_gemv_rows(const uint16_t* X, int64_t M, const uint8_t* codes,
 cudaError_t launch_gemv_lut(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                             int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                             cudaStream_t stream, int sm_count, size_t smem_limit);
+cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
+                                  int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
+                                  cudaStream_t stream, int sm_count);
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                               int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                               cudaStream_t stream, int sm_count, bool* handled);
@@ -182,7 +185,13 @@ tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* sc
     if (K == 0) return TQ_ERR_UNSUPPORTED;
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
-    cudaError_t e = launch_gemv_lut(static_cast<const uint16_t*>(X), M, codes,
+    // M == 1, small matrix: weights decoded before the activations are awaited
+    cudaError_t e = launch_gemv_predecode(static_cast<const uint16_t*>(X), M, codes,
+                                          static_cast<const uint16_t*>(scales), N, K, G, Y, yt == TQ_OUT_BF16,
+                                          d_err, (cudaStream_t)stream, d->sm_count);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+    cudaGetLastError();
+    e = launch_gemv_lut(static_cast<const uint16_t*>(X), M, codes,
                                     static_cast<const uint16_t*>(scales), N, K, G, Y,
                                     yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count,
                                     d->smem_optin);

@@ -10,7 +10,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-#include "../../include/tq.h"
+#include "tq.h"
 
 namespace tq {
 
@@ -142,5 +142,59 @@ __device__ __forceinline__ uint32_t byte_digit_pattern(uint32_t b) {
 // Digit pattern of a canonical last byte: digits >= `real` are all 1.
 __host__ __device__ constexpr uint32_t padding_mask(int real) { return 0x3FFu & ~((1u << (2 * real)) - 1u); }
 __host__ __device__ constexpr uint32_t padding_ones(int real) { return 0x155u & padding_mask(real); }
+
+// PRMT selector byte of a digit d: the bf16 value of a weight is picked from
+// the 8 bytes {V, Z} = {-s, 0, +s, NaN}; digit d (d = t + 1) selects bytes
+// 2d and 2d+1, i.e. selector 0x10 + 0x22 d, and d = 3 (invalid) selects NaN.
+__device__ __forceinline__ uint32_t digit_selector(uint32_t d) { return 0x10u + 0x22u * d; }
+
+__device__ __forceinline__ uint32_t prmt32(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
+// Selector bytes of the 8 consecutive weights p0 .. p0+7 of a group (p0 % 8
+// == 0) from the code bytes b0, b1, b2 holding them (weight p0 is digit
+// r = p0 % 5 of b0) and a byte -> selectors table; invalid bytes select NaN.
+__device__ __forceinline__ void eight_selectors(const uint2* sel_lut, uint32_t b0, uint32_t b1, uint32_t b2,
+                                                uint32_t shift, uint32_t& o0, uint32_t& o1) {
+    const uint2 e0 = sel_lut[b0], e1 = sel_lut[b1], e2 = sel_lut[b2];
+    const uint32_t w0 = e0.x;                                                // s0..s3
+    const uint32_t w1 = prmt32(e0.y, e1.x, 0x6540u);                         // s4..s7
+    const uint32_t w2 = prmt32(prmt32(e1.x, e1.y, 0x4343u), e2.x, 0x5410u);  // s8..s11
+    o0 = __funnelshift_rc(w0, w1, shift);
+    o1 = __funnelshift_rc(w1, w2, shift);
+}
+
+// Fills a byte -> selector-bytes table (digit i in byte i) for the {-s, 0, +s, NaN} layout.
+__device__ __forceinline__ void fill_digit_selector_lut(uint2* sel_lut, int tid, int nthreads) {
+    for (int b = tid; b < 256; b += nthreads) {
+        uint32_t sv[5];
+        uint32_t v = b;
+        for (int i = 0; i < 5; ++i) {
+            sv[i] = digit_selector(b >= 243 ? 3u : v % 3);
+            v /= 3;
+        }
+        sel_lut[b] = make_uint2(sv[0] | (sv[1] << 8) | (sv[2] << 16) | (sv[3] << 24), sv[4]);
+    }
+}
+
+// Error bits of one weight row (its ng groups of B code bytes and ng scales);
+// the GEMV kernels call it only for an output row that came out NaN.
+static __device__ __noinline__ uint32_t scan_row_errors(const uint8_t* crow, const uint16_t* srow, int ng, int G, int B) {
+    const int real = G - 5 * (B - 1);
+    const uint32_t pm = padding_mask(real), po = padding_ones(real);
+    uint32_t bad = 0;
+    for (int g = 0; g < ng; ++g) {
+        if (scale_is_bad(srow[g])) bad |= TQ_DERR_SCALE;
+        for (int q = 0; q < B; ++q) {
+            const uint32_t p = byte_digit_pattern(crow[g * B + q]);
+            if (p & 0x8000u) bad |= TQ_DERR_BYTE;
+            else if (q == B - 1 && (p & pm) != po) bad |= TQ_DERR_PADDING;
+        }
+    }
+    return bad;
+}
 
 }  // namespace tq

@@ -13,17 +13,6 @@
 
 namespace tq {
 
-// PRMT selector byte of a digit d: the bf16 value of a weight is picked from
-// the 8 bytes {V, Z} = {-s, 0, +s, NaN}; digit d (d = t + 1) selects bytes
-// 2d and 2d+1, i.e. selector 0x10 + 0x22 d, and d = 3 (invalid) selects NaN.
-__device__ __forceinline__ uint32_t digit_selector(uint32_t d) { return 0x10u + 0x22u * d; }
-
-__device__ __forceinline__ uint32_t prmt32(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t r;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
-    return r;
-}
-
 template <int G>
 __global__ void __launch_bounds__(256) unpack_pow2_kernel(
     const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales, int64_t num_groups,
@@ -32,17 +21,8 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
     constexpr int GPW = 32 / LPG;
     constexpr int B = bytes_per_group(G);
     constexpr int REAL = G - 5 * (B - 1);  // real digits in the last byte (1..5)
-    // byte -> selector bytes of its five digits (digit i in byte i of the entry)
     __shared__ uint2 sel_lut[256];
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
-        uint32_t sv[5];
-        uint32_t v = b;
-        for (int i = 0; i < 5; ++i) {
-            sv[i] = digit_selector(b >= 243 ? 3u : v % 3);
-            v /= 3;
-        }
-        sel_lut[b] = make_uint2(sv[0] | (sv[1] << 8) | (sv[2] << 16) | (sv[3] << 24), sv[4]);
-    }
+    fill_digit_selector_lut(sel_lut, threadIdx.x, blockDim.x);
     __syncthreads();
 
     const int lane = threadIdx.x & 31;
@@ -84,14 +64,8 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
         bad = seg_or_u32(bad, LPG);
         if (!active) bad = 0;
 
-        // selector bytes of the lane's 8 digits: stream s0.. = digits of bv[0], bv[1], bv[2]
-        const uint2 e0 = sel_lut[bv[0]], e1 = sel_lut[bv[1]], e2 = sel_lut[bv[2]];
-        const uint32_t w0 = e0.x;                                          // s0..s3
-        const uint32_t w1 = prmt32(e0.y, e1.x, 0x6540u);                   // s4..s7
-        const uint32_t w2 = prmt32(prmt32(e1.x, e1.y, 0x4343u), e2.x, 0x5410u);  // s8..s11
-        const uint32_t o0 = __funnelshift_rc(w0, w1, shift);               // selectors of weights 0..3
-        const uint32_t o1 = __funnelshift_rc(w1, w2, shift);               // weights 4..7
-
+        uint32_t o0, o1;  // selector bytes of the lane's 8 weights
+        eight_selectors(sel_lut, bv[0], bv[1], bv[2], shift, o0, o1);
         uint32_t V, Z;  // {-s, 0} and {+s, NaN}
         if (bad) {
             V = Z = 0x7FC07FC0u;

@@ -62,16 +62,18 @@ def test_msweep_shapes(name, M):
     check(X, W, 128, dtypes=(torch.float32,))
 
 
+@pytest.mark.parametrize("M", [1, 3])
 @pytest.mark.parametrize("G", [1, 5, 8, 40, 64, 100, 128, 256, 4096])
-def test_group_sizes_and_ragged_rows(G):
+def test_group_sizes_and_ragged_rows(G, M):
     K = G * max(2, 1024 // G)
     N = 77
     W = synthetic.weights(N, K, index=G + 50, outlier_frac=1e-3)
-    X = synthetic.activations(3, K)
+    X = synthetic.activations(M, K)
     check(X, W, G)
 
 
-def test_rejected_groups_give_nan_rows():
+@pytest.mark.parametrize("M", [1, 2])
+def test_rejected_groups_give_nan_rows(M):
     G, N, K = 64, 40, 512
     W = synthetic.weights(N, K, index=12)
     codes, scales, _ = oracle.quantize_pack(W, G)
@@ -80,18 +82,19 @@ def test_rejected_groups_give_nan_rows():
     scales[11, 5] = 0x7C00        # Inf scale
     scales[13, 0] = 0x8001        # negative scale
     scales[17, 3] = 0             # zero group: finite result
-    X = synthetic.activations(2, K)
+    X = synthetic.activations(M, K)
     ref = check(X, W, G, codes=codes, scales=scales)
     assert np.all(np.isnan(ref[:, [3, 7, 11, 13]])) and np.all(np.isfinite(ref[:, 17]))
 
 
-def test_unaligned_codes_pointer():
+@pytest.mark.parametrize("M", [1, 2])
+def test_unaligned_codes_pointer(M):
     """Codes starting at an odd address are still served (the 16-bit code
     loads are not used then)."""
     G, N, K = 128, 300, 1024
     W = synthetic.weights(N, K, index=21)
     codes, scales, _ = oracle.quantize_pack(W, G)
-    X = synthetic.activations(1, K)
+    X = synthetic.activations(M, K)
     ref = oracle.linear(X, codes, scales, N, K, G)
     buf = torch.zeros(codes.size + 1, dtype=torch.uint8, device="cuda")
     buf[1:] = to_dev_u8(codes.reshape(-1))
@@ -106,6 +109,17 @@ def test_row_counts(N):
     W = synthetic.weights(N, K, index=N)
     X = synthetic.activations(1, K)
     check(X, W, G, dtypes=(torch.float32,))
+
+
+@pytest.mark.parametrize("N,K,G", [(9477, 512, 64), (2000, 512, 32), (150, 4096, 256), (1500, 3072, 8),
+                                   (700, 2048, 128), (300, 1024, 16)])
+def test_predecode_row_batches(N, K, G):
+    """One token over matrices whose per-CTA rows fit in shared memory: more
+    than eight 8-row batches per CTA, chunks split over two to eight warps,
+    ragged last CTA."""
+    W = synthetic.weights(N, K, index=N + K)
+    X = synthetic.activations(1, K)
+    check(X, W, G)
 
 
 @pytest.mark.parametrize("M", [5, 15, 16, 17, 31, 32, 48, 64])
