@@ -36,6 +36,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "ternary x bf16 GEMV HBM GB/s (% of peak); prefill GEMM TFLOP/s; pack GB/s"
 FFN = {"gate": (3584, 1024), "up": (3584, 1024), "down": (1024, 3584)}
+MSWEEP = {"q": (1536, 1536), "o": (1536, 1536), "gate": (4096, 1536), "up": (4096, 1536), "down": (1536, 4096)}
+MSWEEP_LAYERS = 28
+MSWEEP_M = (1, 2, 4, 8, 16, 32, 64)
 GROUPS = (64, 128)
 LAYERS = 48
 L2_BYTES = 126 * 1024 * 1024
@@ -266,6 +269,7 @@ def run_ours(args, rank, world, local):
         results["stream"] = bench_gemv_stream(tq, args, world, peaks)
         results["pack"], results["unpack"] = bench_bulk_codec(tq, args, world, peaks)
         results["prefill"] = bench_prefill(tq, args, world, peaks)
+        results["msweep"] = bench_msweep(tq, args, world, peaks)
     clk = clocks.summary()
 
     ms_step = ms / K_steps
@@ -317,6 +321,7 @@ def run_ours(args, rank, world, local):
         "pack": results["pack"],
         "unpack": results["unpack"],
         "prefill_gemm": results["prefill"],
+        "msweep": results["msweep"],
     }
     print(json.dumps(line), flush=True)
 
@@ -370,6 +375,48 @@ def bench_gemv_shapes(tq, args, world, peaks):
             res[f"{name}{N}x{K}_G{G}"] = {"us": round(us, 2), "GB/s": round(byts / us / 1e3, 1),
                                            "launches": max(3, args.steps) * len(packs)}
             del packs
+    return res
+
+
+def bench_msweep(tq, args, world, peaks):
+    """M-sweep over a 28-layer stack of q, o (1536x1536), gate, up (4096x1536)
+    and down (1536x4096), G=128: one step = the 140 tq_gemv launches of one
+    token batch of M rows, replayed from a CUDA graph (packed weights 144.5 MB,
+    larger than L2).  Reports GB/s on the algorithmic bytes and TFLOP/s."""
+    import torch
+    G = 128
+    packs = []
+    for l in range(MSWEEP_LAYERS):
+        for i, (name, (N, K)) in enumerate(MSWEEP.items()):
+            W = device_weights(N, K, seed=9000 + 5 * l + i, outliers=False)
+            packs.append((N, K) + tq.quantize_pack(W, G))
+            del W
+    wbytes = sum(packed_bytes(N, K, G) for (N, K, _, _) in packs)
+    flops1 = sum(2 * N * K for (N, K, _, _) in packs)
+    res = {}
+    for M in MSWEEP_M:
+        Xs = {K: device_acts(M, K, seed=9500 + K) for K in {k for (_, k, _, _) in packs}}
+        Ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for N in {n for (n, _, _, _) in packs}}
+
+        def step():
+            for (N, K, c, s_) in packs:
+                tq.gemv(Xs[K], c, s_, N, K, G, out=Ys[N])
+        step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+            step()
+        steps = max(3, args.steps // 5)
+        ms = timed(graph.replay, steps, max(3, args.warmup), world)
+        us = ms * 1e3 / steps
+        byts = wbytes + sum(2 * M * (K + N) for (N, K, _, _) in packs)
+        gbs = byts / us / 1e3
+        tfs = flops1 * M / us / 1e6
+        bound = min(peaks["hbm_gbs"] * (flops1 * M / byts) / 1e3, peaks["bf16_tflops"])
+        res[f"M{M}"] = {"us": round(us, 1), "GB/s": round(gbs, 1), "TFLOP/s": round(tfs, 2),
+                        "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "roofline_TFLOP/s": round(bound, 1),
+                        "frac_roofline": round(tfs / bound, 4), "launches": steps * len(packs)}
+        del graph
     return res
 
 
@@ -525,7 +572,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
-    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv"], default=None,
+    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv", "msweep"], default=None,
                     help="run one sub-benchmark alone and print its result (profiling aid)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -541,7 +588,7 @@ def main():
             torch.cuda.set_device(local)
             peaks = load_peaks()
             fn = {"stream": bench_gemv_stream, "codec": bench_bulk_codec, "prefill": bench_prefill,
-                  "gemv": bench_gemv_shapes}
+                  "gemv": bench_gemv_shapes, "msweep": bench_msweep}
             res = fn[args.only](tq, args, world, peaks)
             if rank == 0:
                 print(json.dumps({"only": args.only, "result": res}), flush=True)

@@ -65,15 +65,6 @@ struct Params {
     int y_bf16;
 };
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
 template <int NT, bool CODES_TMA>
 __global__ void __launch_bounds__(kThreads, 1) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                  const __grid_constant__ CUtensorMap tmap_c,
@@ -239,17 +230,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_small_kernel(const __grid_co
     tc_fence_after();
     // owner: rows [crank*RPQ, (crank+1)*RPQ) of the tile, all tokens
     const int64_t Mv = p.M < NT ? p.M : NT;
+    uint32_t err_acc = 0;
     for (int i = threadIdx.x; i < RPQ * Mv; i += kThreads) {
         const int m = i / RPQ, rr = i - m * RPQ;
         float acc = 0.f;
         for (int qr = 0; qr < p.CS; ++qr) acc += sm.red[(qr * RPQ + rr) * NT + m];
         const int64_t n = n0 + crank * RPQ + rr;
         if (n < p.N) {
+            if (m == 0 && acc != acc)  // NaN output of the first token: rescan that W row
+                err_acc |= scan_row_errors(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G, p.B);
             const int64_t o = (int64_t)m * p.N + n;
             if (p.y_bf16) reinterpret_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(acc);
             else reinterpret_cast<float*>(p.Y)[o] = acc;
         }
     }
+
+    if (err_acc && p.d_err) atomicOr(p.d_err, err_acc);
 
     // ---------------- teardown
     tc_fence_before();
@@ -294,8 +290,11 @@ static cudaError_t launch_nt(const CUtensorMap& tx, const CUtensorMap& tc_, cons
 
 }  // namespace small
 
-// Covered shapes: 1 <= M <= 64, K % 64 == 0, G % 64 == 0, code rows a
-// multiple of 16 bytes with a 16-byte aligned base.  Otherwise *handled is
+cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
+                               int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
+                               cudaStream_t stream, int sm_count, bool* handled);
+
+// Covered shapes: 1 <= M <= 64, K % 64 == 0, G % 64 == 0.  Otherwise *handled is
 // left false and nothing is launched.
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                               int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
@@ -324,6 +323,8 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     // split K so the grid covers the SMs, keeping at least two stages per CTA
     int CS = 1;
     while (CS < kMaxCS && tiles * CS * 2 <= sm_count && nk / (CS * 2) >= 2) CS *= 2;
+    if (CS == 1)  // no K split: the persistent kernel walks the tiles
+        return launch_gemm_stream(X, M, codes, scales, N, K, G, Y, y_bf16, d_err, stream, sm_count, handled);
     Params p{};
     p.codes = codes;
     p.row_bytes = row_bytes;

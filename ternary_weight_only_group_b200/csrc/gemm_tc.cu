@@ -21,7 +21,8 @@
 // its five weights; one PRMT gathers the selectors of a weight pair, a second
 // PRMT picks the pair's bf16 values among {+s, -s, 0, NaN}.  Invalid bytes,
 // non-canonical padding and bad scales decode to NaN (the row's outputs are
-// then NaN, as the decoder defines).
+// then NaN, as the decoder defines); the W rows behind NaN outputs of the
+// first X row are rescanned for the error bits.
 // Every mbarrier wait is bounded by a %globaltimer deadline; a timeout sets
 // TQ_DERR_TIMEOUT, stops issuing work, drains what is in flight, frees tensor
 // memory and returns.
@@ -202,6 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         // ---------------- epilogue: warps 4..7 read their accumulator quadrant
         if (warp < kDecodeWarp0 + 4) {
             const int q = warp - kDecodeWarp0;  // TMEM lanes 32q .. 32q+31
+            uint32_t err_acc = 0;
             const bool ok = mbar_wait(&sm.done, 0, abort_flag);
             tc_fence_after();
             if (ok) {
@@ -213,6 +215,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                         const int64_t nb = n0 + 32 * c;
                         if (m < p.M && nb < p.N) {
                             const int cnt = (int)(p.N - nb < 32 ? p.N - nb : 32);
+                            if (m == 0) {  // a NaN output of the first X row: rescan that W row's groups
+#pragma unroll
+                                for (int j = 0; j < 32; ++j)
+                                    if (j < cnt && __uint_as_float(r[j]) != __uint_as_float(r[j]))
+                                        err_acc |= scan_row_errors(p.codes + (nb + j) * p.row_bytes,
+                                                                   p.scales + (nb + j) * p.ng, p.ng, p.G, p.B);
+                            }
                             if (p.y_bf16) {
                                 __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.Y) + m * p.N + nb;
                                 if (cnt == 32 && p.y_vec) {
@@ -251,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                     }
                 }
             }
+            if (err_acc && p.d_err) atomicOr(p.d_err, err_acc);
         }
     }
 

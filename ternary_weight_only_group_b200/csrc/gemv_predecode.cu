@@ -3,7 +3,8 @@
 //
 // Y[n] = sum_k X[k] * What[n][k] with What = t * RNE_bf16(scale) (tiny-llm
 // "Week 2 Day 3: Quantize the Model", "Mathematical Formulation"; the
-// decoding of "precisit/pack-unpack-run", codec.py), fp32 accumulation, M = 1.
+// decoding of "precisit/pack-unpack-run", codec.py), fp32 accumulation,
+// 1 <= M <= 4 tokens.
 //
 // In a chain of dependent layers a kernel's weights are known long before its
 // activations.  Each CTA (one per SM, R rows) therefore stages its codes and
@@ -11,8 +12,10 @@
 // BEFORE griddepcontrol.wait, while the previous kernels are still running
 // (up to three CTAs share an SM, so two later launches decode while one
 // computes).  After the wait only the activation load, one mixed-precision
-// FMA per weight (bf16 inputs, fp32 accumulator), a transposing butterfly
-// per eight rows and the stores remain: no tables, no cluster barrier.
+// FMA per weight and token (bf16 inputs, fp32 accumulator), a transposing
+// butterfly per eight rows and token and the stores remain: no tables, no
+// cluster barrier.  When one CTA per SM would need more shared memory than
+// fits, two CTAs per SM take half the rows each (less overlap).
 //
 // Decode: one lane per 64 weights of a group (a whole group when G <= 64).
 // Code byte i of the lane's window contributes its five PRMT selector bytes
@@ -65,9 +68,11 @@ __device__ const PdSelectorTables kPdSelectors;
 // chunk (< 16) plus the range, rounded to 16.
 __host__ __device__ constexpr int pd_codes_area(int n) { return (n + 16 + 15) & ~15; }
 
-// Shared memory: [selector tables, later the activations] | R x K decoded
-// bf16 (swizzled chunks) | staged codes | staged scales.
-__host__ __device__ constexpr int pd_head_bytes(int K) { return K * 2 > kPdTableBytes ? K * 2 : kPdTableBytes; }
+// Shared memory: [selector tables, later the MT x K activations] | R x K
+// decoded bf16 (swizzled chunks) | staged codes | staged scales.
+__host__ __device__ constexpr int pd_head_bytes(int K, int MT) {
+    return MT * K * 2 > kPdTableBytes ? MT * K * 2 : kPdTableBytes;
+}
 
 template <int RB>
 __device__ __forceinline__ float pd_transpose_reduce(float (&v)[RB]) {
@@ -140,9 +145,9 @@ __device__ __forceinline__ float fma_bf16(uint16_t a, uint16_t b, float c) {
 // chunks; both are free of bank conflicts this way.
 __device__ __forceinline__ int pd_swizzle(int c) { return c ^ ((c >> 3) & 7); }
 
-template <int G>
-__global__ void __launch_bounds__(kPdThreads, 3) gemv_predecode_kernel(
-    const uint16_t* __restrict__ X, const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
+template <int G, int MT>
+__global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_kernel(
+    const uint16_t* __restrict__ X, int M, const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
     int64_t N, int K, int R, void* __restrict__ Y, int y_bf16, uint32_t* __restrict__ d_err) {
     constexpr int B = bytes_per_group(G);
     constexpr int REAL = G - 5 * (B - 1);   // real digits in a group's last byte
@@ -157,9 +162,9 @@ __global__ void __launch_bounds__(kPdThreads, 3) gemv_predecode_kernel(
     constexpr uint32_t PAD_BASE = REAL == 1 ? 120u : (REAL == 2 ? 117u : (REAL == 3 ? 108u : 81u));
 
     extern __shared__ __align__(16) unsigned char smem[];
-    __shared__ float red[kPdWarps * 8];  // slice sums when the chunks are split over warps
+    __shared__ float red[kPdWarps * 8 * MT];  // slice sums when the chunks are split over warps
     const uint2* tabs = reinterpret_cast<const uint2*>(smem);  // [4][256]
-    uint16_t* w = reinterpret_cast<uint16_t*>(smem + pd_head_bytes(K));  // [R][K] decoded bf16
+    uint16_t* w = reinterpret_cast<uint16_t*>(smem + pd_head_bytes(K, MT));  // [R][K] decoded bf16
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t row0 = (int64_t)blockIdx.x * R;
@@ -170,7 +175,7 @@ __global__ void __launch_bounds__(kPdThreads, 3) gemv_predecode_kernel(
     // ---- stage the selector tables and this CTA's codes and scales (its rows
     // are contiguous) in one round of copies
     const int ngroups = nrows * ng;
-    unsigned char* raw = smem + pd_head_bytes(K) + (size_t)R * K * 2;
+    unsigned char* raw = smem + pd_head_bytes(K, MT) + (size_t)R * K * 2;
     for (int i = threadIdx.x; i < kPdTableBytes / 16; i += kPdThreads)
         cp_async16(smem + 16 * i, reinterpret_cast<const unsigned char*>(&kPdSelectors) + 16 * i);
     const unsigned char* craw = stage_bytes(raw, codes + row0 * ng * B, ngroups * B, threadIdx.x, kPdThreads);
@@ -231,18 +236,19 @@ __global__ void __launch_bounds__(kPdThreads, 3) gemv_predecode_kernel(
     const int nchunk = K / 8;  // 8-column chunks
     __syncthreads();
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    uint4* xs = reinterpret_cast<uint4*>(smem);
-    for (int c0 = 0; c0 < nchunk; c0 += 4 * kPdThreads) {
+    uint4* xs = reinterpret_cast<uint4*>(smem);  // [MT][nchunk]; tokens past M are zero
+    for (int c0 = 0; c0 < MT * nchunk; c0 += 4 * kPdThreads) {
         uint4 xv[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int c = c0 + threadIdx.x + j * kPdThreads;
-            if (c < nchunk) xv[j] = __ldcg(reinterpret_cast<const uint4*>(X) + c);
+            xv[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (c < M * nchunk) xv[j] = __ldcg(reinterpret_cast<const uint4*>(X) + c);
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int c = c0 + threadIdx.x + j * kPdThreads;
-            if (c < nchunk) xs[c] = xv[j];
+            if (c < MT * nchunk) xs[c] = xv[j];
         }
     }
     __syncthreads();
@@ -259,13 +265,22 @@ __global__ void __launch_bounds__(kPdThreads, 3) gemv_predecode_kernel(
         int roff[8];  // element offset of each row (rows past the end repeat the last, never stored)
 #pragma unroll
         for (int i = 0; i < 8; ++i) roff[i] = min(rb0 + i, nrows - 1) * K;
-        float acc[8];
+        float acc[MT][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        for (int m = 0; m < MT; ++m)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[m][i] = 0.f;
 #pragma unroll 2
         for (int c = lane + 32 * sl; c < nchunk; c += 32 * ks) {
-            const uint4 xv = xs[c];
-            const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
+            uint32_t xx[MT][4];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const uint4 xv = xs[m * nchunk + c];
+                xx[m][0] = xv.x;
+                xx[m][1] = xv.y;
+                xx[m][2] = xv.z;
+                xx[m][3] = xv.w;
+            }
             const int pc8 = 8 * pd_swizzle(c);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -273,22 +288,30 @@ __global__ void __launch_bounds__(kPdThreads, 3) gemv_predecode_kernel(
                 const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    acc[i] = fma_bf16((uint16_t)ww[h], (uint16_t)xx[h], acc[i]);
-                    acc[i] = fma_bf16((uint16_t)(ww[h] >> 16), (uint16_t)(xx[h] >> 16), acc[i]);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        acc[m][i] = fma_bf16((uint16_t)ww[h], (uint16_t)xx[m][h], acc[m][i]);
+                        acc[m][i] = fma_bf16((uint16_t)(ww[h] >> 16), (uint16_t)(xx[m][h] >> 16), acc[m][i]);
+                    }
                 }
             }
         }
-        const float tot = pd_transpose_reduce<8>(acc);
+        float tot[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) tot[m] = pd_transpose_reduce<8>(acc[m]);
         if (lane < 8) {
+            const int rr = rb0 + lane;
             if (ks == 1) {
-                const int rr = rb0 + lane;
                 if (rr < nrows) {
-                    if (tot != tot)
+                    if (tot[0] != tot[0])
                         err_acc |= scan_row_errors(codes + (row0 + rr) * ng * B, scales + (row0 + rr) * ng, ng, G, B);
-                    store_y(Y, y_bf16, row0 + rr, tot);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        if (m < M) store_y(Y, y_bf16, (int64_t)m * N + row0 + rr, tot[m]);
                 }
             } else {
-                red[sl * (8 * nb) + rb0 + lane] = tot;  // ks * 8 * nb <= 64
+#pragma unroll
+                for (int m = 0; m < MT; ++m) red[(sl * (8 * nb) + rr) * MT + m] = tot[m];  // ks * 8 * nb <= 64
             }
         }
     }
@@ -296,21 +319,27 @@ __global__ void __launch_bounds__(kPdThreads, 3) gemv_predecode_kernel(
         __syncthreads();
         const int rr = threadIdx.x;
         if (rr < nrows) {
-            float tot = 0.f;
-            for (int sl = 0; sl < ks; ++sl) tot += red[sl * (8 * nb) + rr];
-            if (tot != tot)
+            float tot[MT];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) tot[m] = 0.f;
+            for (int sl = 0; sl < ks; ++sl)
+#pragma unroll
+                for (int m = 0; m < MT; ++m) tot[m] += red[(sl * (8 * nb) + rr) * MT + m];
+            if (tot[0] != tot[0])
                 err_acc |= scan_row_errors(codes + (row0 + rr) * ng * B, scales + (row0 + rr) * ng, ng, G, B);
-            store_y(Y, y_bf16, row0 + rr, tot);
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                if (m < M) store_y(Y, y_bf16, (int64_t)m * N + row0 + rr, tot[m]);
         }
     }
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
-template <int G>
-static cudaError_t launch_pd(const uint16_t* X, const uint8_t* codes, const uint16_t* scales, int64_t N, int K,
-                             int R, int grid, size_t smem, void* Y, int y_bf16, uint32_t* d_err,
+template <int G, int MT>
+static cudaError_t launch_pd(const uint16_t* X, int M, const uint8_t* codes, const uint16_t* scales, int64_t N,
+                             int K, int R, int grid, size_t smem, void* Y, int y_bf16, uint32_t* d_err,
                              cudaStream_t stream) {
-    auto kern = gemv_predecode_kernel<G>;
+    auto kern = gemv_predecode_kernel<G, MT>;
     static std::atomic<int> smem_set{0};
     if ((int)smem > smem_set.load()) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -327,30 +356,44 @@ static cudaError_t launch_pd(const uint16_t* X, const uint8_t* codes, const uint
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, X, codes, scales, N, K, R, Y, y_bf16, d_err);
+    return cudaLaunchKernelEx(&cfg, kern, X, M, codes, scales, N, K, R, Y, y_bf16, d_err);
+}
+
+template <int MT>
+static cudaError_t launch_pd_g(int G, const uint16_t* X, int M, const uint8_t* codes, const uint16_t* scales,
+                               int64_t N, int K, int R, int grid, size_t smem, void* Y, int y_bf16, uint32_t* d_err,
+                               cudaStream_t stream) {
+    switch (G) {
+        case 8: return launch_pd<8, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+        case 16: return launch_pd<16, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+        case 32: return launch_pd<32, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+        case 64: return launch_pd<64, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+        case 128: return launch_pd<128, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+        default: return launch_pd<256, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+    }
 }
 
 // Returns cudaErrorNotSupported when the shape is not covered.
 cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                   int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                                   cudaStream_t stream, int sm_count) {
-    if (M != 1 || K % 512 != 0 || N < 1 || K > 65536) return cudaErrorNotSupported;
+    if (M < 1 || M > 4 || K % 512 != 0 || N < 1 || K > 65536) return cudaErrorNotSupported;
     if (G != 8 && G != 16 && G != 32 && G != 64 && G != 128 && G != 256) return cudaErrorNotSupported;
-    const int64_t R = (N + sm_count - 1) / sm_count;
-    if (R * K * 2 > (int64_t)kPdMaxSmem) return cudaErrorNotSupported;
+    const int MT = M == 1 ? 1 : (M == 2 ? 2 : 4);
     const int64_t ng = K / G, B = bytes_per_group(G);
-    const size_t smem = (size_t)pd_head_bytes((int)K) + (size_t)(R * K * 2) +
-                        (size_t)pd_codes_area((int)(R * ng * B)) + (size_t)pd_codes_area((int)(R * ng * 2));
-    if (smem > kPdMaxSmem) return cudaErrorNotSupported;
-    const int grid = (int)((N + R - 1) / R);
-    switch (G) {
-        case 8: return launch_pd<8>(X, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
-        case 16: return launch_pd<16>(X, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
-        case 32: return launch_pd<32>(X, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
-        case 64: return launch_pd<64>(X, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
-        case 128: return launch_pd<128>(X, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
-        default: return launch_pd<256>(X, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
+    // one CTA per SM if it fits (later launches then decode beside it), else two
+    for (int per_sm = 1; per_sm <= 2; ++per_sm) {
+        const int64_t R = (N + (int64_t)sm_count * per_sm - 1) / ((int64_t)sm_count * per_sm);
+        if (R * K * 2 > (int64_t)kPdMaxSmem) continue;
+        const size_t smem = (size_t)pd_head_bytes((int)K, MT) + (size_t)(R * K * 2) +
+                            (size_t)pd_codes_area((int)(R * ng * B)) + (size_t)pd_codes_area((int)(R * ng * 2));
+        if (smem > kPdMaxSmem) continue;
+        const int grid = (int)((N + R - 1) / R);
+        if (MT == 1) return launch_pd_g<1>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
+        if (MT == 2) return launch_pd_g<2>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
+        return launch_pd_g<4>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
     }
+    return cudaErrorNotSupported;
 }
 
 }  // namespace tq

@@ -66,6 +66,10 @@ def test_rejected_groups_give_nan_rows():
     X = synthetic.activations(130, K)
     ref = check(X, W, G, codes=codes, scales=scales)
     assert np.all(np.isnan(ref[:, [3, 7, 11, 13]])) and np.all(np.isfinite(ref[:, 17]))
+    _, e_ref = oracle.unpack_bf16(codes, scales, N, K, G)
+    for M in (130, 16):  # prefill kernel; small-M kernel
+        _, e = run(X[:M], codes, scales, N, K, G, torch.float32)
+        assert e == e_ref
 
 
 def test_unsupported_group_size():

@@ -113,12 +113,13 @@ def test_row_counts(N):
 
 @pytest.mark.parametrize("N,K,G", [(9477, 512, 64), (2000, 512, 32), (150, 4096, 256), (1500, 3072, 8),
                                    (700, 2048, 128), (300, 1024, 16)])
-def test_predecode_row_batches(N, K, G):
-    """One token over matrices whose per-CTA rows fit in shared memory: more
-    than eight 8-row batches per CTA, chunks split over two to eight warps,
-    ragged last CTA."""
+@pytest.mark.parametrize("M", [1, 4])
+def test_predecode_row_batches(N, K, G, M):
+    """One to four tokens over matrices whose per-CTA rows fit in shared
+    memory: more than eight 8-row batches per CTA, chunks split over two to
+    eight warps, ragged last CTA, one or two CTAs per SM."""
     W = synthetic.weights(N, K, index=N + K)
-    X = synthetic.activations(1, K)
+    X = synthetic.activations(M, K)
     check(X, W, G)
 
 
