@@ -65,6 +65,7 @@ struct Params {
     int K, G, B, ng;
     int tiles;
     int y_bf16;
+    uint32_t pad_base, pad_span;  // canonical range of a group's last code byte
 };
 
 __device__ __forceinline__ void cp_async16(uint8_t* dst, const uint8_t* src) {
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     constexpr uint32_t kCols = 2 * NT < 32 ? 32 : 2 * NT;
     volatile int* abort_flag = &sm.abort_flag;
 
-    init_selector_lut(sm.lut, threadIdx.x, kThreads);
+    fill_digit_selector_lut(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(&sm.full_x[st], 1);
@@ -193,28 +194,40 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     } else if (warp >= kDecWarp0 && warp < kEpiWarp0) {
         const int grp = (warp - kDecWarp0) >> 2;              // stages grp, grp + 2, ...
         const int t = ((warp - kDecWarp0) & 3) * 32 + lane;  // W row of the tile
-        const int real = p.G - 5 * (p.B - 1);
-        const uint32_t pm = padding_mask(real), po = padding_ones(real);
-        // geometry of own stage s: row n, group g, first column c0 in the group, first byte q_lo
-        auto geom = [&](int s, int64_t& n, int& g, int& c0, int& q_lo, int& kb) {
-            const int i = grp + 2 * s;
-            const int j = i / nk;
-            kb = i - j * nk;
-            n = ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * WM + t;
-            if (n >= p.N) n = p.N - 1;  // rows past the end decode a real row; never stored
-            const int k0 = kb * BK;
-            g = k0 / p.G;
-            c0 = k0 - g * p.G;
-            q_lo = c0 / 5;
+        const int SPG = p.G / BK;                             // stages per group
+        // stage position (tile iteration j, group g, part sub of the group),
+        // advanced by two stages at a time without divisions
+        struct Pos {
+            int j, g, sub;
         };
+        auto advance = [&](Pos& q) {
+            q.sub += 2;
+            while (q.sub >= SPG) {
+                q.sub -= SPG;
+                if (++q.g == p.ng) {
+                    q.g = 0;
+                    ++q.j;
+                }
+            }
+        };
+        auto row_of = [&](const Pos& q) {
+            const int64_t n = ((int64_t)blockIdx.x + (int64_t)q.j * gridDim.x) * WM + t;
+            return n < p.N ? n : p.N - 1;  // rows past the end decode a real row; never stored
+        };
+        Pos pd{0, 0, 0}, pi{0, 0, 0};  // decode position, prefetch position
+        if (grp) {                      // group 1 starts at stage 1
+            pd.sub = pi.sub = -1;
+            advance(pd);
+            pi = pd;
+        }
         auto issue = [&](int s) {
             if (grp + 2 * s < total) {
-                int64_t n;
-                int g, c0, q_lo, kb;
-                geom(s, n, g, c0, q_lo, kb);
+                const int64_t n = row_of(pi);
+                const int q_lo = (BK * pi.sub) / 5;
                 uint8_t* slot = sm.win[grp][s % CR] + t * WIN;
-                fetch_window(slot, p.codes + n * p.row_bytes + (int64_t)g * p.B + q_lo, p.codes, p.codes_end);
-                fetch_scale(slot + 32, p.scales + n * p.ng + g, p.scales, p.scales_end);
+                fetch_window(slot, p.codes + n * p.row_bytes + (int64_t)pi.g * p.B + q_lo, p.codes, p.codes_end);
+                fetch_scale(slot + 32, p.scales + n * p.ng + pi.g, p.scales, p.scales_end);
+                advance(pi);
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
         };
@@ -225,19 +238,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
             asm volatile("cp.async.wait_group %0;" ::"n"(CR - 1) : "memory");
             const int i = grp + 2 * s, st = i % STAGES, use = i / STAGES;
             if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
-            int64_t n;
-            int g, c0, q_lo, kb;
-            geom(s, n, g, c0, q_lo, kb);
+            const int64_t n = row_of(pd);
+            const int c0 = BK * pd.sub, q_lo = c0 / 5;
+            const uintptr_t A = reinterpret_cast<uintptr_t>(p.codes + n * p.row_bytes + (int64_t)pd.g * p.B + q_lo);
+            const uintptr_t S = reinterpret_cast<uintptr_t>(p.scales + n * p.ng + pd.g);
             const uint8_t* slot = sm.win[grp][s % CR] + t * WIN;
-            const uintptr_t A = reinterpret_cast<uintptr_t>(p.codes + n * p.row_bytes + (int64_t)g * p.B + q_lo);
-            const uintptr_t S = reinterpret_cast<uintptr_t>(p.scales + n * p.ng + g);
-            uint32_t bytes[14];
-            window_bytes(slot, (int)(A & 15), bytes);
             const uint32_t sc = *reinterpret_cast<const uint16_t*>(slot + 32 + (S & 2));
-            decode_stage_row(sm.lut, bytes, c0, q_lo, p.B, pm, po, sc, sm.w[st] + t * 128, t & 7);
+            decode_stage64(sm.lut, slot + (A & 15), c0 - 5 * q_lo, p.B - 1 - q_lo, p.pad_base, p.pad_span, sc,
+                           sm.w[st] + t * 128, t & 7);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_w[st]);
+            advance(pd);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp >= kEpiWarp0) {
@@ -338,6 +350,7 @@ cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* code
     p.ng = (int)(K / G);
     p.tiles = (int)tiles;
     p.y_bf16 = y_bf16;
+    padding_range(G, p.pad_base, p.pad_span);
     const int grid = (int)(tiles < sm_count ? tiles : sm_count);
     cudaError_t e;
     if (NT == 16) e = launch_nt<16>(tx, p, grid, stream);

@@ -243,6 +243,73 @@ __device__ __forceinline__ void decode_stage_row(const uint2* lut, uint32_t (&by
     }
 }
 
+// Single-path decoder of one row's 64 weights for a stage: columns c0 ..
+// c0+63 of one group, c0 a multiple of 64, r0 = c0 % 5.  `cb` points at code
+// byte q_lo = c0 / 5 of the group in shared memory, and the 14 bytes from
+// there are readable (the ones past the group only feed digits past the
+// stage).  `last` is the group's last byte relative to cb (>= 14 when the
+// stage does not hold it); a canonical last byte lies in [pad_base,
+// pad_base + pad_span).  `lut` maps a byte to its five PRMT selectors with
+// digit d -> 0x10 + 0x22 d over V = {-s, 0}, Z = {+s, NaN} (bytes >= 243
+// select NaN).  The selector stream of the 14 bytes is packed into words by
+// PRMT and funnel-shifted by r0 bytes, so every stage takes the same code.
+// A rejected scale or padding digit makes the row's stage NaN.  Writes the
+// 128-byte swizzled K-major tile row.
+__device__ __forceinline__ void decode_stage64(const uint2* lut, const uint8_t* cb, int r0, int last,
+                                               uint32_t pad_base, uint32_t pad_span, uint32_t scale_bits,
+                                               uint8_t* tile_row, int row_in_atom) {
+    uint2 e[14];
+#pragma unroll
+    for (int i = 0; i < 14; ++i) e[i] = lut[cb[i]];
+    uint32_t W[17];
+#pragma unroll
+    for (int h = 0; h < 3; ++h) {
+        const uint2 a = e[4 * h], b = e[4 * h + 1], c = e[4 * h + 2], d = e[4 * h + 3];
+        W[5 * h + 0] = a.x;
+        W[5 * h + 1] = prmt(a.y, b.x, 0x6540u);
+        W[5 * h + 2] = prmt(prmt(b.x, b.y, 0x0043u), c.x, 0x5410u);
+        W[5 * h + 3] = prmt(prmt(c.x, c.y, 0x0432u), d.x, 0x4210u);
+        W[5 * h + 4] = prmt(d.x, d.y, 0x4321u);
+    }
+    W[15] = e[12].x;
+    W[16] = prmt(e[12].y, e[13].x, 0x6540u);
+    bool bad = scale_is_bad(scale_bits);
+    if (last < 14) bad |= (uint32_t)cb[last] - pad_base >= pad_span;
+    uint32_t V, Z;
+    if (bad) {
+        V = Z = 0x7FC07FC0u;
+    } else {
+        const uint32_t mag = scale_bits == 0 ? 0u : scale_to_bf16_bits((uint16_t)scale_bits);
+        V = mag ? (mag | 0x8000u) : 0u;  // {-s, 0}
+        Z = mag | 0x7FC00000u;           // {+s, NaN}
+    }
+    const uint32_t sh = 8u * (uint32_t)r0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t o0 = __funnelshift_rc(W[2 * k], W[2 * k + 1], sh);
+        const uint32_t o1 = __funnelshift_rc(W[2 * k + 1], W[2 * k + 2], sh);
+        *reinterpret_cast<uint4*>(tile_row + ((k ^ row_in_atom) << 4)) =
+            make_uint4(prmt(V, Z, o0), prmt(V, Z, o0 >> 16), prmt(V, Z, o1), prmt(V, Z, o1 >> 16));
+    }
+}
+
+// Canonical range of a group's last code byte: digits REAL..4 equal to 1,
+// i.e. [base, base + 3^REAL) with base = sum_{i=REAL}^{4} 3^i (REAL < 5);
+// every byte below 243 when REAL == 5.
+__host__ __device__ inline void padding_range(int G, uint32_t& base, uint32_t& span) {
+    const int B = bytes_per_group(G);
+    const int real = G - 5 * (B - 1);
+    uint32_t b = 0, p = 1;
+    for (int i = 0; i < 5; ++i) {
+        if (i >= real) b += p;
+        p *= 3;
+    }
+    uint32_t sp = 1;
+    for (int i = 0; i < real; ++i) sp *= 3;
+    base = b;
+    span = sp;
+}
+
 // Encoder of 2-D TMA descriptors (driver entry point, no libcuda link).
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, void* base, uint64_t dim0, uint64_t dim1,
                     uint64_t stride1_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle swizzle);
