@@ -63,6 +63,7 @@ struct Params {
     int K, G, B, ng;
     int CS;  // cluster size = split of K
     int y_bf16;
+    uint32_t pad_base, pad_span;  // canonical range of a group's last code byte
 };
 
 template <int NT, bool CODES_TMA>
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_small_kernel(const __grid_co
     constexpr uint32_t kCols = NT < 32 ? 32 : NT;
     volatile int* abort_flag = &sm.abort_flag;
 
-    init_selector_lut(sm.lut, threadIdx.x, kThreads);
+    fill_digit_selector_lut(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(&sm.full_x[st], 1);
@@ -159,8 +160,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_small_kernel(const __grid_co
         const int t = threadIdx.x - kDecodeWarp0 * 32;  // W row of the tile
         const int64_t n = n0 + t;
         const uint16_t* srow = p.scales + (n < p.N ? n : 0) * p.ng;
-        const int real = p.G - 5 * (p.B - 1);
-        const uint32_t pm = padding_mask(real), po = padding_ones(real);
         const uint8_t* crow = p.codes + (n < p.N ? n : 0) * p.row_bytes;
         auto load_global = [&](int kb, uint32_t (&bytes)[14]) {
             int g, c0, q_lo;
@@ -171,21 +170,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_small_kernel(const __grid_co
         };
         uint32_t cur[14], nxt[14];
         if (!CODES_TMA && nkl > 0) load_global(kb_lo, cur);
+        uint32_t sc_nxt = nkl > 0 ? __ldg(srow + (kb_lo * BK) / p.G) : 0u;
         for (int i = 0; i < nkl; ++i) {
             const int kb = kb_lo + i, st = i % STAGES, use = i / STAGES;
             int g, c0, q_lo;
             stage_geom(kb, g, c0, q_lo);
-            uint32_t bytes[14];
+            const uint32_t sc = sc_nxt;
+            if (i + 1 < nkl) sc_nxt = __ldg(srow + ((kb + 1) * BK) / p.G);  // next stage's scale in flight
+            const int ql = p.B - 1 - q_lo;  // the group's last byte relative to q_lo
+            uint32_t bytes[14], lastb = 0;
             if (CODES_TMA) {
                 if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag)) break;
-                window_bytes(sm.c[st] + t * C_ROW, (g * p.B + q_lo) & 15, bytes);
+                const int off = (g * p.B + q_lo) & 15;
+                const uint8_t* win = sm.c[st] + t * C_ROW;
+                window_bytes(win, off, bytes);
+                if (ql < 14) lastb = win[off + ql];
             } else {
                 if (i + 1 < nkl) load_global(kb + 1, nxt);  // next stage's bytes in flight
                 if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
 #pragma unroll
                 for (int j = 0; j < 14; ++j) bytes[j] = cur[j];
+                if (ql < 14) lastb = __ldg(crow + (int64_t)g * p.B + p.B - 1);
             }
-            decode_stage_row(sm.lut, bytes, c0, q_lo, p.B, pm, po, __ldg(srow + g), sm.w[st] + t * 128, t & 7);
+            decode_stage64(sm.lut, bytes, c0 - 5 * q_lo, ql < 14, lastb, p.pad_base, p.pad_span, sc,
+                           sm.w[st] + t * 128, t & 7);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_w[st]);
@@ -339,6 +347,7 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     p.ng = (int)(K / G);
     p.CS = CS;
     p.y_bf16 = y_bf16;
+    padding_range(G, p.pad_base, p.pad_span);
     cudaError_t e;
     if (codes_tma) {
         if (NT == 16) e = launch_nt<16, true>(tx, tcm, p, (int)tiles, stream);

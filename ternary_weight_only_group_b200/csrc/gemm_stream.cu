@@ -243,9 +243,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
             const uintptr_t A = reinterpret_cast<uintptr_t>(p.codes + n * p.row_bytes + (int64_t)pd.g * p.B + q_lo);
             const uintptr_t S = reinterpret_cast<uintptr_t>(p.scales + n * p.ng + pd.g);
             const uint8_t* slot = sm.win[grp][s % CR] + t * WIN;
+            const uint8_t* cb = slot + (A & 15);
             const uint32_t sc = *reinterpret_cast<const uint16_t*>(slot + 32 + (S & 2));
-            decode_stage64(sm.lut, slot + (A & 15), c0 - 5 * q_lo, p.B - 1 - q_lo, p.pad_base, p.pad_span, sc,
-                           sm.w[st] + t * 128, t & 7);
+            uint32_t bytes[14];
+#pragma unroll
+            for (int b = 0; b < 14; ++b) bytes[b] = cb[b];
+            const int ql = p.B - 1 - q_lo;  // the group's last byte, relative to cb
+            decode_stage64(sm.lut, bytes, c0 - 5 * q_lo, ql < 14, ql < 14 ? cb[ql] : 0u, p.pad_base, p.pad_span,
+                           sc, sm.w[st] + t * 128, t & 7);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_w[st]);

@@ -18,8 +18,10 @@
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator quadrant, bf16 or
 //               fp32 stores.
 // Decoding: a per-CTA table maps each code byte to the PRMT byte selectors of
-// its five weights; one PRMT gathers the selectors of a weight pair, a second
-// PRMT picks the pair's bf16 values among {+s, -s, 0, NaN}.  Invalid bytes,
+// its five weights; the selectors of a stage's 14 bytes are packed into a
+// stream, shifted to the stage's first column, and one PRMT per weight pair
+// picks the bf16 values among {-s, 0, +s, NaN}.  Each decoder prefetches the
+// next stage's scale (and, without TMA, its code bytes).  Invalid bytes,
 // non-canonical padding and bad scales decode to NaN (the row's outputs are
 // then NaN, as the decoder defines); the W rows behind NaN outputs of the
 // first X row are rescanned for the error bits.
@@ -71,6 +73,7 @@ struct Params {
     int64_t row_bytes;
     int n_tiles;
     int y_bf16;
+    uint32_t pad_base, pad_span;  // canonical range of a group's last code byte
     int y_vec;  // Y rows allow 16-byte vector stores (base aligned, N a multiple of 16 bytes)
 };
 
@@ -86,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int nk = p.K / BK;
     volatile int* abort_flag = &sm.abort_flag;
 
-    init_selector_lut(sm.lut, threadIdx.x, kThreads);
+    fill_digit_selector_lut(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(&sm.full_a[st], 1);
@@ -177,25 +180,39 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         const bool row_ok = n < p.N;
         const uint8_t* crow = p.codes + (row_ok ? n : 0) * p.row_bytes;
         const uint16_t* srow = p.scales + (row_ok ? n : 0) * p.ng;
-        const int real = p.G - 5 * (p.B - 1);
-        const uint32_t pm = padding_mask(real), po = padding_ones(real);
+        auto load_global = [&](int kb, uint32_t (&bytes)[14]) {  // code bytes of a stage, by loads
+            int g, c0, q_lo;
+            stage_geom(kb, g, c0, q_lo);
+            const uint8_t* cb = crow + (int64_t)g * p.B;
+#pragma unroll
+            for (int i = 0; i < 14; ++i) bytes[i] = (q_lo + i < p.B) ? (uint32_t)__ldg(cb + q_lo + i) : kZeroByte;
+        };
+        uint32_t nxt[14];
+        if (!CODES_TMA) load_global(0, nxt);
+        uint32_t sc_nxt = __ldg(srow);  // scale of stage 0 (group 0)
         for (int kb = 0; kb < nk; ++kb) {
             const int st = kb % STAGES, use = kb / STAGES;
             int g, c0, q_lo;
             stage_geom(kb, g, c0, q_lo);
-            uint32_t bytes[14];
+            const uint32_t sc = sc_nxt;
+            if (kb + 1 < nk) sc_nxt = __ldg(srow + ((kb + 1) * BK) / p.G);  // next stage's scale in flight
+            const int ql = p.B - 1 - q_lo;  // the group's last byte relative to q_lo
+            uint32_t bytes[14], lastb = 0;
             if (CODES_TMA) {
                 if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag)) break;
                 const int gb = g * p.B + q_lo;
-                window_bytes(sm.c[st] + t * C_ROW, gb & 15, bytes);
+                const uint8_t* win = sm.c[st] + t * C_ROW;
+                window_bytes(win, gb & 15, bytes);
+                if (ql < 14) lastb = win[(gb & 15) + ql];
             } else {
-                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
-                const uint8_t* cb = crow + (int64_t)g * p.B;
 #pragma unroll
-                for (int i = 0; i < 14; ++i)
-                    bytes[i] = (q_lo + i < p.B) ? (uint32_t)__ldg(cb + q_lo + i) : kZeroByte;
+                for (int i = 0; i < 14; ++i) bytes[i] = nxt[i];
+                if (kb + 1 < nk) load_global(kb + 1, nxt);  // next stage's bytes in flight
+                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
+                if (ql < 14) lastb = __ldg(crow + (int64_t)g * p.B + p.B - 1);
             }
-            decode_stage_row(sm.lut, bytes, c0, q_lo, p.B, pm, po, __ldg(srow + g), sm.b[st] + t * 128, t & 7);
+            decode_stage64(sm.lut, bytes, c0 - 5 * q_lo, ql < 14, lastb, p.pad_base, p.pad_span, sc,
+                           sm.b[st] + t * 128, t & 7);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_b[st]);
@@ -354,6 +371,7 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
     p.ng = (int)(K / G);
     p.row_bytes = row_bytes;
     p.n_tiles = (int)((N + BN - 1) / BN);
+    padding_range(G, p.pad_base, p.pad_span);
     p.y_bf16 = y_bf16;
     p.y_vec = ((reinterpret_cast<uintptr_t>(Y) & 15) == 0) && ((N * (y_bf16 ? 2 : 4)) % 16 == 0);
     const int64_t m_tiles = (M + BM - 1) / BM;

@@ -121,43 +121,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return r;
 }
 
-// PRMT selector byte of one weight: two nibbles naming the bytes of its bf16
-// value inside the 8-byte pair (V = {+s, -s}, Z = {0, NaN}).
-constexpr uint32_t kSelPos = 0x10, kSelNeg = 0x32, kSelZero = 0x54, kSelNaN = 0x76;
-
-// Decode one row's 64 weights of a stage (columns c0..c0+63 of group g, c0 % 5 == R0)
-// into the swizzled tile row.  bytes[] holds code bytes q_lo .. q_lo+13.
-template <int R0>
-__device__ __forceinline__ void decode_row(const uint2* lut, const uint32_t (&bytes)[14], uint32_t V, uint32_t Z,
-                                           uint8_t* tile_row, int row_in_atom) {
-    // selector bytes of the 64 columns: column j uses digit (R0 + j) % 5 of byte (R0 + j) / 5
-    uint2 e[14];
-#pragma unroll
-    for (int t = 0; t < 14; ++t) e[t] = lut[bytes[t]];
-#pragma unroll
-    for (int chunk = 0; chunk < 8; ++chunk) {
-        uint32_t w[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const int j0 = chunk * 8 + 2 * h, j1 = j0 + 1;
-            const int q0 = (R0 + j0) / 5, i0 = (R0 + j0) % 5;
-            const int q1 = (R0 + j1) / 5, i1 = (R0 + j1) % 5;
-            // selector bytes live in byte i of the 8-byte entry {lo, hi}
-            uint32_t sel;
-            if (q0 == q1) {
-                const uint32_t lo = e[q0].x, hi = e[q0].y;
-                sel = prmt(lo, hi, (uint32_t)i0 | ((uint32_t)i1 << 4));
-            } else {  // pair straddles two bytes: digit 4 of one, digit 0 of the next
-                sel = prmt(e[q0].y, e[q1].x, 0u | (4u << 4));
-            }
-            // sel bytes: [s0, s1, ...]; value selector = s0 | s1 << 8 (PRMT uses the low 16 bits)
-            w[h] = prmt(V, Z, sel);
-        }
-        const int phys = chunk ^ row_in_atom;  // 128-byte swizzle: 16-byte chunk index XOR (row % 8)
-        *reinterpret_cast<uint4*>(tile_row + phys * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
 // Code bytes q_lo .. q_lo+13 of one row for a stage, read from the staged
 // 32-byte window (TMA mode): the window starts at the 16-byte-aligned byte at
 // or below the first needed one, `off` bytes earlier.
@@ -190,77 +153,24 @@ __device__ __forceinline__ void window_bytes(const uint8_t* row32, int off, uint
 }
 
 
-// Selector table: byte -> PRMT selector bytes of its five weights (digits
-// 0..4 in bytes 0..4 of the 8-byte entry); bytes >= 243 select NaN.
-__device__ __forceinline__ void init_selector_lut(uint2* lut, int tid, int nthreads) {
-    for (int b = tid; b < 256; b += nthreads) {
-        uint32_t sv[5];
-        if (b >= 243) {
-            for (int i = 0; i < 5; ++i) sv[i] = kSelNaN;
-        } else {
-            uint32_t v = b;
-            for (int i = 0; i < 5; ++i) {
-                const uint32_t d = v % 3;
-                v /= 3;
-                sv[i] = d == 0 ? kSelNeg : (d == 1 ? kSelZero : kSelPos);
-            }
-        }
-        lut[b] = make_uint2(sv[0] | (sv[1] << 8) | (sv[2] << 16) | (sv[3] << 24), sv[4]);
-    }
-}
-
-// Decodes the 64 weights of one W row for a stage (columns c0 .. c0+63 of
-// group g, code bytes q_lo .. q_lo+13 in bytes[]) into a 128-byte swizzled
-// tile row.  A group's last byte with a padding digit other than 1, and a
-// scale that is NaN, Inf or negative, decode to NaN.
-__device__ __forceinline__ void decode_stage_row(const uint2* lut, uint32_t (&bytes)[14], int c0, int q_lo, int B,
-                                                 uint32_t pm, uint32_t po, uint32_t scale_bits, uint8_t* tile_row,
-                                                 int row_in_atom) {
-    const int ql = B - 1 - q_lo;
-#pragma unroll
-    for (int i = 0; i < 14; ++i) {
-        if (q_lo + i >= B) bytes[i] = kZeroByte;
-        if (i == ql) {
-            const uint32_t dp = byte_digit_pattern(bytes[i]);
-            if ((dp & 0x8000u) == 0 && (dp & pm) != po) bytes[i] = 255;
-        }
-    }
-    uint32_t V, Z;
-    if (scale_is_bad(scale_bits)) {
-        V = 0x7FC07FC0u;
-        Z = 0x7FC07FC0u;
-    } else {
-        const uint32_t mag = scale_bits == 0 ? 0u : scale_to_bf16_bits((uint16_t)scale_bits);
-        V = mag | ((mag ? (mag | 0x8000u) : 0u) << 16);  // {+s, -s}
-        Z = 0x7FC00000u;                                // {0, NaN}
-    }
-    switch (c0 % 5) {
-        case 0: decode_row<0>(lut, bytes, V, Z, tile_row, row_in_atom); break;
-        case 1: decode_row<1>(lut, bytes, V, Z, tile_row, row_in_atom); break;
-        case 2: decode_row<2>(lut, bytes, V, Z, tile_row, row_in_atom); break;
-        case 3: decode_row<3>(lut, bytes, V, Z, tile_row, row_in_atom); break;
-        default: decode_row<4>(lut, bytes, V, Z, tile_row, row_in_atom); break;
-    }
-}
-
 // Single-path decoder of one row's 64 weights for a stage: columns c0 ..
-// c0+63 of one group, c0 a multiple of 64, r0 = c0 % 5.  `cb` points at code
-// byte q_lo = c0 / 5 of the group in shared memory, and the 14 bytes from
-// there are readable (the ones past the group only feed digits past the
-// stage).  `last` is the group's last byte relative to cb (>= 14 when the
-// stage does not hold it); a canonical last byte lies in [pad_base,
-// pad_base + pad_span).  `lut` maps a byte to its five PRMT selectors with
-// digit d -> 0x10 + 0x22 d over V = {-s, 0}, Z = {+s, NaN} (bytes >= 243
-// select NaN).  The selector stream of the 14 bytes is packed into words by
-// PRMT and funnel-shifted by r0 bytes, so every stage takes the same code.
-// A rejected scale or padding digit makes the row's stage NaN.  Writes the
-// 128-byte swizzled K-major tile row.
-__device__ __forceinline__ void decode_stage64(const uint2* lut, const uint8_t* cb, int r0, int last,
-                                               uint32_t pad_base, uint32_t pad_span, uint32_t scale_bits,
-                                               uint8_t* tile_row, int row_in_atom) {
+// c0+63 of one group, c0 a multiple of 64, r0 = c0 % 5.  bytes[] holds code
+// bytes q_lo = c0 / 5 .. q_lo + 13 of the group (those past the group only
+// feed digits past the stage, so their values do not matter).  When the
+// stage holds the group's last byte (check_pad), `lastb` is that byte, and a
+// canonical one lies in [pad_base, pad_base + pad_span).  `lut` maps a byte
+// to its five PRMT selectors with digit d -> 0x10 + 0x22 d over V = {-s, 0},
+// Z = {+s, NaN} (bytes >= 243 select NaN).  The selector stream of the 14
+// bytes is packed into words by PRMT and funnel-shifted by r0 bytes, so every
+// stage takes the same code.  A rejected scale or padding digit makes the
+// row's stage NaN.  Writes the 128-byte swizzled K-major tile row.
+__device__ __forceinline__ void decode_stage64(const uint2* lut, const uint32_t (&bytes)[14], int r0,
+                                               bool check_pad, uint32_t lastb, uint32_t pad_base,
+                                               uint32_t pad_span, uint32_t scale_bits, uint8_t* tile_row,
+                                               int row_in_atom) {
     uint2 e[14];
 #pragma unroll
-    for (int i = 0; i < 14; ++i) e[i] = lut[cb[i]];
+    for (int i = 0; i < 14; ++i) e[i] = lut[bytes[i] & 0xFFu];
     uint32_t W[17];
 #pragma unroll
     for (int h = 0; h < 3; ++h) {
@@ -274,7 +184,7 @@ __device__ __forceinline__ void decode_stage64(const uint2* lut, const uint8_t* 
     W[15] = e[12].x;
     W[16] = prmt(e[12].y, e[13].x, 0x6540u);
     bool bad = scale_is_bad(scale_bits);
-    if (last < 14) bad |= (uint32_t)cb[last] - pad_base >= pad_span;
+    if (check_pad) bad |= lastb - pad_base >= pad_span;
     uint32_t V, Z;
     if (bad) {
         V = Z = 0x7FC07FC0u;
