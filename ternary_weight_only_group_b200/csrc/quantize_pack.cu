@@ -13,7 +13,9 @@
 // so the shuffle order cannot change it; dividing by G (a power of two) is
 // exact and cvt.rn.f16.f64 rounds once, ties to even.  A group holding a
 // nonzero |w| more than 2^37 below its maximum takes the multi-word exact
-// path instead.  Other G use one thread per group with the multi-word path.
+// path instead.  Each lane loads the next pass's weights before it computes
+// the current pass.  Other G use one thread per group with the multi-word
+// path.
 #include "tq_internal.cuh"
 
 namespace tq {
@@ -32,11 +34,21 @@ __global__ void __launch_bounds__(256) quantize_pack_pow2_kernel(
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     uint32_t err_acc = 0;
 
-    for (int64_t base = warp * GPW; base < num_groups; base += nwarps * GPW) {
+    // The next pass's 16-byte load is issued before this pass is computed
+    // (two loads in flight per lane).
+    const int64_t stride = nwarps * GPW;
+    auto load = [&](int64_t base) {
+        const int64_t gi = base + lane / LPG;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (gi < num_groups) v = __ldcs(reinterpret_cast<const uint4*>(W + gi * G + p0));
+        return v;
+    };
+    uint4 v_next = load(warp * GPW);
+    for (int64_t base = warp * GPW; base < num_groups; base += stride) {
         const int64_t gi = base + lane / LPG;
         const bool active = gi < num_groups;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (active) v = __ldcs(reinterpret_cast<const uint4*>(W + gi * G + p0));
+        const uint4 v = v_next;
+        v_next = load(base + stride);
         const uint32_t h[4] = {v.x, v.y, v.z, v.w};
         uint32_t a[8];
 #pragma unroll
@@ -117,6 +129,108 @@ __global__ void __launch_bounds__(256) quantize_pack_pow2_kernel(
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
+// One lane per group (G = 8, 16, 32, 64, 128): the group's G weights sit in
+// the lane's registers, so max and sum need no shuffles; every weight's byte
+// and power of three are compile-time constants, so encoding is one
+// multiply-add per weight into packed code words; each warp's 32 groups of
+// code bytes are assembled in shared memory and written with 16-byte stores
+// when the destination allows it.  The scale arithmetic is the one above.
+template <int G>
+__global__ void __launch_bounds__(256, G <= 32 ? 3 : (G == 64 ? 2 : 1)) quantize_pack_group_kernel(
+    const uint16_t* __restrict__ W, int64_t num_groups, uint8_t* __restrict__ codes,
+    uint16_t* __restrict__ scales, uint32_t* __restrict__ d_err) {
+    constexpr int NWD = G / 2;                 // 32-bit words of a group
+    constexpr int B = bytes_per_group(G);
+    constexpr int NCW = (B + 3) / 4;           // packed code words
+    __shared__ __align__(16) uint8_t stage[256 / 32][32 * B];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const bool vec_out = (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
+    uint32_t err_acc = 0;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); g0 < num_groups; g0 += stride) {
+        const int64_t gi = g0 + lane;  // the warp's groups g0 .. g0+31
+        const bool active = gi < num_groups;
+        uint32_t h[NWD];
+        {
+            const uint4* src = reinterpret_cast<const uint4*>(W + (active ? gi : 0) * G);
+#pragma unroll
+            for (int k = 0; k < G / 8; ++k) {
+                const uint4 v = __ldg(src + k);
+                h[4 * k] = v.x;
+                h[4 * k + 1] = v.y;
+                h[4 * k + 2] = v.z;
+                h[4 * k + 3] = v.w;
+            }
+        }
+        uint32_t amax = 0;
+#pragma unroll
+        for (int j = 0; j < G; ++j) amax = max(amax, (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu);
+        const uint32_t emax = amax >> 7;
+        const uint32_t thr = emax > 37 ? (emax - 37) << 7 : 0;  // smallest pattern in the exact window
+        double sum = 0.0;
+        uint32_t outside = 0;
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            const uint32_t a = (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
+            if (a >= thr) sum += bf16_normal_mag_to_f64(a);
+            else outside |= a;
+        }
+        uint16_t s = 0;
+        uint32_t gerr = 0;
+        if (amax >= 0x7F80u) {
+            gerr = TQ_DERR_WEIGHT;
+        } else if (amax > kTinyMaxBits) {
+            if (outside) {
+                gerr = exact_group_scale(W + (active ? gi : 0) * G, G, &s);
+            } else {
+                const uint16_t bits = __half_as_ushort(__double2half(sum * (1.0 / G)));
+                if (bits >= 0x7C00u) gerr = TQ_DERR_OVERFLOW;
+                else s = bits;
+            }
+        }
+        if (gerr) s = 0;
+        const uint32_t th = trit_threshold(s);
+        // code words: byte q of the group in byte q % 4 of word q / 4; digit
+        // d = t + 1 of weight j adds d * 3^(j % 5) to byte j / 5; positions
+        // j >= G hold the padding digit 1
+        uint32_t cw[NCW];
+#pragma unroll
+        for (int i = 0; i < NCW; ++i) cw[i] = 0;
+#pragma unroll
+        for (int j = 0; j < 5 * B; ++j) {
+            const int q = j / 5;
+            const uint32_t pw = (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
+                                << (8 * (q % 4));
+            if (j < G) {
+                const uint32_t hw = h[j >> 1] >> (16 * (j & 1));
+                const uint32_t d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
+                cw[q / 4] += d * pw;
+            } else {
+                cw[q / 4] += pw;  // padding digit 1
+            }
+        }
+        if (active) {
+            scales[gi] = s;
+            err_acc |= gerr;
+        }
+        // the warp's 32 * B code bytes, contiguous from g0 * B
+        uint8_t* st = stage[wib] + lane * B;
+#pragma unroll
+        for (int q = 0; q < B; ++q) st[q] = (uint8_t)(cw[q / 4] >> (8 * (q % 4)));
+        __syncwarp();
+        const int64_t nvalid = (num_groups - g0 < 32 ? num_groups - g0 : 32) * B;
+        uint8_t* out = codes + g0 * B;
+        if (vec_out && nvalid == 32 * B) {  // 32 * B is a multiple of 16 for these G
+            for (int c = lane; c < 2 * B; c += 32)
+                reinterpret_cast<uint4*>(out)[c] = reinterpret_cast<const uint4*>(stage[wib])[c];
+        } else {
+            for (int c = lane; c < nvalid; c += 32) out[c] = stage[wib][c];
+        }
+        __syncwarp();
+    }
+    if (err_acc && d_err) atomicOr(d_err, err_acc);
+}
+
 // Any G: one thread per group, multi-word exact scale.
 __global__ void __launch_bounds__(128) quantize_pack_generic_kernel(
     const uint16_t* __restrict__ W, int64_t num_groups, int G, uint8_t* __restrict__ codes,
@@ -170,17 +284,25 @@ cudaError_t launch_quantize_pack(const uint16_t* W, int64_t N, int64_t K, int G,
             W, num_groups, codes, scales, d_err);                                                \
         return cudaGetLastError();                                                               \
     }
+#define TQ_QG_CASE(GG)                                                                              \
+    case GG: {                                                                                      \
+        const int64_t threads = (num_groups + 31) / 32 * 32;                                        \
+        quantize_pack_group_kernel<GG><<<grid_for(threads, block, sm_count), block, 0, stream>>>(   \
+            W, num_groups, codes, scales, d_err);                                                   \
+        return cudaGetLastError();                                                                  \
+    }
     switch (G) {
-        TQ_QP_CASE(8)
-        TQ_QP_CASE(16)
-        TQ_QP_CASE(32)
-        TQ_QP_CASE(64)
-        TQ_QP_CASE(128)
+        TQ_QG_CASE(8)
+        TQ_QG_CASE(16)
+        TQ_QG_CASE(32)
+        TQ_QG_CASE(64)
+        TQ_QG_CASE(128)
         TQ_QP_CASE(256)
         default:
             break;
     }
 #undef TQ_QP_CASE
+#undef TQ_QG_CASE
     quantize_pack_generic_kernel<<<grid_for(num_groups, 128, sm_count), 128, 0, stream>>>(
         W, num_groups, G, codes, scales, d_err);
     return cudaGetLastError();

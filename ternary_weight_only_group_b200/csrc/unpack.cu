@@ -35,19 +35,30 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     uint32_t err_acc = 0;
 
-    for (int64_t base = warp * GPW; base < num_groups; base += nwarps * GPW) {
+    // weights p0..p0+7 lie in bytes q_first .. q_first+2 (the third only for its
+    // first digits); the next pass's bytes and scale are loaded before this
+    // pass is decoded
+    const int64_t stride = nwarps * GPW;
+    auto load = [&](int64_t base, uint32_t (&bv)[3], uint32_t& s) {
         const int64_t gi = base + lane / LPG;
-        const bool active = gi < num_groups;
-        // weights p0..p0+7 lie in bytes q_first .. q_first+2 (the third only for its first digits)
-        uint32_t bv[3] = {kZeroByte, kZeroByte, kZeroByte};
-        uint32_t s = 0;
-        if (active) {
+        bv[0] = bv[1] = bv[2] = kZeroByte;
+        s = 0;
+        if (gi < num_groups) {
             const uint8_t* in = codes + gi * B;
 #pragma unroll
             for (int t = 0; t < 3; ++t)
                 if (q_first + t < B) bv[t] = __ldcs(in + q_first + t);
             s = __ldg(scales + gi);
         }
+    };
+    uint32_t bv_next[3], s_next;
+    load(warp * GPW, bv_next, s_next);
+    for (int64_t base = warp * GPW; base < num_groups; base += stride) {
+        const int64_t gi = base + lane / LPG;
+        const bool active = gi < num_groups;
+        const uint32_t bv[3] = {bv_next[0], bv_next[1], bv_next[2]};
+        const uint32_t s = s_next;
+        load(base + stride, bv_next, s_next);
         // validation of the bytes starting in [p0, p0+8)
         uint32_t bad = 0;
 #pragma unroll
