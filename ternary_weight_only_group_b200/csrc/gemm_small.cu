@@ -47,7 +47,7 @@ struct Smem {
     uint8_t x[STAGES][NT * 128];  // X tiles (UMMA B): NT rows of 128 bytes
     uint8_t c[STAGES][C_STAGE];   // code-byte windows
     float red[WM * NT];           // partials pushed by the cluster: [rank][row of owner][token]
-    uint2 lut[256];
+    uint32_t lut[256];                // byte -> PRMT selectors of its digits 0..3
     uint64_t full_x[STAGES], full_c[STAGES], full_w[STAGES], empty[STAGES], done;
     uint32_t tmem_base;
     int abort_flag;
@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_small_kernel(const __grid_co
     constexpr uint32_t kCols = NT < 32 ? 32 : NT;
     volatile int* abort_flag = &sm.abort_flag;
 
-    fill_digit_selector_lut(sm.lut, threadIdx.x, kThreads);
+    fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(&sm.full_x[st], 1);

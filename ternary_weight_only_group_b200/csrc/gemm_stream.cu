@@ -46,7 +46,7 @@ struct Smem {
     uint8_t w[STAGES][W_STAGE];     // decoded W stages (UMMA A), 1024-byte aligned
     uint8_t x[STAGES][NT * 128];    // X stages (UMMA B): NT rows of 128 bytes
     uint8_t win[2][CR][WM * WIN];   // code windows + scales, per decoder group
-    uint2 lut[256];
+    uint32_t lut[256];                // byte -> PRMT selectors of its digits 0..3
     uint64_t full_x[STAGES], full_w[STAGES], empty[STAGES];
     uint64_t tfull[2], tempty[2], done;
     uint32_t tmem_base;
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     constexpr uint32_t kCols = 2 * NT < 32 ? 32 : 2 * NT;
     volatile int* abort_flag = &sm.abort_flag;
 
-    fill_digit_selector_lut(sm.lut, threadIdx.x, kThreads);
+    fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(&sm.full_x[st], 1);

@@ -57,7 +57,7 @@ struct Smem {
     uint8_t a[STAGES][2][A_SUB];     // X subtiles, 1024-byte aligned
     uint8_t b[STAGES][B_STAGE];      // decoded W tiles
     uint8_t c[STAGES][C_STAGE];      // packed code bytes of the stage (TMA mode)
-    uint2 lut[256];                  // byte -> PRMT selectors of its five weights
+    uint32_t lut[256];                // byte -> PRMT selectors of its digits 0..3
     uint64_t full_a[STAGES], full_c[STAGES], full_b[STAGES], empty[STAGES], done;
     uint32_t tmem_base;
     int abort_flag;
@@ -77,7 +77,9 @@ struct Params {
     int y_vec;  // Y rows allow 16-byte vector stores (base aligned, N a multiple of 16 bytes)
 };
 
-template <bool CODES_TMA>
+// TBN: W rows per tile (256, or 224 when that leaves a fuller last wave);
+// buffers and tensor memory are laid out for 256.
+template <bool CODES_TMA, int TBN>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                               const __grid_constant__ CUtensorMap tmap_c,
                                                               const Params p) {
@@ -85,11 +87,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     Smem& sm = *reinterpret_cast<Smem*>(smem_raw + ((1024 - (s32(smem_raw) & 1023)) & 1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m_tile = blockIdx.x / p.n_tiles, n_tile = blockIdx.x % p.n_tiles;
-    const int64_t m0 = (int64_t)m_tile * BM, n0 = (int64_t)n_tile * BN;
+    const int64_t m0 = (int64_t)m_tile * BM, n0 = (int64_t)n_tile * TBN;
     const int nk = p.K / BK;
     volatile int* abort_flag = &sm.abort_flag;
 
-    fill_digit_selector_lut(sm.lut, threadIdx.x, kThreads);
+    fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(&sm.full_a[st], 1);
@@ -135,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                     int g, c0, q_lo;
                     stage_geom(kb, g, c0, q_lo);
                     const int gb = g * p.B + q_lo;
-                    mbar_arrive_expect_tx(&sm.full_c[st], C_STAGE);
+                    mbar_arrive_expect_tx(&sm.full_c[st], (uint32_t)TBN * C_ROW);  // the TMA box is TBN rows
                     tma_load_2d(sm.c[st], &tmap_c, gb & ~15, (int)n0, &sm.full_c[st]);
                 }
                 ++issued;
@@ -154,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     } else if (warp == 1) {
         // ---------------- MMA issuer: two 128 x 256 x 16 MMAs per k-step
         if (lane == 0) {
-            const uint32_t idesc = instr_desc(UM, BN);
+            const uint32_t idesc = instr_desc(UM, TBN);
             for (int kb = 0; kb < nk; ++kb) {
                 const int st = kb % STAGES, use = kb / STAGES;
                 if (!mbar_wait(&sm.full_a[st], use & 1, abort_flag)) break;
@@ -211,8 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
                 if (ql < 14) lastb = __ldg(crow + (int64_t)g * p.B + p.B - 1);
             }
-            decode_stage64(sm.lut, bytes, c0 - 5 * q_lo, ql < 14, lastb, p.pad_base, p.pad_span, sc,
-                           sm.b[st] + t * 128, t & 7);
+            if (t < TBN)
+                decode_stage64(sm.lut, bytes, c0 - 5 * q_lo, ql < 14, lastb, p.pad_base, p.pad_span, sc,
+                               sm.b[st] + t * 128, t & 7);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_b[st]);
@@ -226,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             if (ok) {
                 for (int sub = 0; sub < 2; ++sub) {
                     const int64_t m = m0 + sub * UM + 32 * q + lane;
-                    for (int c = 0; c < BN / 32; ++c) {
+                    for (int c = 0; c < TBN / 32; ++c) {
                         uint32_t r[32];
                         tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(sub * BN + 32 * c), r);
                         const int64_t nb = n0 + 32 * c;
@@ -339,7 +342,6 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
                            int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err, cudaStream_t stream,
                            int sm_count, bool* handled) {
     using namespace gemm;
-    (void)sm_count;
     *handled = false;
     // Shapes this kernel covers: K a multiple of the 64-column stage, G a
     // multiple of 64 (a stage never crosses a group).
@@ -354,8 +356,16 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
         return cudaErrorInvalidValue;
     // Codes by TMA when their rows are 16-byte multiples and the base is 16-byte aligned.
     const bool codes_tma = (row_bytes % 16 == 0) && ((reinterpret_cast<uintptr_t>(codes) & 15) == 0);
+    // W rows per tile: 256, or 224 when the grid then ends in a fuller wave
+    // (fewer waves x tile width; every CTA runs one tile, one CTA per SM)
+    const int64_t m_tiles = (M + BM - 1) / BM;
+    auto cost = [&](int bn) {
+        const int64_t tiles = m_tiles * ((N + bn - 1) / bn);
+        return ((tiles + sm_count - 1) / sm_count) * bn;
+    };
+    const int tbn = cost(224) < cost(256) ? 224 : 256;
     if (codes_tma && !encode_tmap_2d(&tmap_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<uint8_t*>(codes),
-                                     (uint64_t)row_bytes, (uint64_t)N, (uint64_t)row_bytes, C_ROW, BN,
+                                     (uint64_t)row_bytes, (uint64_t)N, (uint64_t)row_bytes, C_ROW, (uint32_t)tbn,
                                      CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     Params p{};
@@ -370,17 +380,17 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
     p.B = B;
     p.ng = (int)(K / G);
     p.row_bytes = row_bytes;
-    p.n_tiles = (int)((N + BN - 1) / BN);
+    p.n_tiles = (int)((N + tbn - 1) / tbn);
     padding_range(G, p.pad_base, p.pad_span);
     p.y_bf16 = y_bf16;
     p.y_vec = ((reinterpret_cast<uintptr_t>(Y) & 15) == 0) && ((N * (y_bf16 ? 2 : 4)) % 16 == 0);
-    const int64_t m_tiles = (M + BM - 1) / BM;
     const int64_t grid = m_tiles * p.n_tiles;
     if (grid > 0x7FFFFFFF) return cudaSuccess;
     const size_t smem = gemm_smem_bytes();
-    auto kern = codes_tma ? gemm_tc_kernel<true> : gemm_tc_kernel<false>;
-    static std::atomic<int> smem_set[2];
-    std::atomic<int>& slot = smem_set[codes_tma ? 1 : 0];
+    auto kern = codes_tma ? (tbn == 224 ? gemm_tc_kernel<true, 224> : gemm_tc_kernel<true, 256>)
+                          : (tbn == 224 ? gemm_tc_kernel<false, 224> : gemm_tc_kernel<false, 256>);
+    static std::atomic<int> smem_set[4];
+    std::atomic<int>& slot = smem_set[(codes_tma ? 2 : 0) + (tbn == 224 ? 1 : 0)];
     if ((int)smem > slot.load()) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;

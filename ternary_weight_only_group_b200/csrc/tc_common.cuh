@@ -158,19 +158,25 @@ __device__ __forceinline__ void window_bytes(const uint8_t* row32, int off, uint
 // bytes q_lo = c0 / 5 .. q_lo + 13 of the group (those past the group only
 // feed digits past the stage, so their values do not matter).  When the
 // stage holds the group's last byte (check_pad), `lastb` is that byte, and a
-// canonical one lies in [pad_base, pad_base + pad_span).  `lut` maps a byte
-// to its five PRMT selectors with digit d -> 0x10 + 0x22 d over V = {-s, 0},
-// Z = {+s, NaN} (bytes >= 243 select NaN).  The selector stream of the 14
+// canonical one lies in [pad_base, pad_base + pad_span).  `lut4` maps a byte
+// to the PRMT selectors of its digits 0..3 (digit d -> 0x10 + 0x22 d over
+// V = {-s, 0}, Z = {+s, NaN}; bytes >= 243 select NaN); digit 4 is
+// floor(b / 81) = (b * 810) >> 16, exact for every byte, and 3 (NaN) for
+// b >= 243.  Four-byte entries halve the bank conflicts of the lookups.  The selector stream of the 14
 // bytes is packed into words by PRMT and funnel-shifted by r0 bytes, so every
 // stage takes the same code.  A rejected scale or padding digit makes the
 // row's stage NaN.  Writes the 128-byte swizzled K-major tile row.
-__device__ __forceinline__ void decode_stage64(const uint2* lut, const uint32_t (&bytes)[14], int r0,
+__device__ __forceinline__ void decode_stage64(const uint32_t* lut4, const uint32_t (&bytes)[14], int r0,
                                                bool check_pad, uint32_t lastb, uint32_t pad_base,
                                                uint32_t pad_span, uint32_t scale_bits, uint8_t* tile_row,
                                                int row_in_atom) {
     uint2 e[14];
 #pragma unroll
-    for (int i = 0; i < 14; ++i) e[i] = lut[bytes[i] & 0xFFu];
+    for (int i = 0; i < 14; ++i) {
+        const uint32_t b = bytes[i] & 0xFFu;
+        e[i].x = lut4[b];                            // selectors of digits 0..3
+        e[i].y = 0x10u + 0x22u * ((b * 810u) >> 16);  // digit 4 = floor(b / 81), 3 for b >= 243
+    }
     uint32_t W[17];
 #pragma unroll
     for (int h = 0; h < 3; ++h) {

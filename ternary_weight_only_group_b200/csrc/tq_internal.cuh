@@ -168,6 +168,18 @@ __device__ __forceinline__ void eight_selectors(const uint2* sel_lut, uint32_t b
 }
 
 // Fills a byte -> selector-bytes table (digit i in byte i) for the {-s, 0, +s, NaN} layout.
+// Selectors of digits 0..3 of every byte (bytes >= 243: all NaN).
+__device__ __forceinline__ void fill_digit_selector_lut4(uint32_t* lut4, int tid, int nthreads) {
+    for (int b = tid; b < 256; b += nthreads) {
+        uint32_t w = 0, v = (uint32_t)b;
+        for (int i = 0; i < 4; ++i) {
+            w |= digit_selector(b >= 243 ? 3u : v % 3u) << (8 * i);
+            v /= 3u;
+        }
+        lut4[b] = w;
+    }
+}
+
 __device__ __forceinline__ void fill_digit_selector_lut(uint2* sel_lut, int tid, int nthreads) {
     for (int b = tid; b < 256; b += nthreads) {
         uint32_t sv[5];
