@@ -385,15 +385,16 @@ def bench_gemv_stream(tq, args, world, peaks):
 
 
 def bench_gemv_shapes(tq, args, world, peaks):
-    """Each decode projection alone (M=1, both G): per-launch time over 160
-    weight copies (130-138 MB, more than the 126 MB L2) replayed from a CUDA
+    """Each decode projection alone (M=1, both G), and gate and up stacked as
+    one [7168 x 1024] matrix (one launch for both): per-launch time over 160
+    weight copies (130-275 MB, more than the 126 MB L2) replayed from a CUDA
     graph."""
     import torch
     res = {}
+    shapes = [(n, nk) for n, nk in FFN.items() if n != "up"]
+    shapes.append(("gateup", (2 * FFN["gate"][0], FFN["gate"][1])))  # gate and up stacked: one launch
     for G in GROUPS:
-        for name, (N, K) in FFN.items():
-            if name == "up":
-                continue
+        for name, (N, K) in shapes:
             packs = []
             for c in range(160):
                 W = device_weights(N, K, seed=7000 + c)

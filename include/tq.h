@@ -132,7 +132,8 @@ TQ_API tq_status tq_gemv(const void *X_bf16, int64_t M, const uint8_t *codes, co
  * Fused unpack-and-scale matmul for prefill: same result definition as
  * tq_gemv, computed on the tensor cores (tcgen05, fp32 accumulators in
  * tensor memory) from bf16 weights decoded on chip: What = t * RNE_bf16(s).
- * Same arguments and alignment rules as tq_gemv.
+ * Same arguments, alignment and ordering rules as tq_gemv (with M <= 64
+ * the small-M kernels are launched as programmatic dependents too).
  */
 TQ_API tq_status tq_gemm(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
                   int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,

@@ -82,6 +82,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_small_kernel(const __grid_co
     constexpr uint32_t kCols = NT < 32 ? 32 : NT;
     volatile int* abort_flag = &sm.abort_flag;
 
+    // Dependent launches may start now: only the X loads below wait for the
+    // preceding kernel (codes and scales are weights, see tq_gemv's ordering
+    // rule); every Y store follows MMAs that consumed X.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
@@ -115,6 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_small_kernel(const __grid_co
 
     if (warp == 0) {
         if (lane == 0) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");  // X comes from the preceding kernel
             int issued = 0;
             for (int i = 0; i < nkl; ++i) {
                 const int kb = kb_lo + i, st = i % STAGES, use = i / STAGES;
@@ -286,13 +291,15 @@ static cudaError_t launch_nt(const CUtensorMap& tx, const CUtensorMap& tc_, cons
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = p.CS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, tx, tc_, p);
 }
 

@@ -117,6 +117,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     constexpr uint32_t kCols = 2 * NT < 32 ? 32 : 2 * NT;
     volatile int* abort_flag = &sm.abort_flag;
 
+    // Dependent launches may start now: only the X loads below wait for the
+    // preceding kernel (codes and scales are weights, see tq_gemv's ordering
+    // rule); every Y store follows MMAs that consumed X.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
@@ -146,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
 
     if (warp == 0) {
         if (lane == 0) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");  // X comes from the preceding kernel
             int issued = 0;
             for (int i = 0; i < total; ++i) {
                 const int kb = i % nk, st = i % STAGES, use = i / STAGES;
@@ -317,8 +322,17 @@ static cudaError_t launch_nt(const CUtensorMap& tx, const Params& p, int grid, c
         if (e != cudaSuccess) return e;
         smem_set.store((int)smem);
     }
-    kern<<<grid, kThreads, smem, stream>>>(tx, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tx, p);
 }
 
 }  // namespace stream
