@@ -35,6 +35,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ternary x bf16 GEMV HBM GB/s (% of peak); prefill GEMM TFLOP/s; pack GB/s"
+# DRAM bytes (read + write) of one gemv_predecode_kernel launch per decode
+# shape (N, K, G), M=1, from an ncu capture of dram__bytes_read.sum +
+# dram__bytes_write.sum on `bench.py --only gemv` (one launch per shape).
+# Valid for the kernel as captured; set to None when it changes.
+PREDECODE_DRAM_BYTES = {(3584, 1024, 64): 906496, (1024, 3584, 64): 911104,
+                        (3584, 1024, 128): 848896, (1024, 3584, 128): 854528}
 FFN = {"gate": (3584, 1024), "up": (3584, 1024), "down": (1024, 3584)}
 MSWEEP = {"q": (1536, 1536), "o": (1536, 1536), "gate": (4096, 1536), "up": (4096, 1536), "down": (1536, 4096)}
 MSWEEP_LAYERS = 28
@@ -306,6 +312,9 @@ def run_ours(args, rank, world, local):
     e2e = world * step_bytes * K_steps / (ms_e2e * 1e-3) / 1e9
     per_launch_us = ms_step * 1e3 / launches_per_step
     avg_bytes = step_bytes / launches_per_step
+    traffic = None  # measured DRAM bytes per launch, averaged like avg_bytes
+    if PREDECODE_DRAM_BYTES is not None and all((N, K, G) in PREDECODE_DRAM_BYTES for (G, l, name, N, K, xo, yo) in calls):
+        traffic = round(sum(PREDECODE_DRAM_BYTES[(N, K, G)] for (G, l, name, N, K, xo, yo) in calls) / len(calls), 1)
     achieved = avg_bytes / (per_launch_us * 1e-6) / 1e9
     if rank != 0:
         return
@@ -338,7 +347,7 @@ def run_ours(args, rank, world, local):
             "peak_source": peaks["source"],
             "per_launch_us": round(per_launch_us, 3),
             "bytes_per_launch": round(avg_bytes, 1),
-            "traffic": None,
+            "traffic": traffic,
         },
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e, 2), "unit": "GB/s",
