@@ -5,10 +5,11 @@
 // stored scale produces a zero group (the paragraph after it).
 //
 // Fast path (G = 8 * 2^k, 8 <= G <= 256): G/8 lanes per group, each lane
-// writes 8 consecutive bf16 with one 16-byte store.  The lanes of a group
-// validate the bytes that start in their range (the union is every byte of
-// the group), OR the verdict across the segment, and a rejected group is
-// written as bf16 NaN.  Digits come from a 256-entry shared-memory table.
+// writes 8 consecutive bf16 with one 16-byte store.  Each lane checks the
+// code bytes it loads (>= 243 invalid; the group's last byte against the
+// canonical padding range), the verdicts are OR-ed across the group's lanes,
+// and a rejected group is written as bf16 NaN.  Selectors come from a
+// 256-entry shared-memory table.
 #include "tq_internal.cuh"
 
 namespace tq {
@@ -21,6 +22,9 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
     constexpr int GPW = 32 / LPG;
     constexpr int B = bytes_per_group(G);
     constexpr int REAL = G - 5 * (B - 1);  // real digits in the last byte (1..5)
+    // a canonical last byte has digits REAL..4 equal to 1: [PAD_BASE, PAD_BASE + 3^REAL)
+    constexpr uint32_t PAD_SPAN = REAL == 1 ? 3u : (REAL == 2 ? 9u : (REAL == 3 ? 27u : 81u));
+    constexpr uint32_t PAD_BASE = REAL == 1 ? 120u : (REAL == 2 ? 117u : (REAL == 3 ? 108u : 81u));
     __shared__ uint2 sel_lut[256];
     fill_digit_selector_lut(sel_lut, threadIdx.x, blockDim.x);
     __syncthreads();
@@ -59,17 +63,15 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
         const uint32_t bv[3] = {bv_next[0], bv_next[1], bv_next[2]};
         const uint32_t s = s_next;
         load(base + stride, bv_next, s_next);
-        // validation of the bytes starting in [p0, p0+8)
+        // validation of the lane's bytes (a byte seen by two lanes is checked
+        // twice; the verdicts are OR-ed): >= 243 is invalid; the group's last
+        // byte must lie in [PAD_BASE, PAD_BASE + PAD_SPAN) (padding digits 1)
         uint32_t bad = 0;
 #pragma unroll
         for (int t = 0; t < 3; ++t) {
-            const int q = q_first + t;
-            if (5 * q >= p0 && 5 * q < p0 + 8 && q < B) {
-                if (bv[t] >= 243) bad |= TQ_DERR_BYTE;
-                else if (q == B - 1 && REAL < 5 &&
-                         (byte_digit_pattern(bv[t]) & padding_mask(REAL)) != padding_ones(REAL))
-                    bad |= TQ_DERR_PADDING;
-            }
+            const uint32_t b = bv[t];  // 121 (valid) past the group
+            if (b >= 243) bad |= TQ_DERR_BYTE;
+            else if (REAL < 5 && q_first + t == B - 1 && b - PAD_BASE >= PAD_SPAN) bad |= TQ_DERR_PADDING;
         }
         if (sub == 0 && scale_is_bad(s)) bad |= TQ_DERR_SCALE;
         bad = seg_or_u32(bad, LPG);
