@@ -97,6 +97,91 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
+// G >= 16: G/16 lanes per group, 16 weights per lane (two 16-byte stores).
+// The lane's weights span four code bytes; their 20 selectors are packed into
+// five words by PRMT and funnel-shifted to the lane's first weight, so the
+// fixed per-lane work (loads, validation, scale) covers twice the weights.
+template <int G>
+__global__ void __launch_bounds__(256) unpack16_kernel(
+    const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales, int64_t num_groups,
+    uint16_t* __restrict__ out, uint32_t* __restrict__ d_err) {
+    constexpr int LPG = G / 16;
+    constexpr int GPW = 32 / LPG;
+    constexpr int B = bytes_per_group(G);
+    constexpr int REAL = G - 5 * (B - 1);
+    constexpr uint32_t PAD_SPAN = REAL == 1 ? 3u : (REAL == 2 ? 9u : (REAL == 3 ? 27u : 81u));
+    constexpr uint32_t PAD_BASE = REAL == 1 ? 120u : (REAL == 2 ? 117u : (REAL == 3 ? 108u : 81u));
+    __shared__ uint2 sel_lut[256];
+    fill_digit_selector_lut(sel_lut, threadIdx.x, blockDim.x);
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % LPG;
+    const int p0 = 16 * sub;
+    const int q_first = p0 / 5;  // weights p0..p0+15 lie in bytes q_first .. q_first+3
+    const uint32_t shift = 8u * (uint32_t)(p0 - 5 * q_first);
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t stride = nwarps * GPW;
+    uint32_t err_acc = 0;
+    auto load = [&](int64_t base, uint32_t (&bv)[4], uint32_t& s) {
+        const int64_t gi = base + lane / LPG;
+        bv[0] = bv[1] = bv[2] = bv[3] = kZeroByte;
+        s = 0;
+        if (gi < num_groups) {
+            const uint8_t* in = codes + gi * B;
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                if (q_first + t < B) bv[t] = __ldcs(in + q_first + t);
+            s = __ldg(scales + gi);
+        }
+    };
+    uint32_t bv_next[4], s_next;
+    load(warp * GPW, bv_next, s_next);
+    for (int64_t base = warp * GPW; base < num_groups; base += stride) {
+        const int64_t gi = base + lane / LPG;
+        const bool active = gi < num_groups;
+        const uint32_t bv[4] = {bv_next[0], bv_next[1], bv_next[2], bv_next[3]};
+        const uint32_t s = s_next;
+        load(base + stride, bv_next, s_next);
+        uint32_t bad = scale_is_bad(s) ? TQ_DERR_SCALE : 0u;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const uint32_t b = bv[t];  // 121 (valid) past the group
+            if (b >= 243) bad |= TQ_DERR_BYTE;
+            else if (REAL < 5 && q_first + t == B - 1 && b - PAD_BASE >= PAD_SPAN) bad |= TQ_DERR_PADDING;
+        }
+        bad = seg_or_u32(bad, LPG);
+        if (!active) bad = 0;
+        // selector stream of the four bytes (5 per byte), then the lane's 16
+        const uint2 e0 = sel_lut[bv[0]], e1 = sel_lut[bv[1]], e2 = sel_lut[bv[2]], e3 = sel_lut[bv[3]];
+        const uint32_t W[5] = {e0.x, prmt32(e0.y, e1.x, 0x6540u), prmt32(prmt32(e1.x, e1.y, 0x0043u), e2.x, 0x5410u),
+                               prmt32(prmt32(e2.x, e2.y, 0x0432u), e3.x, 0x4210u), prmt32(e3.x, e3.y, 0x4321u)};
+        uint32_t V, Z;  // {-s, 0} and {+s, NaN}
+        if (bad) {
+            V = Z = 0x7FC07FC0u;
+        } else {
+            const uint32_t mag = (s == 0) ? 0u : scale_to_bf16_bits((uint16_t)s);
+            V = mag ? (mag | 0x8000u) : 0u;
+            Z = mag | 0x7FC00000u;
+        }
+        uint32_t v[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t o = __funnelshift_rc(W[j], W[j + 1], shift);
+            v[2 * j] = prmt32(V, Z, o);
+            v[2 * j + 1] = prmt32(V, Z, o >> 16);
+        }
+        if (active) {
+            uint4* dst = reinterpret_cast<uint4*>(out + gi * G + p0);
+            __stcs(dst, make_uint4(v[0], v[1], v[2], v[3]));
+            __stcs(dst + 1, make_uint4(v[4], v[5], v[6], v[7]));
+            if (sub == 0) err_acc |= bad;
+        }
+    }
+    if (err_acc && d_err) atomicOr(d_err, err_acc);
+}
+
 // Any G: one thread per group.
 __global__ void __launch_bounds__(128) unpack_generic_kernel(
     const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales, int64_t num_groups,
@@ -142,13 +227,17 @@ cudaError_t launch_unpack(const uint8_t* codes, const uint16_t* scales, int64_t 
     };
 #define TQ_UP_CASE(GG)                                                                          \
     case GG: {                                                                                  \
-        const int64_t threads = (num_groups + (32 / (GG / 8)) - 1) / (32 / (GG / 8)) * 32;      \
-        unpack_pow2_kernel<GG><<<grid(threads, 256), 256, 0, stream>>>(codes, scales, num_groups, \
-                                                                      out, d_err);              \
+        const int64_t threads = (num_groups + (32 / (GG / 16)) - 1) / (32 / (GG / 16)) * 32;    \
+        unpack16_kernel<GG><<<grid(threads, 256), 256, 0, stream>>>(codes, scales, num_groups,  \
+                                                                   out, d_err);                 \
         return cudaGetLastError();                                                              \
     }
     switch (G) {
-        TQ_UP_CASE(8)
+        case 8: {
+            const int64_t threads = (num_groups + 3) / 4 * 32;
+            unpack_pow2_kernel<8><<<grid(threads, 256), 256, 0, stream>>>(codes, scales, num_groups, out, d_err);
+            return cudaGetLastError();
+        }
         TQ_UP_CASE(16)
         TQ_UP_CASE(32)
         TQ_UP_CASE(64)
