@@ -129,14 +129,15 @@ __global__ void __launch_bounds__(256) quantize_pack_pow2_kernel(
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
-// One lane per group (G = 8, 16, 32, 64, 128): the group's G weights sit in
-// the lane's registers, so max and sum need no shuffles; every weight's byte
+// One lane per group (G = 8, 16, 32, 64, 128): the group's weights sit in
+// the lane's registers (G = 128: one half at a time, read twice), so max and
+// sum need no shuffles; every weight's byte
 // and power of three are compile-time constants, so encoding is one
 // multiply-add per weight into packed code words; each warp's 32 groups of
 // code bytes are assembled in shared memory and written with 16-byte stores
 // when the destination allows it.  The scale arithmetic is the one above.
 template <int G>
-__global__ void __launch_bounds__(256, G <= 32 ? 3 : (G == 64 ? 2 : 1)) quantize_pack_group_kernel(
+__global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kernel(
     const uint16_t* __restrict__ W, int64_t num_groups, uint8_t* __restrict__ codes,
     uint16_t* __restrict__ scales, uint32_t* __restrict__ d_err) {
     constexpr int NWD = G / 2;                 // 32-bit words of a group
@@ -150,64 +151,140 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : (G == 64 ? 2 : 1)) quantize
     for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); g0 < num_groups; g0 += stride) {
         const int64_t gi = g0 + lane;  // the warp's groups g0 .. g0+31
         const bool active = gi < num_groups;
-        uint32_t h[NWD];
-        {
-            const uint4* src = reinterpret_cast<const uint4*>(W + (active ? gi : 0) * G);
-#pragma unroll
-            for (int k = 0; k < G / 8; ++k) {
-                const uint4 v = __ldg(src + k);
-                h[4 * k] = v.x;
-                h[4 * k + 1] = v.y;
-                h[4 * k + 2] = v.z;
-                h[4 * k + 3] = v.w;
-            }
-        }
-        uint32_t amax = 0;
-#pragma unroll
-        for (int j = 0; j < G; ++j) amax = max(amax, (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu);
-        const uint32_t emax = amax >> 7;
-        const uint32_t thr = emax > 37 ? (emax - 37) << 7 : 0;  // smallest pattern in the exact window
-        double sum = 0.0;
-        uint32_t outside = 0;
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-            const uint32_t a = (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
-            if (a >= thr) sum += bf16_normal_mag_to_f64(a);
-            else outside |= a;
-        }
         uint16_t s = 0;
         uint32_t gerr = 0;
-        if (amax >= 0x7F80u) {
-            gerr = TQ_DERR_WEIGHT;
-        } else if (amax > kTinyMaxBits) {
-            if (outside) {
-                gerr = exact_group_scale(W + (active ? gi : 0) * G, G, &s);
-            } else {
-                const uint16_t bits = __half_as_ushort(__double2half(sum * (1.0 / G)));
-                if (bits >= 0x7C00u) gerr = TQ_DERR_OVERFLOW;
-                else s = bits;
-            }
-        }
-        if (gerr) s = 0;
-        const uint32_t th = trit_threshold(s);
-        // code words: byte q of the group in byte q % 4 of word q / 4; digit
-        // d = t + 1 of weight j adds d * 3^(j % 5) to byte j / 5; positions
-        // j >= G hold the padding digit 1
         uint32_t cw[NCW];
-#pragma unroll
-        for (int i = 0; i < NCW; ++i) cw[i] = 0;
-#pragma unroll
-        for (int j = 0; j < 5 * B; ++j) {
-            const int q = j / 5;
-            const uint32_t pw = (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
-                                << (8 * (q % 4));
-            if (j < G) {
-                const uint32_t hw = h[j >> 1] >> (16 * (j & 1));
-                const uint32_t d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
-                cw[q / 4] += d * pw;
-            } else {
-                cw[q / 4] += pw;  // padding digit 1
+        if constexpr (G <= 64) {
+            uint32_t h[NWD];
+            {
+                const uint4* src = reinterpret_cast<const uint4*>(W + (active ? gi : 0) * G);
+    #pragma unroll
+                for (int k = 0; k < G / 8; ++k) {
+                    const uint4 v = __ldg(src + k);
+                    h[4 * k] = v.x;
+                    h[4 * k + 1] = v.y;
+                    h[4 * k + 2] = v.z;
+                    h[4 * k + 3] = v.w;
+                }
             }
+            uint32_t amax = 0;
+    #pragma unroll
+            for (int j = 0; j < G; ++j) amax = max(amax, (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu);
+            const uint32_t emax = amax >> 7;
+            const uint32_t thr = emax > 37 ? (emax - 37) << 7 : 0;  // smallest pattern in the exact window
+            double sum = 0.0;
+            uint32_t outside = 0;
+    #pragma unroll
+            for (int j = 0; j < G; ++j) {
+                const uint32_t a = (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
+                if (a >= thr) sum += bf16_normal_mag_to_f64(a);
+                else outside |= a;
+            }
+            if (amax >= 0x7F80u) {
+                gerr = TQ_DERR_WEIGHT;
+            } else if (amax > kTinyMaxBits) {
+                if (outside) {
+                    gerr = exact_group_scale(W + (active ? gi : 0) * G, G, &s);
+                } else {
+                    const uint16_t bits = __half_as_ushort(__double2half(sum * (1.0 / G)));
+                    if (bits >= 0x7C00u) gerr = TQ_DERR_OVERFLOW;
+                    else s = bits;
+                }
+            }
+            if (gerr) s = 0;
+            const uint32_t th = trit_threshold(s);
+            // code words: byte q of the group in byte q % 4 of word q / 4; digit
+            // d = t + 1 of weight j adds d * 3^(j % 5) to byte j / 5; positions
+            // j >= G hold the padding digit 1
+    #pragma unroll
+            for (int i = 0; i < NCW; ++i) cw[i] = 0;
+    #pragma unroll
+            for (int j = 0; j < 5 * B; ++j) {
+                const int q = j / 5;
+                const uint32_t pw = (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
+                                    << (8 * (q % 4));
+                if (j < G) {
+                    const uint32_t hw = h[j >> 1] >> (16 * (j & 1));
+                    const uint32_t d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
+                    cw[q / 4] += d * pw;
+                } else {
+                    cw[q / 4] += pw;  // padding digit 1
+                }
+            }
+        } else {
+            // G = 128: the group is read twice in halves of 64 weights, so only
+            // one half (32 words) is live at a time.  Pass 1 takes max, the
+            // smallest nonzero magnitude and the binary64 sum of every nonzero
+            // magnitude; the sum is exact when all of them lie within 2^37 of the
+            // maximum (the same window as above), else the group takes the exact
+            // multi-word path.  Pass 2 re-reads the halves (cache hits) to encode.
+            const uint4* src = reinterpret_cast<const uint4*>(W + (active ? gi : 0) * G);
+            uint32_t amax = 0, amin1 = 0xFFFFFFFFu;  // amin1 = smallest nonzero magnitude - 1
+            double sum = 0.0;
+    #pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t h[32];
+    #pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint4 v = __ldg(src + 8 * half + k);
+                    h[4 * k] = v.x;
+                    h[4 * k + 1] = v.y;
+                    h[4 * k + 2] = v.z;
+                    h[4 * k + 3] = v.w;
+                }
+    #pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    const uint32_t a = (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
+                    amax = max(amax, a);
+                    amin1 = min(amin1, a - 1u);  // a = 0 wraps to the largest value
+                    if (a) sum += bf16_normal_mag_to_f64(a);
+                }
+                asm volatile("" ::: "memory");  // keep the halves' loads apart
+            }
+            const uint32_t emax = amax >> 7;
+            const uint32_t thr = emax > 37 ? (emax - 37) << 7 : 0;
+            const bool outside = amin1 != 0xFFFFFFFFu && amin1 + 1u < thr;
+            if (amax >= 0x7F80u) {
+                gerr = TQ_DERR_WEIGHT;
+            } else if (amax > kTinyMaxBits) {
+                if (outside) {
+                    gerr = exact_group_scale(W + (active ? gi : 0) * G, G, &s);
+                } else {
+                    const uint16_t bits = __half_as_ushort(__double2half(sum * (1.0 / G)));
+                    if (bits >= 0x7C00u) gerr = TQ_DERR_OVERFLOW;
+                    else s = bits;
+                }
+            }
+            if (gerr) s = 0;
+            const uint32_t th = trit_threshold(s);
+    #pragma unroll
+            for (int i = 0; i < NCW; ++i) cw[i] = 0;
+    #pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t h[32];
+    #pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint4 v = __ldg(src + 8 * half + k);
+                    h[4 * k] = v.x;
+                    h[4 * k + 1] = v.y;
+                    h[4 * k + 2] = v.z;
+                    h[4 * k + 3] = v.w;
+                }
+    #pragma unroll
+                for (int jj = 0; jj < 64; ++jj) {
+                    const int j = 64 * half + jj, q = j / 5;
+                    const uint32_t pw = (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
+                                        << (8 * (q % 4));
+                    const uint32_t hw = h[jj >> 1] >> (16 * (jj & 1));
+                    const uint32_t d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
+                    cw[q / 4] += d * pw;
+                }
+                asm volatile("" ::: "memory");
+            }
+    #pragma unroll
+            for (int j = G; j < 5 * B; ++j)  // padding digits 1
+                cw[j / 5 / 4] += (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
+                                 << (8 * ((j / 5) % 4));
         }
         if (active) {
             scales[gi] = s;
