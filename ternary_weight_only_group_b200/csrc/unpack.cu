@@ -111,8 +111,8 @@ __global__ void __launch_bounds__(256) unpack16_kernel(
     constexpr int REAL = G - 5 * (B - 1);
     constexpr uint32_t PAD_SPAN = REAL == 1 ? 3u : (REAL == 2 ? 9u : (REAL == 3 ? 27u : 81u));
     constexpr uint32_t PAD_BASE = REAL == 1 ? 120u : (REAL == 2 ? 117u : (REAL == 3 ? 108u : 81u));
-    __shared__ uint2 sel_lut[256];
-    fill_digit_selector_lut(sel_lut, threadIdx.x, blockDim.x);
+    __shared__ uint32_t lut4[256];  // selectors of digits 0..3; digit 4 = floor(b / 81) by arithmetic
+    fill_digit_selector_lut4(lut4, threadIdx.x, blockDim.x);
     __syncthreads();
 
     const int lane = threadIdx.x & 31;
@@ -154,7 +154,8 @@ __global__ void __launch_bounds__(256) unpack16_kernel(
         bad = seg_or_u32(bad, LPG);
         if (!active) bad = 0;
         // selector stream of the four bytes (5 per byte), then the lane's 16
-        const uint2 e0 = sel_lut[bv[0]], e1 = sel_lut[bv[1]], e2 = sel_lut[bv[2]], e3 = sel_lut[bv[3]];
+        auto rec = [&](uint32_t b) { return make_uint2(lut4[b], 0x10u + 0x22u * ((b * 810u) >> 16)); };
+        const uint2 e0 = rec(bv[0]), e1 = rec(bv[1]), e2 = rec(bv[2]), e3 = rec(bv[3]);
         const uint32_t W[5] = {e0.x, prmt32(e0.y, e1.x, 0x6540u), prmt32(prmt32(e1.x, e1.y, 0x0043u), e2.x, 0x5410u),
                                prmt32(prmt32(e2.x, e2.y, 0x0432u), e3.x, 0x4210u), prmt32(e3.x, e3.y, 0x4321u)};
         uint32_t V, Z;  // {-s, 0} and {+s, NaN}
