@@ -4,7 +4,7 @@
 // Y[n] = sum_k X[k] * What[n][k] with What = t * RNE_bf16(scale) (tiny-llm
 // "Week 2 Day 3: Quantize the Model", "Mathematical Formulation"; the
 // decoding of "precisit/pack-unpack-run", codec.py), fp32 accumulation,
-// 1 <= M <= 4 tokens.
+// 1 <= M <= 8 tokens.
 //
 // In a chain of dependent layers a kernel's weights are known long before its
 // activations.  Each CTA (one per SM, R rows) therefore stages its codes and
@@ -253,23 +253,25 @@ __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_ke
     }
     __syncthreads();
 
-    // ---- work units: (batch of 8 rows, slice of the chunks); with fewer than
-    // eight batches the chunks are split over the idle warps and the slices'
-    // sums meet in shared memory.
-    const int nb = (nrows + 7) >> 3;
+    // ---- work units: (batch of RB rows, slice of the chunks); with fewer
+    // than eight batches the chunks are split over the idle warps and the
+    // slices' sums meet in shared memory.  RB = 8 rows up to 4 tokens, 4 rows
+    // for 8 tokens (the accumulators stay at 32 per lane).
+    constexpr int RB = MT <= 4 ? 8 : 4;
+    const int nb = (nrows + RB - 1) / RB;
     const int ks = nb >= kPdWarps ? 1 : kPdWarps / nb;
     uint32_t err_acc = 0;
     for (int u = warp; u < nb * ks; u += kPdWarps) {
         const int b = u / ks, sl = u - b * ks;
-        const int rb0 = 8 * b;
-        int roff[8];  // element offset of each row (rows past the end repeat the last, never stored)
+        const int rb0 = RB * b;
+        int roff[RB];  // element offset of each row (rows past the end repeat the last, never stored)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) roff[i] = min(rb0 + i, nrows - 1) * K;
-        float acc[MT][8];
+        for (int i = 0; i < RB; ++i) roff[i] = min(rb0 + i, nrows - 1) * K;
+        float acc[MT][RB];
 #pragma unroll
         for (int m = 0; m < MT; ++m)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[m][i] = 0.f;
+            for (int i = 0; i < RB; ++i) acc[m][i] = 0.f;
 #pragma unroll 2
         for (int c = lane + 32 * sl; c < nchunk; c += 32 * ks) {
             uint32_t xx[MT][4];
@@ -283,7 +285,7 @@ __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_ke
             }
             const int pc8 = 8 * pd_swizzle(c);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < RB; ++i) {
                 const uint4 wv = *reinterpret_cast<const uint4*>(w + roff[i] + pc8);
                 const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
@@ -298,8 +300,8 @@ __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_ke
         }
         float tot[MT];
 #pragma unroll
-        for (int m = 0; m < MT; ++m) tot[m] = pd_transpose_reduce<8>(acc[m]);
-        if (lane < 8) {
+        for (int m = 0; m < MT; ++m) tot[m] = pd_transpose_reduce<RB>(acc[m]);
+        if (lane < RB) {
             const int rr = rb0 + lane;
             if (ks == 1) {
                 if (rr < nrows) {
@@ -311,7 +313,7 @@ __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_ke
                 }
             } else {
 #pragma unroll
-                for (int m = 0; m < MT; ++m) red[(sl * (8 * nb) + rr) * MT + m] = tot[m];  // ks * 8 * nb <= 64
+                for (int m = 0; m < MT; ++m) red[(sl * (RB * nb) + rr) * MT + m] = tot[m];  // ks * RB * nb <= 64
             }
         }
     }
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_ke
             for (int m = 0; m < MT; ++m) tot[m] = 0.f;
             for (int sl = 0; sl < ks; ++sl)
 #pragma unroll
-                for (int m = 0; m < MT; ++m) tot[m] += red[(sl * (8 * nb) + rr) * MT + m];
+                for (int m = 0; m < MT; ++m) tot[m] += red[(sl * (RB * nb) + rr) * MT + m];
             if (tot[0] != tot[0])
                 err_acc |= scan_row_errors(codes + (row0 + rr) * ng * B, scales + (row0 + rr) * ng, ng, G, B);
 #pragma unroll
@@ -377,9 +379,9 @@ static cudaError_t launch_pd_g(int G, const uint16_t* X, int M, const uint8_t* c
 cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                   int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                                   cudaStream_t stream, int sm_count) {
-    if (M < 1 || M > 4 || K % 512 != 0 || N < 1 || K > 65536) return cudaErrorNotSupported;
+    if (M < 1 || M > 8 || K % 512 != 0 || N < 1 || K > 65536) return cudaErrorNotSupported;
     if (G != 8 && G != 16 && G != 32 && G != 64 && G != 128 && G != 256) return cudaErrorNotSupported;
-    const int MT = M == 1 ? 1 : (M == 2 ? 2 : 4);
+    const int MT = M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8));
     const int64_t ng = K / G, B = bytes_per_group(G);
     // one CTA per SM if it fits (later launches then decode beside it), else two
     for (int per_sm = 1; per_sm <= 2; ++per_sm) {
@@ -391,7 +393,8 @@ cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* c
         const int grid = (int)((N + R - 1) / R);
         if (MT == 1) return launch_pd_g<1>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
         if (MT == 2) return launch_pd_g<2>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
-        return launch_pd_g<4>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
+        if (MT == 4) return launch_pd_g<4>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
+        return launch_pd_g<8>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
     }
     return cudaErrorNotSupported;
 }

@@ -113,11 +113,12 @@ def test_row_counts(N):
 
 @pytest.mark.parametrize("N,K,G", [(9477, 512, 64), (2000, 512, 32), (150, 4096, 256), (1500, 3072, 8),
                                    (700, 2048, 128), (300, 1024, 16)])
-@pytest.mark.parametrize("M", [1, 4])
+@pytest.mark.parametrize("M", [1, 4, 6, 8])
 def test_predecode_row_batches(N, K, G, M):
-    """One to four tokens over matrices whose per-CTA rows fit in shared
-    memory: more than eight 8-row batches per CTA, chunks split over two to
-    eight warps, ragged last CTA, one or two CTAs per SM."""
+    """One to eight tokens over matrices whose per-CTA rows fit in shared
+    memory: more than eight row batches per CTA (8 rows, 4 rows from 5
+    tokens), chunks split over two to eight warps, ragged last CTA, one or
+    two CTAs per SM, tokens padded with zeros up to the kernel's 4 or 8."""
     W = synthetic.weights(N, K, index=N + K)
     X = synthetic.activations(M, K)
     check(X, W, G)
