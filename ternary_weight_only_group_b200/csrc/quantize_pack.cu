@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
             uint32_t h[NWD];
             {
                 const uint4* src = reinterpret_cast<const uint4*>(W + (active ? gi : 0) * G);
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < G / 8; ++k) {
                     const uint4 v = __ldg(src + k);
                     h[4 * k] = v.x;
@@ -168,13 +168,13 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
                 }
             }
             uint32_t amax = 0;
-    #pragma unroll
+#pragma unroll
             for (int j = 0; j < G; ++j) amax = max(amax, (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu);
             const uint32_t emax = amax >> 7;
             const uint32_t thr = emax > 37 ? (emax - 37) << 7 : 0;  // smallest pattern in the exact window
             double sum = 0.0;
             uint32_t outside = 0;
-    #pragma unroll
+#pragma unroll
             for (int j = 0; j < G; ++j) {
                 const uint32_t a = (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
                 if (a >= thr) sum += bf16_normal_mag_to_f64(a);
@@ -196,9 +196,9 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
             // code words: byte q of the group in byte q % 4 of word q / 4; digit
             // d = t + 1 of weight j adds d * 3^(j % 5) to byte j / 5; positions
             // j >= G hold the padding digit 1
-    #pragma unroll
+#pragma unroll
             for (int i = 0; i < NCW; ++i) cw[i] = 0;
-    #pragma unroll
+#pragma unroll
             for (int j = 0; j < 5 * B; ++j) {
                 const int q = j / 5;
                 const uint32_t pw = (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
@@ -221,10 +221,10 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
             const uint4* src = reinterpret_cast<const uint4*>(W + (active ? gi : 0) * G);
             uint32_t amax = 0, amin1 = 0xFFFFFFFFu;  // amin1 = smallest nonzero magnitude - 1
             double sum = 0.0;
-    #pragma unroll
+#pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t h[32];
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint4 v = __ldg(src + 8 * half + k);
                     h[4 * k] = v.x;
@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
                     h[4 * k + 2] = v.z;
                     h[4 * k + 3] = v.w;
                 }
-    #pragma unroll
+#pragma unroll
                 for (int j = 0; j < 64; ++j) {
                     const uint32_t a = (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
                     amax = max(amax, a);
@@ -257,12 +257,12 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
             }
             if (gerr) s = 0;
             const uint32_t th = trit_threshold(s);
-    #pragma unroll
+#pragma unroll
             for (int i = 0; i < NCW; ++i) cw[i] = 0;
-    #pragma unroll
+#pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t h[32];
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint4 v = __ldg(src + 8 * half + k);
                     h[4 * k] = v.x;
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
                     h[4 * k + 2] = v.z;
                     h[4 * k + 3] = v.w;
                 }
-    #pragma unroll
+#pragma unroll
                 for (int jj = 0; jj < 64; ++jj) {
                     const int j = 64 * half + jj, q = j / 5;
                     const uint32_t pw = (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
                 }
                 asm volatile("" ::: "memory");
             }
-    #pragma unroll
+#pragma unroll
             for (int j = G; j < 5 * B; ++j)  // padding digits 1
                 cw[j / 5 / 4] += (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
                                  << (8 * ((j / 5) % 4));
