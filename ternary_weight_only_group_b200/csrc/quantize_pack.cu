@@ -16,6 +16,8 @@
 // path instead.  Each lane loads the next pass's weights before it computes
 // the current pass.  Other G use one thread per group with the multi-word
 // path.
+#include <atomic>
+
 #include "tq_internal.cuh"
 
 namespace tq {
@@ -148,7 +150,32 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
     const bool vec_out = (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
     uint32_t err_acc = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t g0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); g0 < num_groups; g0 += stride) {
+    // G <= 64: the warp's next 32 groups are copied into a double-buffered
+    // shared-memory ring by coalesced cp.async while the current 32 are
+    // quantized (the loads cost no registers, which the group occupies).
+    // Rows are padded to 2G + 16 bytes so that the 16-byte reads of the
+    // lanes' own groups are free of bank conflicts.
+    constexpr int RS = 2 * G + 16;
+    extern __shared__ __align__(16) uint8_t qring[];  // [2][8 warps][32 groups][RS]
+    auto issue = [&](int64_t gb, int buf) {
+        if constexpr (G <= 64) {
+            uint8_t* base = qring + ((size_t)buf * 8 + wib) * 32 * RS;
+#pragma unroll
+            for (int k = 0; k < G / 8; ++k) {
+                const int c = lane + 32 * k, grp = c / (G / 8), piece = c - grp * (G / 8);
+                if (gb + grp < num_groups)
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                                     (uint32_t)__cvta_generic_to_shared(base + grp * RS + piece * 16)),
+                                 "l"(__cvta_generic_to_global(W + (gb + grp) * G + piece * 8))
+                                 : "memory");
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        }
+    };
+    const int64_t g_first = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+    if (g_first < num_groups) issue(g_first, 0);
+    int pass = 0;
+    for (int64_t g0 = g_first; g0 < num_groups; g0 += stride, ++pass) {
         const int64_t gi = g0 + lane;  // the warp's groups g0 .. g0+31
         const bool active = gi < num_groups;
         uint16_t s = 0;
@@ -157,15 +184,20 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
         if constexpr (G <= 64) {
             uint32_t h[NWD];
             {
-                const uint4* src = reinterpret_cast<const uint4*>(W + (active ? gi : 0) * G);
+                issue(g0 + stride, (pass + 1) & 1);  // that buffer was read last pass
+                asm volatile("cp.async.wait_group 1;" ::: "memory");
+                __syncwarp();
+                const uint4* row =
+                    reinterpret_cast<const uint4*>(qring + (((size_t)(pass & 1) * 8 + wib) * 32 + lane) * RS);
 #pragma unroll
                 for (int k = 0; k < G / 8; ++k) {
-                    const uint4 v = __ldg(src + k);
+                    const uint4 v = row[k];
                     h[4 * k] = v.x;
                     h[4 * k + 1] = v.y;
                     h[4 * k + 2] = v.z;
                     h[4 * k + 3] = v.w;
                 }
+                __syncwarp();  // every lane has read this buffer before it is refilled
             }
             uint32_t amax = 0;
 #pragma unroll
@@ -305,7 +337,26 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
         }
         __syncwarp();
     }
+    if constexpr (G <= 64) asm volatile("cp.async.wait_all;" ::: "memory");
     if (err_acc && d_err) atomicOr(d_err, err_acc);
+}
+
+// Dynamic shared memory of quantize_pack_group_kernel<G>: the load ring.
+static size_t quantize_ring_bytes(int G) { return G <= 64 ? (size_t)2 * 8 * 32 * (2 * G + 16) : 0; }
+
+template <int G>
+static cudaError_t launch_quantize_group(const uint16_t* W, int64_t num_groups, uint8_t* codes, uint16_t* scales,
+                                         uint32_t* d_err, cudaStream_t stream, int grid) {
+    auto kern = quantize_pack_group_kernel<G>;
+    const size_t smem = quantize_ring_bytes(G);
+    static std::atomic<int> smem_set{0};
+    if ((int)smem > 48 * 1024 && (int)smem > smem_set.load()) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        smem_set.store((int)smem);
+    }
+    kern<<<grid, 256, smem, stream>>>(W, num_groups, codes, scales, d_err);
+    return cudaGetLastError();
 }
 
 // Any G: one thread per group, multi-word exact scale.
@@ -362,12 +413,9 @@ cudaError_t launch_quantize_pack(const uint16_t* W, int64_t N, int64_t K, int G,
         return cudaGetLastError();                                                               \
     }
 #define TQ_QG_CASE(GG)                                                                              \
-    case GG: {                                                                                      \
-        const int64_t threads = (num_groups + 31) / 32 * 32;                                        \
-        quantize_pack_group_kernel<GG><<<grid_for(threads, block, sm_count), block, 0, stream>>>(   \
-            W, num_groups, codes, scales, d_err);                                                   \
-        return cudaGetLastError();                                                                  \
-    }
+    case GG:                                                                                        \
+        return launch_quantize_group<GG>(W, num_groups, codes, scales, d_err, stream,              \
+                                         grid_for((num_groups + 31) / 32 * 32, block, sm_count));
     switch (G) {
         TQ_QG_CASE(8)
         TQ_QG_CASE(16)
