@@ -33,7 +33,10 @@ using namespace tc;
 
 constexpr int WM = 128;  // W rows per CTA (UMMA M)
 constexpr int BK = 64;
-constexpr int STAGES = 6;
+// Pipeline depth: 4 stages for 16-token tiles (97 KB of shared memory, two
+// CTAs per SM), 6 otherwise.
+template <int NT>
+constexpr int kStages = NT == 16 ? 4 : 6;
 constexpr int kThreads = 256;
 constexpr int kDecodeWarp0 = 4, kDecodeWarps = 4;
 constexpr uint32_t W_STAGE = WM * BK * 2;  // 16 KB
@@ -43,6 +46,7 @@ constexpr int kMaxCS = 8;
 
 template <int NT>
 struct Smem {
+    static constexpr int STAGES = kStages<NT>;
     uint8_t w[STAGES][W_STAGE];   // decoded W tiles (UMMA A), 1024-byte aligned
     uint8_t x[STAGES][NT * 128];  // X tiles (UMMA B): NT rows of 128 bytes
     uint8_t c[STAGES][C_STAGE];   // code-byte windows
@@ -67,9 +71,10 @@ struct Params {
 };
 
 template <int NT, bool CODES_TMA>
-__global__ void __launch_bounds__(kThreads, 1) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
+__global__ void __launch_bounds__(kThreads, NT == 16 ? 2 : 1) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                  const __grid_constant__ CUtensorMap tmap_c,
                                                                  const Params p) {
+    constexpr int STAGES = kStages<NT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem<NT>& sm = *reinterpret_cast<Smem<NT>*>(smem_raw + ((1024 - (s32(smem_raw) & 1023)) & 1023));
     cg::cluster_group cluster = cg::this_cluster();
@@ -337,7 +342,8 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     if (tiles * kMaxCS > 0x7FFFFFFF) return cudaSuccess;
     // split K so the grid covers the SMs, keeping at least two stages per CTA
     int CS = 1;
-    while (CS < kMaxCS && tiles * CS * 2 <= sm_count && nk / (CS * 2) >= 2) CS *= 2;
+    const int64_t slots = (M <= 16 ? 2 : 1) * (int64_t)sm_count;  // resident CTAs (16-token tiles: two per SM)
+    while (CS < kMaxCS && tiles * CS * 2 <= slots && nk / (CS * 2) >= 2) CS *= 2;
     if (CS == 1)  // no K split: the persistent kernel walks the tiles
         return launch_gemm_stream(X, M, codes, scales, N, K, G, Y, y_bf16, d_err, stream, sm_count, handled);
     Params p{};
