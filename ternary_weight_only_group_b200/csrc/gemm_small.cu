@@ -33,10 +33,10 @@ using namespace tc;
 
 constexpr int WM = 128;  // W rows per CTA (UMMA M)
 constexpr int BK = 64;
-// Pipeline depth: 4 stages for 16-token tiles (97 KB of shared memory, two
-// CTAs per SM), 6 otherwise.
+// Pipeline depth: 4 stages for 16-token tiles (97 KB of shared memory) and 3
+// for 32-token tiles (89 KB), so two CTAs fit per SM; 6 for 64-token tiles.
 template <int NT>
-constexpr int kStages = NT == 16 ? 4 : 6;
+constexpr int kStages = NT == 16 ? 4 : (NT == 32 ? 3 : 6);
 constexpr int kThreads = 256;
 constexpr int kDecodeWarp0 = 4, kDecodeWarps = 4;
 constexpr uint32_t W_STAGE = WM * BK * 2;  // 16 KB
@@ -71,7 +71,7 @@ struct Params {
 };
 
 template <int NT, bool CODES_TMA>
-__global__ void __launch_bounds__(kThreads, NT == 16 ? 2 : 1) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
+__global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                  const __grid_constant__ CUtensorMap tmap_c,
                                                                  const Params p) {
     constexpr int STAGES = kStages<NT>;
@@ -342,7 +342,7 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     if (tiles * kMaxCS > 0x7FFFFFFF) return cudaSuccess;
     // split K so the grid covers the SMs, keeping at least two stages per CTA
     int CS = 1;
-    const int64_t slots = (M <= 16 ? 2 : 1) * (int64_t)sm_count;  // resident CTAs (16-token tiles: two per SM)
+    const int64_t slots = (M <= 32 ? 2 : 1) * (int64_t)sm_count;  // resident CTAs (16/32-token tiles: two per SM)
     while (CS < kMaxCS && tiles * CS * 2 <= slots && nk / (CS * 2) >= 2) CS *= 2;
     if (CS == 1)  // no K split: the persistent kernel walks the tiles
         return launch_gemm_stream(X, M, codes, scales, N, K, G, Y, y_bf16, d_err, stream, sm_count, handled);
