@@ -185,7 +185,8 @@ tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* sc
     if (K == 0) return TQ_ERR_UNSUPPORTED;
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
-    // M == 1, small matrix: weights decoded before the activations are awaited
+    // 1..8 tokens, matrix small enough for one or two CTAs per SM to hold its
+    // decoded rows: weights decoded before the activations are awaited
     cudaError_t e = launch_gemv_predecode(static_cast<const uint16_t*>(X), M, codes,
                                           static_cast<const uint16_t*>(scales), N, K, G, Y, yt == TQ_OUT_BF16,
                                           d_err, (cudaStream_t)stream, d->sm_count);
