@@ -46,7 +46,7 @@ struct Smem {
     uint8_t w[STAGES][W_STAGE];     // decoded W stages (UMMA A), 1024-byte aligned
     uint8_t x[STAGES][NT * 128];    // X stages (UMMA B): NT rows of 128 bytes
     uint8_t win[2][CR][WM * WIN];   // code windows + scales, per decoder group
-    uint32_t lut[256];                // byte -> PRMT selectors of its digits 0..3
+    uint32_t lut[256 * 32];           // byte -> PRMT selectors of its digits 0..3, one copy per lane
     uint64_t full_x[STAGES], full_w[STAGES], empty[STAGES];
     uint64_t tfull[2], tempty[2], done;
     uint32_t tmem_base;
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     // preceding kernel (codes and scales are weights, see tq_gemv's ordering
     // rule); every Y store follows MMAs that consumed X.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
+    fill_digit_selector_lut4_lanes(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(&sm.full_x[st], 1);
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
 #pragma unroll
             for (int b = 0; b < 14; ++b) bytes[b] = cb[b];
             const int ql = p.B - 1 - q_lo;  // the group's last byte, relative to cb
-            decode_stage64(sm.lut, bytes, c0 - 5 * q_lo, ql < 14, ql < 14 ? cb[ql] : 0u, p.pad_base, p.pad_span,
+            decode_stage64<32>(sm.lut + (t & 31), bytes, c0 - 5 * q_lo, ql < 14, ql < 14 ? cb[ql] : 0u, p.pad_base, p.pad_span,
                            sc, sm.w[st] + t * 128, t & 7);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();

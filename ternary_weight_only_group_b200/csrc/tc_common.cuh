@@ -166,6 +166,7 @@ __device__ __forceinline__ void window_bytes(const uint8_t* row32, int off, uint
 // bytes is packed into words by PRMT and funnel-shifted by r0 bytes, so every
 // stage takes the same code.  A rejected scale or padding digit makes the
 // row's stage NaN.  Writes the 128-byte swizzled K-major tile row.
+template <int LUT_STRIDE = 1>
 __device__ __forceinline__ void decode_stage64(const uint32_t* lut4, const uint32_t (&bytes)[14], int r0,
                                                bool check_pad, uint32_t lastb, uint32_t pad_base,
                                                uint32_t pad_span, uint32_t scale_bits, uint8_t* tile_row,
@@ -174,7 +175,7 @@ __device__ __forceinline__ void decode_stage64(const uint32_t* lut4, const uint3
 #pragma unroll
     for (int i = 0; i < 14; ++i) {
         const uint32_t b = bytes[i] & 0xFFu;
-        e[i].x = lut4[b];                            // selectors of digits 0..3
+        e[i].x = lut4[b * LUT_STRIDE];               // selectors of digits 0..3
         e[i].y = 0x10u + 0x22u * ((b * 810u) >> 16);  // digit 4 = floor(b / 81), 3 for b >= 243
     }
     uint32_t W[17];

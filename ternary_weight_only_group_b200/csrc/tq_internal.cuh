@@ -169,14 +169,30 @@ __device__ __forceinline__ void eight_selectors(const uint2* sel_lut, uint32_t b
 
 // Fills a byte -> selector-bytes table (digit i in byte i) for the {-s, 0, +s, NaN} layout.
 // Selectors of digits 0..3 of every byte (bytes >= 243: all NaN).
+__device__ __forceinline__ uint32_t digit_selector_word4(uint32_t b) {
+    uint32_t w = 0, v = b;
+    for (int i = 0; i < 4; ++i) {
+        w |= digit_selector(b >= 243 ? 3u : v % 3u) << (8 * i);
+        v /= 3u;
+    }
+    return w;
+}
+
 __device__ __forceinline__ void fill_digit_selector_lut4(uint32_t* lut4, int tid, int nthreads) {
-    for (int b = tid; b < 256; b += nthreads) {
-        uint32_t w = 0, v = (uint32_t)b;
-        for (int i = 0; i < 4; ++i) {
-            w |= digit_selector(b >= 243 ? 3u : v % 3u) << (8 * i);
-            v /= 3u;
-        }
-        lut4[b] = w;
+    for (int b = tid; b < 256; b += nthreads) lut4[b] = digit_selector_word4((uint32_t)b);
+}
+
+// The same table held once per lane: word b * 32 + lane (bank `lane`), so
+// the 32 lookups of a warp never conflict, whatever the bytes.  32 KB.  Every
+// thread of the block calls it (whole warps; blockDim a multiple of 32): warp
+// w computes the words of bytes 32w .. 32w+31, one per lane, and stores each
+// byte's 32 copies with one conflict-free store.
+__device__ __forceinline__ void fill_digit_selector_lut4_lanes(uint32_t* lut, int tid, int nthreads) {
+    const int ln = tid & 31;
+    for (int b0 = (tid >> 5) * 32; b0 < 256; b0 += (nthreads >> 5) * 32) {
+        const uint32_t mine = digit_selector_word4((uint32_t)(b0 + ln));
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) lut[(b0 + j) * 32 + ln] = __shfl_sync(0xFFFFFFFFu, mine, j);
     }
 }
 

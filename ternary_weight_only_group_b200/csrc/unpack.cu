@@ -101,8 +101,14 @@ __global__ void __launch_bounds__(256) unpack_pow2_kernel(
 // The lane's weights span four code bytes; their 20 selectors are packed into
 // five words by PRMT and funnel-shifted to the lane's first weight, so the
 // fixed per-lane work (loads, validation, scale) covers twice the weights.
+// The selector table is held once per lane (word b * 32 + lane lies in bank
+// `lane`), so a warp's 32 lookups of random bytes take one shared-memory
+// wavefront instead of the 3-4 that bank conflicts on a single copy cost.
+// 32 KB per CTA; the grid is persistent (six CTAs per SM at 40 registers).
+constexpr int kUnpackThreads = 256, kUnpackCtasPerSm = 6;
+
 template <int G>
-__global__ void __launch_bounds__(256) unpack16_kernel(
+__global__ void __launch_bounds__(kUnpackThreads, kUnpackCtasPerSm) unpack16_kernel(
     const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales, int64_t num_groups,
     uint16_t* __restrict__ out, uint32_t* __restrict__ d_err) {
     constexpr int LPG = G / 16;
@@ -111,8 +117,9 @@ __global__ void __launch_bounds__(256) unpack16_kernel(
     constexpr int REAL = G - 5 * (B - 1);
     constexpr uint32_t PAD_SPAN = REAL == 1 ? 3u : (REAL == 2 ? 9u : (REAL == 3 ? 27u : 81u));
     constexpr uint32_t PAD_BASE = REAL == 1 ? 120u : (REAL == 2 ? 117u : (REAL == 3 ? 108u : 81u));
-    __shared__ uint32_t lut4[256];  // selectors of digits 0..3; digit 4 = floor(b / 81) by arithmetic
-    fill_digit_selector_lut4(lut4, threadIdx.x, blockDim.x);
+    // selectors of digits 0..3, one copy per lane; digit 4 = floor(b / 81) by arithmetic
+    __shared__ uint32_t lut[256 * 32];
+    fill_digit_selector_lut4_lanes(lut, threadIdx.x, blockDim.x);
     __syncthreads();
 
     const int lane = threadIdx.x & 31;
@@ -154,7 +161,7 @@ __global__ void __launch_bounds__(256) unpack16_kernel(
         bad = seg_or_u32(bad, LPG);
         if (!active) bad = 0;
         // selector stream of the four bytes (5 per byte), then the lane's 16
-        auto rec = [&](uint32_t b) { return make_uint2(lut4[b], 0x10u + 0x22u * ((b * 810u) >> 16)); };
+        auto rec = [&](uint32_t b) { return make_uint2(lut[b * 32 + lane], 0x10u + 0x22u * ((b * 810u) >> 16)); };
         const uint2 e0 = rec(bv[0]), e1 = rec(bv[1]), e2 = rec(bv[2]), e3 = rec(bv[3]);
         const uint32_t W[5] = {e0.x, prmt32(e0.y, e1.x, 0x6540u), prmt32(prmt32(e1.x, e1.y, 0x0043u), e2.x, 0x5410u),
                                prmt32(prmt32(e2.x, e2.y, 0x0432u), e3.x, 0x4210u), prmt32(e3.x, e3.y, 0x4321u)};
@@ -229,8 +236,10 @@ cudaError_t launch_unpack(const uint8_t* codes, const uint16_t* scales, int64_t 
 #define TQ_UP_CASE(GG)                                                                          \
     case GG: {                                                                                  \
         const int64_t threads = (num_groups + (32 / (GG / 16)) - 1) / (32 / (GG / 16)) * 32;    \
-        unpack16_kernel<GG><<<grid(threads, 256), 256, 0, stream>>>(codes, scales, num_groups,  \
-                                                                   out, d_err);                 \
+        const int64_t blocks = (threads + kUnpackThreads - 1) / kUnpackThreads;                 \
+        const int64_t cap = (int64_t)sm_count * kUnpackCtasPerSm;                               \
+        unpack16_kernel<GG><<<(int)(blocks < cap ? blocks : cap), kUnpackThreads, 0, stream>>>( \
+            codes, scales, num_groups, out, d_err);                                             \
         return cudaGetLastError();                                                              \
     }
     switch (G) {
