@@ -74,6 +74,12 @@ def _load():
             lib.oracle_quantize_pack.restype = ctypes.c_uint32
             lib.oracle_unpack_bf16.argtypes = [u8p, u16p, i64, i64, i64, u16p]
             lib.oracle_unpack_bf16.restype = ctypes.c_uint32
+            lib.oracle_bytes_per_group2.argtypes = [i64]
+            lib.oracle_bytes_per_group2.restype = i64
+            lib.oracle_quantize_pack2.argtypes = [u16p, i64, i64, i64, u8p, u16p]
+            lib.oracle_quantize_pack2.restype = ctypes.c_uint32
+            lib.oracle_unpack2_bf16.argtypes = [u8p, u16p, i64, i64, i64, u16p]
+            lib.oracle_unpack2_bf16.restype = ctypes.c_uint32
             lib.oracle_matmul.argtypes = [u16p, i64, i64p, i64, u16p, i64, i64, f64p]
             lib.oracle_matmul.restype = None
             lib.oracle_matmul_points.argtypes = [u16p, u16p, i64, i64p, i64p, i64, f64p]
@@ -160,6 +166,39 @@ def unpack_bf16(codes: np.ndarray, scales: np.ndarray, N: int, K: int, G: int):
     return out, int(err)
 
 
+# ---------------------------------------------------------------- 2-bit codec
+
+def bytes_per_group2(G: int) -> int:
+    """ceil(G/4): four 2-bit codes per byte, each group byte-aligned."""
+    return int(_load().oracle_bytes_per_group2(int(G)))
+
+
+def quantize_pack2(W_bits: np.ndarray, G: int):
+    """[N, K] bf16 bit patterns -> (codes u8 [N, K/G, ceil(G/4)], scales u16 [N, K/G], err),
+    2-bit format (code t + 1, first weight in the low bits)."""
+    W = _u16(W_bits)
+    N, K = W.shape
+    _check_shape(N, K, G)
+    ng, B = K // G, bytes_per_group2(G)
+    codes = np.zeros((N, ng, B), dtype=np.uint8)
+    scales = np.zeros((N, ng), dtype=np.uint16)
+    err = _load().oracle_quantize_pack2(_ptr(W, ctypes.c_uint16), N, K, G,
+                                        _ptr(codes, ctypes.c_uint8), _ptr(scales, ctypes.c_uint16))
+    return codes, scales, int(err)
+
+
+def unpack2_bf16(codes: np.ndarray, scales: np.ndarray, N: int, K: int, G: int):
+    """2-bit codes + scales -> (decoded bf16 bit patterns [N, K], err)."""
+    _check_shape(N, K, G)
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    s = _u16(scales)
+    assert c.size == N * (K // G) * bytes_per_group2(G) and s.size == N * (K // G)
+    out = np.zeros((N, K), dtype=np.uint16)
+    err = _load().oracle_unpack2_bf16(_ptr(c, ctypes.c_uint8), _ptr(s, ctypes.c_uint16), N, K, G,
+                                      _ptr(out, ctypes.c_uint16))
+    return out, int(err)
+
+
 # ---------------------------------------------------------------- matmul
 
 def matmul(X_bits: np.ndarray, What_bits: np.ndarray, rows=None) -> np.ndarray:
@@ -211,3 +250,9 @@ def round_bf16_array(Y: np.ndarray) -> np.ndarray:
     f = _load().oracle_bf16_round
     flat = np.asarray(Y, dtype=np.float64).ravel()
     return np.array([f(float(v)) for v in flat], dtype=np.uint16).reshape(np.shape(Y))
+
+
+def linear2(X_bits, codes, scales, N: int, K: int, G: int, rows=None) -> np.ndarray:
+    """The fused layer on the 2-bit format: Y = X . unpack2(codes, scales)^T (binary64)."""
+    Wd, _ = unpack2_bf16(codes, scales, N, K, G)
+    return matmul(X_bits, Wd, rows)

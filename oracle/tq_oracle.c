@@ -18,6 +18,9 @@
  *            a zero stored scale produces a zero group, columns divisible by G.
  *   [rate]   precisit/pack-unpack-run, payload-rate paragraph:
  *            8*(ceil(G/5)+2)/G bits per weight.
+ *   [two]    "Autoregressive Language Model on the 6502 Processor", summary:
+ *            BitNet ternary weights (-1, 0, 1) packed four parameters per
+ *            byte (the 2-bit alternative to the base-3 codec).
  *   [mm]     tiny-llm "Week 2 Day 3: Quantize the Model", "Mathematical
  *            Formulation" and "Computation Flow": C[i,k] = sum_j A[i,j]*B[k,j]
  *            with B reconstructed per group of G input columns, accumulated in
@@ -39,6 +42,11 @@
  *     bf16 NaN so that any product with it is NaN;
  *   - matmul reference: fp64 sum of exact products of bf16 activations and
  *     decoded bf16 weights.
+ *   - 2-bit format [two]: the same groups, scales and trits as the base-3
+ *     codec; code c = t + 1 in two bits, four per byte, the first weight in
+ *     the least-significant bits; ceil(G/4) bytes per group, byte-aligned,
+ *     padding codes 1 (zero trit); code 3 is invalid (error bit 1, like a
+ *     byte >= 243), a padding code other than 1 sets error bit 2.
  *
  * Error bits returned (same meaning as the library's asynchronous flags):
  *   1  a code byte >= 243          2  non-canonical padding digit
@@ -397,4 +405,97 @@ void oracle_matmul_points(const uint16_t *X, const uint16_t *What, int64_t K,
             acc += v[x[k]] * v[w[k]];
         Y[i] = acc;
     }
+}
+
+/* ------------------------------------------------------------------ */
+/* [two] The 2-bit ternary format: four codes per byte.                */
+/* ------------------------------------------------------------------ */
+
+/* [two] bytes per group: ceil(G/4) */
+int64_t oracle_bytes_per_group2(int64_t G)
+{
+    return (G + 3) / 4;
+}
+
+/*
+ * Quantize and pack into the 2-bit format.  Scale and trits are those of
+ * oracle_group_scale and oracle_trit ([codec], [rules]); weight j of a
+ * group is code (t + 1) at bits 2 (j % 4) of byte j / 4 ([two]).
+ * codes: [N][K/G][ceil(G/4)] bytes, scales: [N][K/G] binary16.
+ */
+uint32_t oracle_quantize_pack2(const uint16_t *W, int64_t N, int64_t K, int64_t G,
+                               uint8_t *codes, uint16_t *scales)
+{
+    uint32_t err = 0;
+    int64_t ng = K / G, B = oracle_bytes_per_group2(G);
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t g = 0; g < ng; g++) {
+            const uint16_t *w = W + n * K + g * G;
+            uint16_t s;
+            uint32_t e = oracle_group_scale(w, G, &s);
+            err |= e;
+            scales[n * ng + g] = s;
+            uint8_t *out = codes + (n * ng + g) * B;
+            for (int64_t q = 0; q < B; q++) {
+                int byte = 0;
+                for (int i = 0; i < 4; i++) {
+                    int64_t j = 4 * q + i;
+                    int t = (j < G && e == 0) ? oracle_trit(w[j], s) : 0; /* pad = zero trit */
+                    byte |= (t + 1) << (2 * i);                            /* code c = t + 1 */
+                }
+                out[q] = (uint8_t)byte;
+            }
+        }
+    }
+    return err;
+}
+
+/*
+ * [two] decoding: code 3 is invalid; padding codes must be 1; decoded
+ * weights as for the base-3 codec (+0 for a zero trit or zero scale, else
+ * sign(t) * RNE_bf16(scale); a rejected group decodes to NaN).
+ */
+uint32_t oracle_unpack2_bf16(const uint8_t *codes, const uint16_t *scales, int64_t N,
+                             int64_t K, int64_t G, uint16_t *W_out)
+{
+    uint32_t err = 0;
+    int64_t ng = K / G, B = oracle_bytes_per_group2(G);
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t g = 0; g < ng; g++) {
+            uint16_t s = scales[n * ng + g];
+            const uint8_t *in = codes + (n * ng + g) * B;
+            uint16_t *w = W_out + n * K + g * G;
+            uint32_t e = 0;
+            if ((s & 0x8000) || ((s >> 10) & 0x1F) == 0x1F)
+                e |= ERR_SCALE;                     /* negative, NaN or Inf scale */
+            for (int64_t q = 0; q < B; q++) {
+                for (int i = 0; i < 4; i++) {
+                    int c = (in[q] >> (2 * i)) & 3;
+                    int64_t j = 4 * q + i;
+                    if (c == 3) {
+                        e |= ERR_BYTE;
+                        continue;
+                    }
+                    if (j >= G) {
+                        if (c != 1)
+                            e |= ERR_PADDING;
+                        continue;
+                    }
+                    int t = c - 1;
+                    if (t == 0 || s == 0)
+                        w[j] = 0x0000;
+                    else {
+                        uint16_t mag = oracle_bf16_round(oracle_fp16_value(s));
+                        w[j] = (uint16_t)(mag | (t < 0 ? 0x8000 : 0));
+                    }
+                }
+            }
+            if (e) {
+                for (int64_t j = 0; j < G; j++)
+                    w[j] = 0x7FC0;                  /* rejected group: NaN */
+            }
+            err |= e;
+        }
+    }
+    return err;
 }

@@ -150,30 +150,45 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
     const bool vec_out = (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
     uint32_t err_acc = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    // G <= 64: the warp's next 32 groups are copied into a double-buffered
-    // shared-memory ring by coalesced cp.async while the current 32 are
-    // quantized (the loads cost no registers, which the group occupies).
-    // Rows are padded to 2G + 16 bytes so that the 16-byte reads of the
-    // lanes' own groups are free of bank conflicts.
-    constexpr int RS = 2 * G + 16;
-    extern __shared__ __align__(16) uint8_t qring[];  // [2][8 warps][32 groups][RS]
-    auto issue = [&](int64_t gb, int buf) {
-        if constexpr (G <= 64) {
-            uint8_t* base = qring + ((size_t)buf * 8 + wib) * 32 * RS;
+    // The warp's next 32 groups (G <= 64) or next half-groups of 64 weights
+    // (G = 128) are copied into a double-buffered shared-memory ring by
+    // coalesced cp.async while the current ones are quantized (the loads cost
+    // no registers, which the group occupies).  Ring rows are padded to
+    // 16 bytes past the data so that the 16-byte reads of the lanes' own rows
+    // are free of bank conflicts.
+    constexpr int RS = (G <= 64 ? 2 * G : 128) + 16;
+    extern __shared__ __align__(16) uint8_t qring[];  // [2][8 warps][32 rows][RS]
+    auto issue = [&](int64_t gb, int half, int buf) {
+        constexpr int PIECES = (G <= 64 ? G : 64) / 8;  // 16-byte pieces of a ring row
+        uint8_t* base = qring + ((size_t)buf * 8 + wib) * 32 * RS;
 #pragma unroll
-            for (int k = 0; k < G / 8; ++k) {
-                const int c = lane + 32 * k, grp = c / (G / 8), piece = c - grp * (G / 8);
-                if (gb + grp < num_groups)
-                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                                     (uint32_t)__cvta_generic_to_shared(base + grp * RS + piece * 16)),
-                                 "l"(__cvta_generic_to_global(W + (gb + grp) * G + piece * 8))
-                                 : "memory");
-            }
-            asm volatile("cp.async.commit_group;" ::: "memory");
+        for (int k = 0; k < PIECES; ++k) {
+            const int c = lane + 32 * k, grp = c / PIECES, piece = c - grp * PIECES;
+            if (gb + grp < num_groups)
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                                 (uint32_t)__cvta_generic_to_shared(base + grp * RS + piece * 16)),
+                             "l"(__cvta_generic_to_global(W + (gb + grp) * G + half * 64 + piece * 8))
+                             : "memory");
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // Waits for the oldest copy group in flight and reads this lane's ring row.
+    auto take = [&](int buf, uint32_t* h) {
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        __syncwarp();
+        const uint4* row = reinterpret_cast<const uint4*>(qring + (((size_t)buf * 8 + wib) * 32 + lane) * RS);
+#pragma unroll
+        for (int k = 0; k < (RS - 16) / 16; ++k) {
+            const uint4 v = row[k];
+            h[4 * k] = v.x;
+            h[4 * k + 1] = v.y;
+            h[4 * k + 2] = v.z;
+            h[4 * k + 3] = v.w;
+        }
+        __syncwarp();  // every lane has read this buffer before it is refilled
     };
     const int64_t g_first = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-    if (g_first < num_groups) issue(g_first, 0);
+    if (g_first < num_groups) issue(g_first, 0, 0);
     int pass = 0;
     for (int64_t g0 = g_first; g0 < num_groups; g0 += stride, ++pass) {
         const int64_t gi = g0 + lane;  // the warp's groups g0 .. g0+31
@@ -183,22 +198,8 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
         uint32_t cw[NCW];
         if constexpr (G <= 64) {
             uint32_t h[NWD];
-            {
-                issue(g0 + stride, (pass + 1) & 1);  // that buffer was read last pass
-                asm volatile("cp.async.wait_group 1;" ::: "memory");
-                __syncwarp();
-                const uint4* row =
-                    reinterpret_cast<const uint4*>(qring + (((size_t)(pass & 1) * 8 + wib) * 32 + lane) * RS);
-#pragma unroll
-                for (int k = 0; k < G / 8; ++k) {
-                    const uint4 v = row[k];
-                    h[4 * k] = v.x;
-                    h[4 * k + 1] = v.y;
-                    h[4 * k + 2] = v.z;
-                    h[4 * k + 3] = v.w;
-                }
-                __syncwarp();  // every lane has read this buffer before it is refilled
-            }
+            issue(g0 + stride, 0, (pass + 1) & 1);  // that buffer was read last pass
+            take(pass & 1, h);
             uint32_t amax = 0;
 #pragma unroll
             for (int j = 0; j < G; ++j) amax = max(amax, (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu);
@@ -250,20 +251,16 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
             // magnitude; the sum is exact when all of them lie within 2^37 of the
             // maximum (the same window as above), else the group takes the exact
             // multi-word path.  Pass 2 re-reads the halves (cache hits) to encode.
-            const uint4* src = reinterpret_cast<const uint4*>(W + (active ? gi : 0) * G);
+            // Ring steps: half 0 and 1 of pass 1 in buffers 0 and 1, then of
+            // pass 2; each step issues the next (the last one the next 32
+            // groups' first half).
             uint32_t amax = 0, amin1 = 0xFFFFFFFFu;  // amin1 = smallest nonzero magnitude - 1
             double sum = 0.0;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t h[32];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint4 v = __ldg(src + 8 * half + k);
-                    h[4 * k] = v.x;
-                    h[4 * k + 1] = v.y;
-                    h[4 * k + 2] = v.z;
-                    h[4 * k + 3] = v.w;
-                }
+                issue(g0, 1 - half, 1 - half);
+                take(half, h);
 #pragma unroll
                 for (int j = 0; j < 64; ++j) {
                     const uint32_t a = (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
@@ -271,7 +268,6 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
                     amin1 = min(amin1, a - 1u);  // a = 0 wraps to the largest value
                     if (a) sum += bf16_normal_mag_to_f64(a);
                 }
-                asm volatile("" ::: "memory");  // keep the halves' loads apart
             }
             const uint32_t emax = amax >> 7;
             const uint32_t thr = emax > 37 ? (emax - 37) << 7 : 0;
@@ -294,14 +290,8 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t h[32];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint4 v = __ldg(src + 8 * half + k);
-                    h[4 * k] = v.x;
-                    h[4 * k + 1] = v.y;
-                    h[4 * k + 2] = v.z;
-                    h[4 * k + 3] = v.w;
-                }
+                issue(half == 0 ? g0 : g0 + stride, 1 - half, 1 - half);
+                take(half, h);
 #pragma unroll
                 for (int jj = 0; jj < 64; ++jj) {
                     const int j = 64 * half + jj, q = j / 5;
@@ -311,7 +301,6 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
                     const uint32_t d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
                     cw[q / 4] += d * pw;
                 }
-                asm volatile("" ::: "memory");
             }
 #pragma unroll
             for (int j = G; j < 5 * B; ++j)  // padding digits 1
@@ -337,12 +326,12 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
         }
         __syncwarp();
     }
-    if constexpr (G <= 64) asm volatile("cp.async.wait_all;" ::: "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
 // Dynamic shared memory of quantize_pack_group_kernel<G>: the load ring.
-static size_t quantize_ring_bytes(int G) { return G <= 64 ? (size_t)2 * 8 * 32 * (2 * G + 16) : 0; }
+static size_t quantize_ring_bytes(int G) { return (size_t)2 * 8 * 32 * ((G <= 64 ? 2 * G : 128) + 16); }
 
 template <int G>
 static cudaError_t launch_quantize_group(const uint16_t* W, int64_t num_groups, uint8_t* codes, uint16_t* scales,
