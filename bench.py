@@ -65,6 +65,11 @@ def packed_bytes(N, K, G):
     return N * (K // G) * ((G + 4) // 5) + N * (K // G) * 2
 
 
+def packed2_bytes(N, K, G):
+    """Codes + scales of the 2-bit format (four codes per byte)."""
+    return N * (K // G) * ((G + 3) // 4) + N * (K // G) * 2
+
+
 # --------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -229,7 +234,7 @@ def device_acts(M, K, seed):
 
 # --------------------------------------------------------------------- our arm
 
-def build_decode_stack(tq, layers):
+def build_decode_stack(tq, layers, pack="base3"):
     """Packed weights of `layers` x (gate, up, down) for each G, plus one X
     buffer and one Y buffer sliced per launch (so a whole step's inputs and
     outputs are single contiguous transfers for the end-to-end measurement)."""
@@ -243,7 +248,7 @@ def build_decode_stack(tq, layers):
                 x_elems += K
                 y_elems += N
     packs = {}
-    for G in GROUPS:
+    for G in GROUPS if pack else ():
         for l in range(layers):
             for i, (name, (N, K)) in enumerate(FFN.items()):
                 W = device_weights(N, K, seed=1000 + 3 * l + i)
@@ -305,6 +310,7 @@ def run_ours(args, rank, world, local):
         results["pack"], results["unpack"] = bench_bulk_codec(tq, args, world, peaks)
         results["prefill"] = bench_prefill(tq, args, world, peaks)
         results["msweep"] = bench_msweep(tq, args, world, peaks)
+        results["ternary2"] = bench_ternary2(tq, args, world, peaks)
     clk = clocks.summary()
 
     ms_step = ms / K_steps
@@ -352,16 +358,23 @@ def run_ours(args, rank, world, local):
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2},
-        "gpu_launches": launches_per_step * K_steps * 2 + sum(
-            r.get("launches", 0) for r in results.values() if isinstance(r, dict)),
+        "gpu_launches": launches_per_step * K_steps * 2 + count_launches(results),
         "clocks": clk,
         "gemv_stream": results["stream"],
         "pack": results["pack"],
         "unpack": results["unpack"],
         "prefill_gemm": results["prefill"],
         "msweep": results["msweep"],
+        "ternary2": results["ternary2"],
     }
     print(json.dumps(line), flush=True)
+
+
+def count_launches(obj) -> int:
+    """Sum of every "launches" entry in a (nested) result dict."""
+    if isinstance(obj, dict):
+        return sum(v if k == "launches" and isinstance(v, int) else count_launches(v) for k, v in obj.items())
+    return 0
 
 
 def bench_gemv_stream(tq, args, world, peaks):
@@ -509,6 +522,99 @@ def bench_bulk_codec(tq, args, world, peaks):
     return out_pack, out_unpack
 
 
+def bench_ternary2(tq, args, world, peaks):
+    """The 2-bit format (four codes per byte) through its own kernels:
+    quantize + pack and unpack over the 72-matrix FFN stack, the streaming
+    GEMV over the [172032 x 1024] gate/up stack (four copies, 187 MB > L2)
+    and the decode chain of the headline (288 tq2_gemv launches, one graph)."""
+    import torch
+    res = {"pack": {}, "unpack": {}}
+    shapes = [(48 * 3584, 1024), (24 * 1024, 3584)]
+    reps = max(3, args.steps // 4)
+    for G in GROUPS:
+        mats = [device_weights(N, K, seed=500 + i, outliers=False) for i, (N, K) in enumerate(shapes)]
+        packed = [tq.quantize_pack2(W, G) for W in mats]
+        outs = [torch.empty_like(W) for W in mats]
+
+        def do_pack():
+            st = torch.cuda.current_stream().cuda_stream
+            for W, (c, s) in zip(mats, packed):
+                rc = tq.lib().tq2_quantize_pack(W.data_ptr(), W.shape[0], W.shape[1], G,
+                                                c.data_ptr(), s.data_ptr(), None, st)
+                if rc != tq.TQ_OK:
+                    raise tq.TQError(rc, "tq2_quantize_pack")
+
+        def do_unpack():
+            for (c, s), o in zip(packed, outs):
+                tq.unpack2_bf16(c, s, o.shape[0], o.shape[1], G, out=o)
+
+        ms_p = timed(do_pack, reps, max(3, args.warmup), world)
+        ms_u = timed(do_unpack, reps, max(3, args.warmup), world)
+        wbytes = sum(2 * N * K for N, K in shapes)
+        pbytes = sum(packed2_bytes(N, K, G) for N, K in shapes)
+        for d, ms in ((res["pack"], ms_p), (res["unpack"], ms_u)):
+            sec = ms * 1e-3 / reps
+            d[f"G{G}"] = {"us": round(sec * 1e6, 1), "total_GB/s": round((wbytes + pbytes) / sec / 1e9, 1),
+                          "frac": round((wbytes + pbytes) / sec / 1e9 / peaks["hbm_gbs"], 4),
+                          "launches": 2 * reps}
+        del mats, packed, outs
+        torch.cuda.empty_cache()
+
+    N, K, G = 48 * 3584, 1024, 128
+    packs = []
+    for c in range(4):
+        W = device_weights(N, K, seed=77 + c)
+        packs.append(tq.quantize_pack2(W, G))
+        del W
+    X = device_acts(1, K, seed=78)
+    Y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+    sreps = 4 * max(2, args.steps // 4)
+    state = {"i": 0}
+
+    def one():
+        c, s = packs[state["i"] % 4]
+        state["i"] += 1
+        tq.gemv2(X, c, s, N, K, G, out=Y)
+    ms = timed(one, sreps, max(4, args.warmup), world)
+    byts = packed2_bytes(N, K, G) + 2 * K + 2 * N
+    gbs = byts * sreps / (ms * 1e-3) / 1e9
+    res["gemv_stream"] = {"shape": [N, K], "G": G, "us": round(ms * 1e3 / sreps, 2), "GB/s": round(gbs, 1),
+                          "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": sreps,
+                          "kernel": "gemv2_kernel<1, 8>"}
+    del packs
+    torch.cuda.empty_cache()
+
+    calls, _, Xs, Ys = build_decode_stack(tq, LAYERS, pack=None)
+    packs2 = {}
+    for G in GROUPS:
+        for l in range(LAYERS):
+            for i, (name, (N, K)) in enumerate(FFN.items()):
+                W = device_weights(N, K, seed=1000 + 3 * l + i)
+                packs2[(G, l, name)] = tq.quantize_pack2(W, G)
+                del W
+    step_bytes = sum(packed2_bytes(N, K, G) + 2 * K + 2 * N for (G, l, name, N, K, xo, yo) in calls)
+
+    def step():
+        for (G, l, name, N, K, xo, yo) in calls:
+            c, s = packs2[(G, l, name)]
+            tq.gemv2(Xs[xo:xo + K].view(1, K), c, s, N, K, G, out=Ys[yo:yo + N].view(1, N))
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+        step()
+    steps = max(3, args.steps // 5)
+    ms = timed(graph.replay, steps, max(3, args.warmup), world)
+    us = ms * 1e3 / steps
+    res["decode_stack"] = {"launches_per_step": len(calls), "us_per_step": round(us, 1),
+                           "us_per_launch": round(us / len(calls), 3), "GB/s": round(step_bytes / us / 1e3, 1),
+                           "frac": round(step_bytes / us / 1e3 / peaks["hbm_gbs"], 4),
+                           "launches": steps * len(calls), "bytes_per_step": step_bytes}
+    del graph, packs2
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_prefill(tq, args, world, peaks):
     import torch
     M, G = 4096, 128
@@ -621,7 +727,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
-    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv", "msweep"], default=None,
+    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv", "msweep", "ternary2"], default=None,
                     help="run one sub-benchmark alone and print its result (profiling aid)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -637,7 +743,7 @@ def main():
             torch.cuda.set_device(local)
             peaks = load_peaks()
             fn = {"stream": bench_gemv_stream, "codec": bench_bulk_codec, "prefill": bench_prefill,
-                  "gemv": bench_gemv_shapes, "msweep": bench_msweep}
+                  "gemv": bench_gemv_shapes, "msweep": bench_msweep, "ternary2": bench_ternary2}
             res = fn[args.only](tq, args, world, peaks)
             if rank == 0:
                 print(json.dumps({"only": args.only, "result": res}), flush=True)

@@ -112,8 +112,11 @@ TQ_API tq_status tq_unpack_bf16(const uint8_t *codes, const void *scales_f16, in
  * Fused unpack-and-scale matmul for decode (tiny-llm "Week 2 Day 3",
  * "Computation Flow"; the scale is applied once per group as in its "SIMD
  * Matvec" stage): Y[m][n] = sum_g RNE_bf16(s[n][g]) * sum_{j in g} t[n][j] X[m][j],
- * accumulated in fp32, written as fp32 or RNE bf16.  Any M >= 1; tuned for
- * M <= 16 (CUDA cores).  X: [M][K] bf16, 16-byte aligned; Y: [M][N]
+ * accumulated in fp32, written as fp32 or RNE bf16.  Any M >= 1: CUDA-core
+ * kernels up to 8 tokens (weights decoded on chip ahead of the activations
+ * when a matrix's rows fit, lookup tables otherwise), tensor-core small-M
+ * kernels up to 64 tokens, a row kernel beyond and for the shapes those do
+ * not cover.  X: [M][K] bf16, 16-byte aligned; Y: [M][N]
  * (fp32: 4-byte aligned, bf16: 2-byte aligned), must not overlap the inputs.
  * workspace: at least tq_workspace_bytes(M, N, K, G) bytes of device scratch
  * (NULL allowed when that is 0), 256-byte aligned.
@@ -138,6 +141,33 @@ TQ_API tq_status tq_gemv(const void *X_bf16, int64_t M, const uint8_t *codes, co
 TQ_API tq_status tq_gemm(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
                   int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,
                   size_t ws_bytes, uint32_t *d_err, tq_stream_t stream);
+
+/*
+ * The 2-bit ternary format ("Autoregressive Language Model on the 6502
+ * Processor", summary: BitNet ternary weights packed four per byte).  Same
+ * groups, binary16 scales and trits as the base-3 codec; code c = t + 1 in
+ * two bits, weight j of a group in bits 2 (j % 4) of its byte j / 4, each
+ * group ceil(G/4) bytes, padding codes 1, code 3 invalid (TQ_DERR_BYTE; a
+ * padding code other than 1 or 3 sets TQ_DERR_PADDING).  Buffers:
+ * codes [N][K/G][ceil(G/4)] (4-byte aligned), scales as for base-3.
+ */
+/* Bytes of the 2-bit codes buffer: N * (K/G) * ceil(G/4).  0 for invalid shapes. */
+TQ_API size_t tq2_codes_bytes(int64_t N, int64_t K, int G);
+/* Quantize and pack into the 2-bit format; arguments, errors and error bits as
+ * tq_quantize_pack, plus TQ_ERR_ALIGNMENT for codes not 4-byte aligned. */
+TQ_API tq_status tq2_quantize_pack(const void *W_bf16, int64_t N, int64_t K, int G, uint8_t *codes,
+                            void *scales_f16, uint32_t *d_err, tq_stream_t stream);
+/* Decode the 2-bit format to bf16; as tq_unpack_bf16 (rejected groups NaN). */
+TQ_API tq_status tq2_unpack_bf16(const uint8_t *codes, const void *scales_f16, int64_t N, int64_t K,
+                          int G, void *W_bf16_out, uint32_t *d_err, tq_stream_t stream);
+/* Fused unpack-and-scale matmul on the 2-bit format, CUDA cores, any M >= 1
+ * (eight tokens per launch); result definition, arguments, alignment and
+ * ordering as tq_gemv (X is read after the preceding work has completed,
+ * codes and scales too).  Covers G in {16, 32, 64, 128, 256} and
+ * K <= 49152; other shapes return TQ_ERR_UNSUPPORTED. */
+TQ_API tq_status tq2_gemv(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
+                   int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,
+                   size_t ws_bytes, uint32_t *d_err, tq_stream_t stream);
 
 /* Human-readable name of a status code (static string). */
 TQ_API const char *tq_status_string(tq_status s);

@@ -25,7 +25,8 @@ DERR_BYTE, DERR_PADDING, DERR_WEIGHT, DERR_SCALE, DERR_OVERFLOW, DERR_TIMEOUT = 
 MAX_G = 4096
 
 EXPORTS = ("tq_codes_bytes", "tq_scales_bytes", "tq_workspace_bytes", "tq_quantize_pack",
-           "tq_unpack_bf16", "tq_gemv", "tq_gemm", "tq_status_string", "tq_version")
+           "tq_unpack_bf16", "tq_gemv", "tq_gemm", "tq2_codes_bytes", "tq2_quantize_pack",
+           "tq2_unpack_bf16", "tq2_gemv", "tq_status_string", "tq_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -62,6 +63,14 @@ def lib() -> ctypes.CDLL:
             L.tq_gemv.restype = i32
             L.tq_gemm.argtypes = mm
             L.tq_gemm.restype = i32
+            L.tq2_codes_bytes.argtypes = [i64, i64, i32]
+            L.tq2_codes_bytes.restype = sz
+            L.tq2_quantize_pack.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
+            L.tq2_quantize_pack.restype = i32
+            L.tq2_unpack_bf16.argtypes = [vp, vp, i64, i64, i32, vp, vp, vp]
+            L.tq2_unpack_bf16.restype = i32
+            L.tq2_gemv.argtypes = mm
+            L.tq2_gemv.restype = i32
             L.tq_status_string.argtypes = [i32]
             L.tq_status_string.restype = ctypes.c_char_p
             L.tq_version.argtypes = []
@@ -92,6 +101,14 @@ def workspace_bytes(M: int, N: int, K: int, G: int) -> int:
 
 def bytes_per_group(G: int) -> int:
     return (G + 4) // 5
+
+
+def codes2_bytes(N: int, K: int, G: int) -> int:
+    return int(lib().tq2_codes_bytes(N, K, G))
+
+
+def bytes_per_group2(G: int) -> int:
+    return (G + 3) // 4
 
 
 # ----------------------------------------------------------------------------
@@ -188,3 +205,40 @@ def gemm(X, codes, scales, N: int, K: int, G: int, out_dtype=None, out=None, d_e
     torch = _torch()
     return _matmul(lib().tq_gemm, "tq_gemm", X, codes, scales, N, K, G,
                    out_dtype or torch.bfloat16, out, d_err, stream, workspace)
+
+
+# ----------------------------------------------------------------------------
+# the 2-bit ternary format (four codes per byte)
+
+def quantize_pack2(W, G: int, d_err=None, stream=None):
+    """W: [N, K] bf16 CUDA tensor -> (codes uint8 [N, K/G, ceil(G/4)], scales fp16 [N, K/G])."""
+    torch = _torch()
+    W = _as_cuda(W, torch.bfloat16, "W")
+    N, K = W.shape
+    if G < 1 or K % G:
+        raise TQError(TQ_ERR_INVALID_ARG, "quantize_pack2")
+    codes = torch.empty((N, K // G, bytes_per_group2(G)), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N, K // G), dtype=torch.float16, device=W.device)
+    _check(lib().tq2_quantize_pack(_ptr(W), N, K, G, _ptr(codes), _ptr(scales), _ptr(d_err),
+                                   _stream(stream)), "tq2_quantize_pack")
+    return codes, scales
+
+
+def unpack2_bf16(codes, scales, N: int, K: int, G: int, out=None, d_err=None, stream=None):
+    """2-bit codes + scales -> [N, K] bf16 decoded weights."""
+    torch = _torch()
+    codes = _as_cuda(codes, torch.uint8, "codes")
+    scales = _as_cuda(scales, torch.float16, "scales")
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=codes.device)
+    _check(lib().tq2_unpack_bf16(_ptr(codes), _ptr(scales), N, K, G, _ptr(out), _ptr(d_err),
+                                 _stream(stream)), "tq2_unpack_bf16")
+    return out
+
+
+def gemv2(X, codes, scales, N: int, K: int, G: int, out_dtype=None, out=None, d_err=None,
+          stream=None, workspace=None):
+    """Decode matmul on the 2-bit format (CUDA cores): Y[M, N] = X . What^T."""
+    torch = _torch()
+    return _matmul(lib().tq2_gemv, "tq2_gemv", X, codes, scales, N, K, G,
+                   out_dtype or torch.float32, out, d_err, stream, workspace)

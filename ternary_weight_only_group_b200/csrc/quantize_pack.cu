@@ -131,6 +131,17 @@ __global__ void __launch_bounds__(256) quantize_pack_pow2_kernel(
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
+// Place of weight j's code inside the group's packed words: code c of weight
+// j adds c * code_place(j) to word (j / PER) / 4, PER codes per byte.  Base-3
+// (FMT 3): digit j % 5 of byte j / 5, weight 3^(j % 5).  2-bit (FMT 2): bits
+// 2 (j % 4) of byte j / 4.
+template <int FMT>
+__host__ __device__ constexpr uint32_t code_place(int j) {
+    return (FMT == 3 ? (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
+                     : 1u << (2 * (j % 4)))
+           << (8 * ((j / (FMT == 3 ? 5 : 4)) % 4));
+}
+
 // One lane per group (G = 8, 16, 32, 64, 128): the group's weights sit in
 // the lane's registers (G = 128: one half at a time, read twice), so max and
 // sum need no shuffles; every weight's byte
@@ -138,12 +149,15 @@ __global__ void __launch_bounds__(256) quantize_pack_pow2_kernel(
 // multiply-add per weight into packed code words; each warp's 32 groups of
 // code bytes are assembled in shared memory and written with 16-byte stores
 // when the destination allows it.  The scale arithmetic is the one above.
-template <int G>
+// FMT selects the packing: 3 = base-3 (five digits per byte), 2 = the 2-bit
+// format (four codes per byte; these G are multiples of 4, no padding).
+template <int G, int FMT = 3>
 __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kernel(
     const uint16_t* __restrict__ W, int64_t num_groups, uint8_t* __restrict__ codes,
     uint16_t* __restrict__ scales, uint32_t* __restrict__ d_err) {
     constexpr int NWD = G / 2;                 // 32-bit words of a group
-    constexpr int B = bytes_per_group(G);
+    constexpr int PER = FMT == 3 ? 5 : 4;  // codes per byte
+    constexpr int B = (G + PER - 1) / PER;
     constexpr int NCW = (B + 3) / 4;           // packed code words
     __shared__ __align__(16) uint8_t stage[256 / 32][32 * B];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
@@ -226,22 +240,20 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
             }
             if (gerr) s = 0;
             const uint32_t th = trit_threshold(s);
-            // code words: byte q of the group in byte q % 4 of word q / 4; digit
-            // d = t + 1 of weight j adds d * 3^(j % 5) to byte j / 5; positions
-            // j >= G hold the padding digit 1
+            // code words: byte q of the group in byte q % 4 of word q / 4; code
+            // d = t + 1 of weight j at code_place(j); positions j >= G hold the
+            // padding code 1
 #pragma unroll
             for (int i = 0; i < NCW; ++i) cw[i] = 0;
 #pragma unroll
-            for (int j = 0; j < 5 * B; ++j) {
-                const int q = j / 5;
-                const uint32_t pw = (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
-                                    << (8 * (q % 4));
+            for (int j = 0; j < PER * B; ++j) {
+                const uint32_t pw = code_place<FMT>(j);
                 if (j < G) {
                     const uint32_t hw = h[j >> 1] >> (16 * (j & 1));
                     const uint32_t d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
-                    cw[q / 4] += d * pw;
+                    cw[j / PER / 4] += d * pw;
                 } else {
-                    cw[q / 4] += pw;  // padding digit 1
+                    cw[j / PER / 4] += pw;  // padding code 1
                 }
             }
         } else {
@@ -294,18 +306,14 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
                 take(half, h);
 #pragma unroll
                 for (int jj = 0; jj < 64; ++jj) {
-                    const int j = 64 * half + jj, q = j / 5;
-                    const uint32_t pw = (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
-                                        << (8 * (q % 4));
+                    const int j = 64 * half + jj;
                     const uint32_t hw = h[jj >> 1] >> (16 * (jj & 1));
                     const uint32_t d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
-                    cw[q / 4] += d * pw;
+                    cw[j / PER / 4] += d * code_place<FMT>(j);
                 }
             }
 #pragma unroll
-            for (int j = G; j < 5 * B; ++j)  // padding digits 1
-                cw[j / 5 / 4] += (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
-                                 << (8 * ((j / 5) % 4));
+            for (int j = G; j < PER * B; ++j) cw[j / PER / 4] += code_place<FMT>(j);  // padding codes 1
         }
         if (active) {
             scales[gi] = s;
@@ -330,13 +338,13 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
-// Dynamic shared memory of quantize_pack_group_kernel<G>: the load ring.
+// Dynamic shared memory of quantize_pack_group_kernel: the load ring.
 static size_t quantize_ring_bytes(int G) { return (size_t)2 * 8 * 32 * ((G <= 64 ? 2 * G : 128) + 16); }
 
-template <int G>
+template <int G, int FMT = 3>
 static cudaError_t launch_quantize_group(const uint16_t* W, int64_t num_groups, uint8_t* codes, uint16_t* scales,
                                          uint32_t* d_err, cudaStream_t stream, int grid) {
-    auto kern = quantize_pack_group_kernel<G>;
+    auto kern = quantize_pack_group_kernel<G, FMT>;
     const size_t smem = quantize_ring_bytes(G);
     static std::atomic<int> smem_set{0};
     if ((int)smem > 48 * 1024 && (int)smem > smem_set.load()) {
@@ -418,6 +426,57 @@ cudaError_t launch_quantize_pack(const uint16_t* W, int64_t N, int64_t K, int G,
 #undef TQ_QP_CASE
 #undef TQ_QG_CASE
     quantize_pack_generic_kernel<<<grid_for(num_groups, 128, sm_count), 128, 0, stream>>>(
+        W, num_groups, G, codes, scales, d_err);
+    return cudaGetLastError();
+}
+
+// 2-bit format, any G: one thread per group, multi-word exact scale; code
+// t + 1 of weight j in bits 2 (j % 4) of byte j / 4, padding codes 1.
+__global__ void __launch_bounds__(128) quantize_pack2_generic_kernel(
+    const uint16_t* __restrict__ W, int64_t num_groups, int G, uint8_t* __restrict__ codes,
+    uint16_t* __restrict__ scales, uint32_t* __restrict__ d_err) {
+    const int B = (G + 3) / 4;
+    uint32_t err_acc = 0;
+    for (int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; gi < num_groups;
+         gi += (int64_t)gridDim.x * blockDim.x) {
+        const uint16_t* w = W + gi * G;
+        uint16_t s;
+        const uint32_t gerr = exact_group_scale(w, G, &s);
+        err_acc |= gerr;
+        scales[gi] = s;
+        const uint32_t th = trit_threshold(s);
+        uint8_t* out = codes + gi * B;
+        for (int q = 0; q < B; ++q) {
+            uint32_t byte = 0;
+            for (int i = 0; i < 4; ++i) {
+                const int j = 4 * q + i;
+                uint32_t d = 1;
+                if (j < G) {
+                    const uint32_t hw = w[j];
+                    d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
+                }
+                byte |= d << (2 * i);
+            }
+            out[q] = (uint8_t)byte;
+        }
+    }
+    if (err_acc && d_err) atomicOr(d_err, err_acc);
+}
+
+cudaError_t launch_quantize_pack2(const uint16_t* W, int64_t N, int64_t K, int G, uint8_t* codes,
+                                  uint16_t* scales, uint32_t* d_err, cudaStream_t stream, int sm_count) {
+    const int64_t num_groups = N * (K / G);
+    if (num_groups == 0) return cudaSuccess;
+    const int grid = grid_for((num_groups + 31) / 32 * 32, 256, sm_count);
+    switch (G) {
+        case 8: return launch_quantize_group<8, 2>(W, num_groups, codes, scales, d_err, stream, grid);
+        case 16: return launch_quantize_group<16, 2>(W, num_groups, codes, scales, d_err, stream, grid);
+        case 32: return launch_quantize_group<32, 2>(W, num_groups, codes, scales, d_err, stream, grid);
+        case 64: return launch_quantize_group<64, 2>(W, num_groups, codes, scales, d_err, stream, grid);
+        case 128: return launch_quantize_group<128, 2>(W, num_groups, codes, scales, d_err, stream, grid);
+        default: break;
+    }
+    quantize_pack2_generic_kernel<<<grid_for(num_groups, 128, sm_count), 128, 0, stream>>>(
         W, num_groups, G, codes, scales, d_err);
     return cudaGetLastError();
 }

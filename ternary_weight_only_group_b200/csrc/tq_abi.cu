@@ -27,6 +27,12 @@ cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* c
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                               int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                               cudaStream_t stream, int sm_count, bool* handled);
+cudaError_t launch_quantize_pack2(const uint16_t* W, int64_t N, int64_t K, int G, uint8_t* codes,
+                                  uint16_t* scales, uint32_t* d_err, cudaStream_t stream, int sm_count);
+cudaError_t launch_unpack2(const uint8_t* codes, const uint16_t* scales, int64_t N, int64_t K, int G, uint16_t* out,
+                           uint32_t* d_err, cudaStream_t stream, int sm_count);
+cudaError_t launch_gemv2(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales, int64_t N,
+                         int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err, cudaStream_t stream, int sm_count);
 cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes,
                            const uint16_t* scales, int64_t N, int64_t K, int G, void* Y,
                            int y_bf16, uint32_t* d_err, cudaStream_t stream, int sm_count,
@@ -102,6 +108,7 @@ struct MatmulArgs {
     int G;
     void* Y;
     tq_out_dtype yt;
+    int fmt = 3;  // 3: base-3 codes, 2: 2-bit codes
 };
 
 tq_status check_matmul(const MatmulArgs& a) {
@@ -109,7 +116,8 @@ tq_status check_matmul(const MatmulArgs& a) {
     if (a.yt != TQ_OUT_F32 && a.yt != TQ_OUT_BF16) return TQ_ERR_INVALID_ARG;
     if (a.M > 0 && a.K > (int64_t(1) << 62) / a.M) return TQ_ERR_INVALID_ARG;
     if (a.M > 0 && a.N > (int64_t(1) << 62) / a.M) return TQ_ERR_INVALID_ARG;
-    const size_t cb = tq_codes_bytes(a.N, a.K, a.G), sb = tq_scales_bytes(a.N, a.K, a.G);
+    const size_t cb = a.fmt == 2 ? tq2_codes_bytes(a.N, a.K, a.G) : tq_codes_bytes(a.N, a.K, a.G);
+    const size_t sb = tq_scales_bytes(a.N, a.K, a.G);
     const size_t xb = (size_t)a.M * (size_t)a.K * 2;
     const size_t yb = (size_t)a.M * (size_t)a.N * (a.yt == TQ_OUT_F32 ? 4 : 2);
     if ((xb && !a.X) || (cb && !a.codes) || (sb && !a.scales) || (yb && !a.Y)) return TQ_ERR_INVALID_ARG;
@@ -117,6 +125,7 @@ tq_status check_matmul(const MatmulArgs& a) {
         return TQ_ERR_INVALID_ARG;
     if (!aligned(a.X, 16) || !aligned(a.scales, 2) || !aligned(a.Y, a.yt == TQ_OUT_F32 ? 4 : 2))
         return TQ_ERR_ALIGNMENT;
+    if (a.fmt == 2 && !aligned(a.codes, 4)) return TQ_ERR_ALIGNMENT;
     return TQ_OK;
 }
 
@@ -248,6 +257,62 @@ tq_status tq_gemm(const void* X, int64_t M, const uint8_t* codes, const void* sc
     if (e != cudaSuccess) return from_cuda(e);
     if (!handled) return TQ_ERR_UNSUPPORTED;
     return TQ_OK;
+}
+
+// ---- 2-bit ternary format
+
+size_t tq2_codes_bytes(int64_t N, int64_t K, int G) {
+    if (!shape_ok(N, K, G)) return 0;
+    return (size_t)N * (size_t)(K / G) * (size_t)((G + 3) / 4);
+}
+
+tq_status tq2_quantize_pack(const void* W, int64_t N, int64_t K, int G, uint8_t* codes, void* scales,
+                            uint32_t* d_err, tq_stream_t stream) {
+    if (!shape_ok(N, K, G)) return TQ_ERR_INVALID_ARG;
+    const size_t wb = (size_t)N * (size_t)K * 2;
+    const size_t cb = tq2_codes_bytes(N, K, G), sb = tq_scales_bytes(N, K, G);
+    if ((wb && !W) || (cb && !codes) || (sb && !scales)) return TQ_ERR_INVALID_ARG;
+    if (overlap(codes, cb, W, wb) || overlap(scales, sb, W, wb) || overlap(codes, cb, scales, sb))
+        return TQ_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(scales, 2) || !aligned(codes, 4)) return TQ_ERR_ALIGNMENT;
+    if (wb == 0) return TQ_OK;
+    const DeviceInfo* d = nullptr;
+    if (tq_status st = device_info(&d)) return st;
+    return from_cuda(launch_quantize_pack2(static_cast<const uint16_t*>(W), N, K, G, codes,
+                                           static_cast<uint16_t*>(scales), d_err, (cudaStream_t)stream,
+                                           d->sm_count));
+}
+
+tq_status tq2_unpack_bf16(const uint8_t* codes, const void* scales, int64_t N, int64_t K, int G, void* W_out,
+                          uint32_t* d_err, tq_stream_t stream) {
+    if (!shape_ok(N, K, G)) return TQ_ERR_INVALID_ARG;
+    const size_t wb = (size_t)N * (size_t)K * 2;
+    const size_t cb = tq2_codes_bytes(N, K, G), sb = tq_scales_bytes(N, K, G);
+    if ((wb && !W_out) || (cb && !codes) || (sb && !scales)) return TQ_ERR_INVALID_ARG;
+    if (overlap(W_out, wb, codes, cb) || overlap(W_out, wb, scales, sb)) return TQ_ERR_INVALID_ARG;
+    if (!aligned(W_out, 16) || !aligned(scales, 2) || !aligned(codes, 4)) return TQ_ERR_ALIGNMENT;
+    if (wb == 0) return TQ_OK;
+    const DeviceInfo* d = nullptr;
+    if (tq_status st = device_info(&d)) return st;
+    return from_cuda(launch_unpack2(codes, static_cast<const uint16_t*>(scales), N, K, G,
+                                    static_cast<uint16_t*>(W_out), d_err, (cudaStream_t)stream, d->sm_count));
+}
+
+tq_status tq2_gemv(const void* X, int64_t M, const uint8_t* codes, const void* scales, int64_t N, int64_t K, int G,
+                   void* Y, tq_out_dtype yt, void* workspace, size_t ws_bytes, uint32_t* d_err,
+                   tq_stream_t stream) {
+    (void)workspace; (void)ws_bytes;
+    MatmulArgs a{X, M, codes, scales, N, K, G, Y, yt};
+    a.fmt = 2;
+    if (tq_status st = check_matmul(a)) return st;
+    if (M == 0 || N == 0) return TQ_OK;
+    if (K == 0) return TQ_ERR_UNSUPPORTED;
+    const DeviceInfo* d = nullptr;
+    if (tq_status st = device_info(&d)) return st;
+    const cudaError_t e = launch_gemv2(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
+                                       N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count);
+    if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
+    return from_cuda(e);
 }
 
 const char* tq_status_string(tq_status s) {

@@ -20,7 +20,7 @@ def built():
 
 def header_symbols():
     text = open(os.path.join(ROOT, "include", "tq.h")).read()
-    return sorted(set(re.findall(r"TQ_API\s+[\w\s\*]*?\b(tq_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"TQ_API\s+[\w\s\*]*?\b(tq2?_\w+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported():
@@ -44,12 +44,14 @@ def test_size_queries(N, K, G):
     assert tq.codes_bytes(N, K, G) == N * (K // G) * -(-G // 5)
     assert tq.scales_bytes(N, K, G) == N * (K // G) * 2
     assert tq.workspace_bytes(1, N, K, G) >= 0
+    assert tq.codes2_bytes(N, K, G) == N * (K // G) * -(-G // 4)
 
 
 @pytest.mark.parametrize("N,K,G", [(4, 100, 64), (4, 64, 0), (4, 64, -1), (-1, 64, 64),
                                    (4, -64, 64), (4, 8192, 8192)])
 def test_size_queries_reject_bad_shapes(N, K, G):
     assert tq.codes_bytes(N, K, G) == 0 and tq.scales_bytes(N, K, G) == 0
+    assert tq.codes2_bytes(N, K, G) == 0
 
 
 def fake(addr):
@@ -92,6 +94,22 @@ BAD_CALLS = [
                                              None, 0, None, None), tq.TQ_ERR_INVALID_ARG),
     ("gemm K%G", lambda L: L.tq_gemm(fake(0x1000), 1, fake(0x9000), fake(0xA000), 4, 96, 64, fake(0xB000), 1,
                                      None, 0, None, None), tq.TQ_ERR_INVALID_ARG),
+    ("2-bit pack G=0", lambda L: L.tq2_quantize_pack(fake(0x1000), 4, 64, 0, fake(0x9000), fake(0xA000), None,
+                                                     None), tq.TQ_ERR_INVALID_ARG),
+    ("2-bit pack codes misaligned", lambda L: L.tq2_quantize_pack(fake(0x1000), 4, 64, 64, fake(0x9002),
+                                                                  fake(0xA000), None, None), tq.TQ_ERR_ALIGNMENT),
+    ("2-bit pack overlap", lambda L: L.tq2_quantize_pack(fake(0x1000), 4, 64, 64, fake(0x1100), fake(0xA000),
+                                                         None, None), tq.TQ_ERR_INVALID_ARG),
+    ("2-bit unpack codes misaligned", lambda L: L.tq2_unpack_bf16(fake(0x9001), fake(0xA000), 4, 64, 64,
+                                                                  fake(0x1000), None, None), tq.TQ_ERR_ALIGNMENT),
+    ("2-bit unpack null scales", lambda L: L.tq2_unpack_bf16(fake(0x9000), None, 4, 64, 64, fake(0x1000), None,
+                                                             None), tq.TQ_ERR_INVALID_ARG),
+    ("2-bit gemv codes misaligned", lambda L: L.tq2_gemv(fake(0x1000), 1, fake(0x9002), fake(0xA000), 4, 64, 64,
+                                                         fake(0xB000), 0, None, 0, None, None), tq.TQ_ERR_ALIGNMENT),
+    ("2-bit gemv Y overlaps codes", lambda L: L.tq2_gemv(fake(0x1000), 1, fake(0x9000), fake(0xA000), 4, 64, 64,
+                                                         fake(0x9010), 0, None, 0, None, None), tq.TQ_ERR_INVALID_ARG),
+    ("2-bit gemv K%G", lambda L: L.tq2_gemv(fake(0x1000), 1, fake(0x9000), fake(0xA000), 4, 96, 64,
+                                            fake(0xB000), 0, None, 0, None, None), tq.TQ_ERR_INVALID_ARG),
 ]
 
 
@@ -105,6 +123,9 @@ def test_empty_inputs_are_noops():
     assert L.tq_quantize_pack(None, 0, 64, 64, None, None, None, None) == tq.TQ_OK
     assert L.tq_unpack_bf16(None, None, 0, 128, 64, None, None, None) == tq.TQ_OK
     assert L.tq_gemv(None, 0, fake(0x9000), fake(0xA000), 4, 64, 64, None, 0, None, 0, None, None) == tq.TQ_OK
+    assert L.tq2_quantize_pack(None, 0, 64, 64, None, None, None, None) == tq.TQ_OK
+    assert L.tq2_unpack_bf16(None, None, 0, 128, 64, None, None, None) == tq.TQ_OK
+    assert L.tq2_gemv(None, 0, fake(0x9000), fake(0xA000), 4, 64, 64, None, 0, None, 0, None, None) == tq.TQ_OK
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):

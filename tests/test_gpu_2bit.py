@@ -1,0 +1,167 @@
+"""GPU parity of the 2-bit ternary format (four codes per byte) against the oracle.
+
+tq2_quantize_pack and tq2_unpack_bf16: bit-exact on scales, code bytes,
+decoded bf16 weights and error bits.  tq2_gemv: the fused matmul's
+tolerances (fp32 max_n |gpu - oracle| <= 1e-3 * max_n |oracle| per row; bf16
+|gpu - oracle| <= 2e-2 + 2e-2 |oracle|; NaN rows must coincide) and the
+oracle's error bits.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+import ternary_weight_only_group_b200 as tq
+from tests.parity import (assert_close_bf16, assert_rows_close_f32, bits_u16, to_dev_bf16, to_dev_f16,
+                          to_dev_u8, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_pack2(W_bits, G):
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    codes, scales = tq.quantize_pack2(to_dev_bf16(W_bits), G, d_err=err)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), bits_u16(scales), int(err.item())
+
+
+def gpu_unpack2(codes, scales_bits, N, K, G):
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = tq.unpack2_bf16(to_dev_u8(codes), to_dev_f16(scales_bits), N, K, G, d_err=err)
+    torch.cuda.synchronize()
+    return bits_u16(out), int(err.item())
+
+
+def check_pack2(W_bits, G):
+    c_ref, s_ref, e_ref = oracle.quantize_pack2(W_bits, G)
+    c, s, e = gpu_pack2(W_bits, G)
+    assert np.array_equal(s.reshape(s_ref.shape), s_ref), np.argwhere(s.reshape(s_ref.shape) != s_ref)[:8]
+    assert np.array_equal(c.reshape(c_ref.shape), c_ref), np.argwhere(c.reshape(c_ref.shape) != c_ref)[:8]
+    assert e == e_ref
+    return c_ref, s_ref
+
+
+def check_unpack2(codes, scales, N, K, G):
+    w_ref, e_ref = oracle.unpack2_bf16(codes, scales, N, K, G)
+    w, e = gpu_unpack2(codes, scales, N, K, G)
+    assert np.array_equal(w.reshape(w_ref.shape), w_ref), np.argwhere(w.reshape(w_ref.shape) != w_ref)[:8]
+    assert e == e_ref
+
+
+@pytest.mark.parametrize("G", [8, 16, 32, 64, 128, 256, 6, 12, 48, 100])
+def test_group_sizes(G):
+    """Group kernels (G = 8..128), the generic kernel (others), word and
+    generic unpack; ragged row counts; every exponent, zero and subnormal
+    groups, non-finite weights and overflowing means."""
+    K = G * max(2, 512 // G)
+    N = 37
+    W = synthetic.weights(N, K, index=G, outlier_frac=0.01)
+    W[5] = synthetic.random_bf16_bits(K, seed=G)
+    W[6] = 0
+    W[7, : K // 2] = 0x0001
+    W[8, 1] = 0x7F80
+    W[9, :G] = 0x7F7F
+    codes, scales = check_pack2(W, G)
+    check_unpack2(codes, scales, N, K, G)
+
+
+@pytest.mark.parametrize("G", [64, 128])
+def test_ffn_full_size(G):
+    W = synthetic.ffn_matrix("gate")
+    codes, scales = check_pack2(W, G)
+    check_unpack2(codes, scales, W.shape[0], W.shape[1], G)
+
+
+@pytest.mark.parametrize("G", [16, 64, 128, 256, 10])
+def test_unpack2_rejections(G):
+    """Code 3 anywhere, padding codes other than 1, rejected scales and zero
+    groups; a rejected group is NaN as a whole, the error bits are the oracle's."""
+    N, K = 50, 4 * G
+    W = synthetic.weights(N, K, index=5)
+    codes, scales, _ = oracle.quantize_pack2(W, G)
+    rng = np.random.default_rng(G)
+    B = codes.shape[2]
+    for n in range(0, N, 3):
+        g = rng.integers(0, K // G)
+        kind = n % 4
+        if kind == 0:
+            q, i = rng.integers(0, B), rng.integers(0, 4)
+            codes[n, g, q] |= 3 << (2 * i)
+        elif kind == 1 and G % 4:
+            codes[n, g, B - 1] &= 0x3F  # last padding code 0
+        elif kind == 2:
+            scales[n, g] = [0x7C00, 0xFC00, 0x7E01, 0x8001][n % 4]
+        else:
+            scales[n, g] = 0
+    check_unpack2(codes, scales, N, K, G)
+
+
+def run_gemv2(X, codes, scales, N, K, G, out_dtype):
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Y = tq.gemv2(to_dev_bf16(X), to_dev_u8(codes), to_dev_f16(scales), N, K, G, out_dtype=out_dtype, d_err=err)
+    torch.cuda.synchronize()
+    return to_f64(Y), int(err.item())
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 11])
+@pytest.mark.parametrize("N,K,G", [(3584, 1024, 64), (1024, 3584, 128), (1037, 1152, 128), (301, 1040, 16),
+                                   (130, 4096, 256), (77, 2048, 32)])
+def test_gemv2(N, K, G, M):
+    """Token counts 1..11 (two launches past 8), ragged row batches and code
+    words per row that are not multiples of 32 lanes; fp32 and bf16 outputs."""
+    W = synthetic.weights(N, K, index=N + G)
+    codes, scales, _ = oracle.quantize_pack2(W, G)
+    X = synthetic.activations(M, K)
+    ref = oracle.linear2(X, codes, scales, N, K, G)
+    Y, e = run_gemv2(X, codes, scales, N, K, G, torch.float32)
+    assert_rows_close_f32(Y, ref)
+    assert e == 0
+    Yb, _ = run_gemv2(X, codes, scales, N, K, G, torch.bfloat16)
+    assert_close_bf16(Yb, ref)
+
+
+def test_gemv2_rejected_groups():
+    N, K, G, M = 515, 1024, 64, 3
+    W = synthetic.weights(N, K, index=11)
+    codes, scales, _ = oracle.quantize_pack2(W, G)
+    codes[5, 2, 7] |= 0xC0      # code 3
+    scales[130, 0] = 0x7C00     # Inf scale
+    scales[514, 15] = 0x8000    # -0 scale, last row
+    scales[77, 3] = 0           # zero group: finite
+    X = synthetic.activations(M, K)
+    ref = oracle.linear2(X, codes, scales, N, K, G)
+    _, e_ref = oracle.unpack2_bf16(codes, scales, N, K, G)
+    Y, e = run_gemv2(X, codes, scales, N, K, G, torch.float32)
+    assert_rows_close_f32(Y, ref)
+    assert np.all(np.isnan(Y[:, [5, 130, 514]])) and np.all(np.isfinite(Y[:, 77]))
+    assert e == e_ref == tq.DERR_BYTE | tq.DERR_SCALE
+
+
+def test_gemv2_stack_full_size_sampled():
+    """The 24-layer gate/up stack as one [172032 x 1024] matrix, G=128, M=1
+    (the streaming decode workload), packed on the GPU; sampled output
+    columns against the oracle."""
+    N, K, G = 48 * 3584, 1024, 128
+    W = np.concatenate([synthetic.ffn_matrix(n, layer=l, outliers=False)
+                        for l in range(24) for n in ("gate", "up")])
+    c, s, e = gpu_pack2(W, G)
+    assert e == 0
+    X = synthetic.activations(1, K)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Y = tq.gemv2(to_dev_bf16(X), to_dev_u8(c), to_dev_f16(s), N, K, G, out_dtype=torch.float32, d_err=err)
+    torch.cuda.synchronize()
+    cols = np.random.default_rng(0).choice(N, size=512, replace=False)
+    c_ref, s_ref, _ = oracle.quantize_pack2(W[cols], G)
+    assert np.array_equal(c.reshape(N, K // G, -1)[cols], c_ref)
+    ref = oracle.linear2(X, c_ref, s_ref, len(cols), K, G)
+    assert_rows_close_f32(to_f64(Y)[:, cols], ref)
+    assert int(err.item()) == 0
+
+
+def test_gemv2_unsupported_group_size():
+    N, K, G = 64, 480, 48
+    W = synthetic.weights(N, K, index=1)
+    codes, scales, _ = oracle.quantize_pack2(W, G)
+    with pytest.raises(tq.TQError, match="UNSUPPORTED"):
+        run_gemv2(synthetic.activations(1, K), codes, scales, N, K, G, torch.float32)
