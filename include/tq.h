@@ -162,9 +162,11 @@ TQ_API tq_status tq2_unpack_bf16(const uint8_t *codes, const void *scales_f16, i
                           int G, void *W_bf16_out, uint32_t *d_err, tq_stream_t stream);
 /* Fused unpack-and-scale matmul on the 2-bit format, CUDA cores, any M >= 1
  * (eight tokens per launch); result definition, arguments, alignment and
- * ordering as tq_gemv (X is read after the preceding work has completed,
- * codes and scales too).  Covers G in {16, 32, 64, 128, 256} and
- * K <= 49152; other shapes return TQ_ERR_UNSUPPORTED. */
+ * ordering rule as tq_gemv (X is read after the preceding work has
+ * completed; codes and scales may be read before, so the kernel launched
+ * immediately before on the same stream must not write them).  Covers G in
+ * {16, 32, 64, 128, 256} and K <= 49152; other shapes return
+ * TQ_ERR_UNSUPPORTED. */
 TQ_API tq_status tq2_gemv(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
                    int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,
                    size_t ws_bytes, uint32_t *d_err, tq_stream_t stream);
