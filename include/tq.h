@@ -3,10 +3,11 @@
  *
  * The operations follow two pages:
  *   "precisit/pack-unpack-run" (codec.py description and payload-rate
- *   paragraph): per group of G input columns, a mean-absolute scale rounded to
- *   fp16 (binary16), nearest-even ternary codes, five base-three digits per
- *   byte, each group byte-aligned with zero-trit padding, bytes 243..255
- *   invalid, a zero stored scale producing a zero group, decoding to bf16.
+ *   paragraph): per group of G input columns, a scale equal to the mean of
+ *   |w| kept as binary16, trits by rounding w / scale half to even, base-3
+ *   digits five to a byte, every group starting on a byte boundary with its
+ *   unused digit slots holding the zero trit, byte values 243..255 invalid,
+ *   a zero scale decoding to an all-zero group, and decoding to bf16.
  *   tiny-llm "Week 2 Day 3: Quantize the Model" ("Mathematical Formulation",
  *   "Computation Flow"): C = A B^T with B reconstructed per group and the
  *   products accumulated in float.
@@ -83,8 +84,8 @@ TQ_API size_t tq_scales_bytes(int64_t N, int64_t K, int G);
 TQ_API size_t tq_workspace_bytes(int64_t M, int64_t N, int64_t K, int G);
 
 /*
- * Quantize and pack ("precisit/pack-unpack-run", codec.py: mean-absolute
- * scale rounded to fp16, nearest-even ternary codes, base-3 packing).
+ * Quantize and pack ("precisit/pack-unpack-run", codec.py: per-group mean
+ * |w| scale in fp16, round-half-even trits, base-3 packing).
  * W_bf16: [N][K] bf16, 16-byte aligned.  codes: tq_codes_bytes() bytes.
  * scales_f16: [N][K/G] binary16, 2-byte aligned.
  * Scale = RNE_binary16(exact mean of |w| over the group); trit =

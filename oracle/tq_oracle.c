@@ -10,12 +10,14 @@
  * fusion or reordering beyond what those definitions state.
  *
  * Sources (page title, section):
- *   [codec]  precisit/pack-unpack-run, the codec.py description: mean-absolute
- *            scale rounded to fp16, nearest-even ternary codes, five base-three
- *            digits per byte, each group byte-aligned with zero-trit padding,
- *            values 243..255 invalid; decoding restores bf16.
- *   [rules]  precisit/pack-unpack-run, the paragraph after it: no calibration,
- *            a zero stored scale produces a zero group, columns divisible by G.
+ *   [codec]  precisit/pack-unpack-run, the codec.py description: the group
+ *            scale is the mean of |w| kept as fp16; trits round w / scale
+ *            half to even; base-3 digits, five to a byte; each group starts
+ *            on a byte boundary, its unused digit slots holding the zero
+ *            trit; byte values 243..255 are invalid; the decoder gives bf16.
+ *   [rules]  precisit/pack-unpack-run, the paragraph after it: no calibration;
+ *            a scale stored as zero decodes to an all-zero group; G divides
+ *            the number of columns.
  *   [rate]   precisit/pack-unpack-run, payload-rate paragraph:
  *            8*(ceil(G/5)+2)/G bits per weight.
  *   [two]    "Autoregressive Language Model on the 6502 Processor", summary:
@@ -195,7 +197,7 @@ static int big_any_below(const bigsum *s, int k)
 }
 
 /*
- * [codec] "mean-absolute scale rounded to fp16".
+ * [codec] the group scale: mean of |w|, kept as fp16.
  * Computes S = sum |w_j| exactly, then s = RNE_binary16(S / G) by exact
  * comparison with the binary16 grid.  Returns error bits; *s_out is the
  * stored scale (+0 for an all-zero, tiny, non-finite or overflowing group).
@@ -243,7 +245,7 @@ uint32_t oracle_group_scale(const uint16_t *w, int64_t G, uint16_t *s_out)
 }
 
 /*
- * [codec] "nearest-even ternary codes", [rules] zero scale => zero group.
+ * [codec] trits by rounding half to even, [rules] zero scale => zero group.
  * t = clamp(round_half_even(w / s), -1, +1); the quotient of a bf16 by a
  * binary16 is computed in binary64, where it is exact enough that no false
  * tie can appear (a true quotient near 1/2 differs from it by far more than

@@ -1,8 +1,9 @@
 // quantize_pack.cu -- per-group ternary quantizer and base-3 packer.
 //
-// "precisit/pack-unpack-run", codec.py description: mean-absolute scale
-// rounded to fp16, nearest-even ternary codes, five base-three digits per
-// byte, each group byte-aligned with zero-trit padding.
+// "precisit/pack-unpack-run", codec.py description: each group's scale is
+// the mean of |w| stored as fp16; trits come from rounding w / scale half to
+// even; five trits go into a byte as base-3 digits; every group starts on a
+// byte boundary and unused digit slots hold the zero trit.
 //
 // The matrix is treated as a flat run of N*K/G groups (a group never crosses
 // a row because K % G == 0).  Fast path (G = 8 * 2^k, 8 <= G <= 256): a warp

@@ -1,8 +1,8 @@
 // unpack.cu -- base-3 decoder to bf16.
 //
-// "precisit/pack-unpack-run", codec.py description: decoding; values 243
-// through 255 are invalid; the decoder restores the weights as bf16.  A zero
-// stored scale produces a zero group (the paragraph after it).
+// "precisit/pack-unpack-run", codec.py description: the decoder turns codes
+// back into bf16 weights and treats byte values from 243 up as invalid; the
+// paragraph after it: a scale stored as zero decodes its whole group to 0.
 //
 // Fast path (G = 8 * 2^k, 8 <= G <= 256): G/8 lanes per group, each lane
 // writes 8 consecutive bf16 with one 16-byte store.  Each lane checks the

@@ -140,8 +140,8 @@ def test_invalid_bytes_rejected(b):
 
 
 def test_changed_valid_byte_changes_reconstruction():
-    """The page's test list: a changed valid code byte must change the
-    reconstruction.  Full bytes: the 243 decodings are pairwise distinct.
+    """The page's test list: altering any valid code byte alters the decoded
+    weights.  Full bytes: the 243 decodings are pairwise distinct.
     Partial last byte (G=64: 4 digits + 1 padding): any change either
     changes the decoded values or is rejected."""
     scales = np.array([[0x3C00]], dtype=np.uint16)
@@ -187,7 +187,7 @@ def test_no_padding_when_G_multiple_of_5(G):
 
 
 def test_zero_group_encoding():
-    """Zero stored scale produces a zero group: every byte 1+3+9+27+81 = 121,
+    """A scale of zero gives an all-zero group: every byte 1+3+9+27+81 = 121,
     decoded as +0."""
     for G in (1, 3, 5, 64, 128):
         W = np.zeros((2, 2 * G), dtype=np.uint16)

@@ -2,8 +2,8 @@
 
 "precisit/pack-unpack-run", screen.py and test_codec.py descriptions: per-
 tensor NPZ files with codes and fp16 scales; the decoder accepts only the
-package and checks it; file replay; a changed valid code byte must change
-the reconstruction.  Codes come from the oracle; decoding on the CPU side of
+package and checks it; file replay; altering any valid code byte alters the
+decoded weights.  Codes come from the oracle; decoding on the CPU side of
 these tests is the oracle's.
 """
 import json
@@ -49,8 +49,8 @@ def test_round_trip_bit_exact(tmp_path):
 
 
 def test_payload_rates_in_manifest(tmp_path):
-    """The page's rates: 1.875 bpw at G=64 and 1.750 at G=128 (base-3); the
-    2-bit format stores 8 * (G/4 + 2) / G."""
+    """The page's rates for base-3 (G=64: 1.875 bits per weight, G=128:
+    1.75); the 2-bit format stores 8 * (G/4 + 2) / G."""
     man = pkg.write_package(str(tmp_path / "p"), make_tensors())["tensors"]
     assert man["layers.0.mlp.gate_proj"]["payload_bits_per_weight"] == 1.875
     assert man["layers.0.mlp.down_proj"]["payload_bits_per_weight"] == 1.75
