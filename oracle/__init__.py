@@ -80,6 +80,9 @@ def _load():
             lib.oracle_quantize_pack2.restype = ctypes.c_uint32
             lib.oracle_unpack2_bf16.argtypes = [u8p, u16p, i64, i64, i64, u16p]
             lib.oracle_unpack2_bf16.restype = ctypes.c_uint32
+            u32p = ctypes.POINTER(ctypes.c_uint32)
+            lib.oracle_w4_dequant.argtypes = [u32p, u16p, u16p, i64, i64, i64, f64p]
+            lib.oracle_w4_dequant.restype = None
             lib.oracle_matmul.argtypes = [u16p, i64, i64p, i64, u16p, i64, i64, f64p]
             lib.oracle_matmul.restype = None
             lib.oracle_matmul_points.argtypes = [u16p, u16p, i64, i64p, i64p, i64, f64p]
@@ -256,3 +259,28 @@ def linear2(X_bits, codes, scales, N: int, K: int, G: int, rows=None) -> np.ndar
     """The fused layer on the 2-bit format: Y = X . unpack2(codes, scales)^T (binary64)."""
     Wd, _ = unpack2_bf16(codes, scales, N, K, G)
     return matmul(X_bits, Wd, rows)
+
+
+# ---------------------------------------------------------------- W4A16 affine format
+
+def w4_dequant(codes: np.ndarray, scales: np.ndarray, biases: np.ndarray, N: int, K: int, G: int) -> np.ndarray:
+    """codes uint32 [N, K/8] (first code in the low nibble), bf16 scales and
+    biases [N, K/G] -> binary64 weights q * s + b [N, K]."""
+    if G < 1 or K % G or K % 8:
+        raise ValueError(f"K={K} must be a multiple of G={G} and of 8")
+    c = np.ascontiguousarray(codes, dtype=np.uint32)
+    s = _u16(scales)
+    b = _u16(biases)
+    assert c.size == N * (K // 8) and s.size == N * (K // G) and b.size == N * (K // G)
+    out = np.zeros((N, K), dtype=np.float64)
+    _load().oracle_w4_dequant(_ptr(c, ctypes.c_uint32), _ptr(s, ctypes.c_uint16), _ptr(b, ctypes.c_uint16),
+                              N, K, G, _ptr(out, ctypes.c_double))
+    return out
+
+
+def linear_w4(X_bits, codes, scales, biases, N: int, K: int, G: int) -> np.ndarray:
+    """Y = X . W^T with W the W4 weights reconstructed in binary64 and X bf16
+    widened exactly; the products and sums in binary64 (numpy matmul)."""
+    X = _u16(X_bits)
+    xv = (X.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return xv @ w4_dequant(codes, scales, biases, N, K, G).T

@@ -23,6 +23,11 @@
  *   [two]    "Autoregressive Language Model on the 6502 Processor", summary:
  *            BitNet ternary weights (-1, 0, 1) packed four parameters per
  *            byte (the 2-bit alternative to the base-3 codec).
+ *   [w4]     tiny-llm "Week 2 Day 3: Quantize the Model", "Group-Wise Affine
+ *            Quantization", "Reconstruct a Stored Group" and "Packed Storage
+ *            Layout": unsigned 4-bit codes, eight per 32-bit word with the
+ *            first code in the low nibble; per group of G columns a bf16
+ *            scale (signed) and a bf16 bias; weight = q * scale + bias.
  *   [mm]     tiny-llm "Week 2 Day 3: Quantize the Model", "Mathematical
  *            Formulation" and "Computation Flow": C[i,k] = sum_j A[i,j]*B[k,j]
  *            with B reconstructed per group of G input columns, accumulated in
@@ -500,4 +505,32 @@ uint32_t oracle_unpack2_bf16(const uint8_t *codes, const uint16_t *scales, int64
         }
     }
     return err;
+}
+
+/* ------------------------------------------------------------------ */
+/* [w4] The W4A16 affine format: decoding only (the page's checkpoint   */
+/* supplies codes, scales and biases; it gives no quantizer).           */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Reconstruct every weight of a row-major [N x K] W4 matrix in binary64:
+ * code q of column k is nibble k % 8 (bits 4 (k % 8) .. 4 (k % 8) + 3) of
+ * word k / 8 of its row; w = q * s + b with the group's bf16 scale s and bias
+ * b (group k / G).  q * s is exact (a 4-bit integer times an 8-bit
+ * significand); the sum with b is exact unless the two differ by more than
+ * about 40 binades.  codes: [N][K/8] uint32; scales, biases: [N][K/G] bf16.
+ */
+void oracle_w4_dequant(const uint32_t *codes, const uint16_t *scales, const uint16_t *biases,
+                       int64_t N, int64_t K, int64_t G, double *W_out)
+{
+    int64_t ng = K / G, words = K / 8;
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t k = 0; k < K; k++) {
+            uint32_t word = codes[n * words + k / 8];
+            int q = (int)((word >> (4 * (k % 8))) & 0xFu);
+            double sc = oracle_bf16_value(scales[n * ng + k / G]);
+            double bi = oracle_bf16_value(biases[n * ng + k / G]);
+            W_out[n * K + k] = (double)q * sc + bi;
+        }
+    }
 }
