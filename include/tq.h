@@ -34,7 +34,10 @@
  * synchronous error code means nothing was launched.  Data errors found by
  * the kernels are OR-ed into *d_err (a device word the caller zeroes; may be
  * NULL) using the TQ_DERR_* bits.  No exceptions cross this boundary and
- * there is no CPU fallback.  Calls are thread-safe.
+ * there is no CPU fallback.  Calls are thread-safe.  One device per process:
+ * the kernels' shared-memory size attributes are raised once per process, on
+ * the device current at the first call that needs them, so launches on a
+ * second device of the same process may fail with TQ_ERR_CUDA.
  */
 #ifndef TQ_H
 #define TQ_H
