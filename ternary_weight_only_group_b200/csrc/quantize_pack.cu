@@ -129,6 +129,9 @@ __global__ void __launch_bounds__(256) quantize_pack_pow2_kernel(
             }
         }
     }
+    // Stores visible device-wide before the block exits: a matmul launched next on
+    // the stream may read codes and scales before its grid-dependency wait.
+    __threadfence();
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
@@ -336,6 +339,9 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
         __syncwarp();
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
+    // Stores visible device-wide before the block exits: a matmul launched next on
+    // the stream may read codes and scales before its grid-dependency wait.
+    __threadfence();
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
@@ -347,12 +353,9 @@ static cudaError_t launch_quantize_group(const uint16_t* W, int64_t num_groups, 
                                          uint32_t* d_err, cudaStream_t stream, int grid) {
     auto kern = quantize_pack_group_kernel<G, FMT>;
     const size_t smem = quantize_ring_bytes(G);
-    static std::atomic<int> smem_set{0};
-    if ((int)smem > 48 * 1024 && (int)smem > smem_set.load()) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        smem_set.store((int)smem);
-    }
+    static SmemAttr smem_attr;
+    if ((int)smem > 48 * 1024)
+        if (cudaError_t e = smem_attr.ensure(kern, (int)smem)) return e;
     kern<<<grid, 256, smem, stream>>>(W, num_groups, codes, scales, d_err);
     return cudaGetLastError();
 }
@@ -387,6 +390,9 @@ __global__ void __launch_bounds__(128) quantize_pack_generic_kernel(
             out[q] = (uint8_t)byte;
         }
     }
+    // Stores visible device-wide before the block exits: a matmul launched next on
+    // the stream may read codes and scales before its grid-dependency wait.
+    __threadfence();
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
@@ -461,6 +467,9 @@ __global__ void __launch_bounds__(128) quantize_pack2_generic_kernel(
             out[q] = (uint8_t)byte;
         }
     }
+    // Stores visible device-wide before the block exits: a matmul launched next on
+    // the stream may read codes and scales before its grid-dependency wait.
+    __threadfence();
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
