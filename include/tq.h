@@ -83,7 +83,12 @@ typedef enum { TQ_OUT_F32 = 0, TQ_OUT_BF16 = 1 } tq_out_dtype;
 TQ_API size_t tq_codes_bytes(int64_t N, int64_t K, int G);
 /* Bytes of the scales buffer: N * (K/G) * 2.  0 for invalid shapes. */
 TQ_API size_t tq_scales_bytes(int64_t N, int64_t K, int G);
-/* Bytes of device scratch tq_gemv / tq_gemm need for these shapes (may be 0). */
+/* Bytes of device scratch tq_gemv / tq_gemm need for these shapes.  Every
+ * kernel of this build keeps its partial sums on chip (registers, shared
+ * memory, distributed shared memory of a cluster, tensor memory), so this is
+ * 0 for every shape and the workspace arguments below are accepted but not
+ * read; callers that pass a buffer of this size stay correct if a later
+ * build needs one. */
 TQ_API size_t tq_workspace_bytes(int64_t M, int64_t N, int64_t K, int G);
 
 /*
@@ -122,6 +127,7 @@ TQ_API tq_status tq_unpack_bf16(const uint8_t *codes, const void *scales_f16, in
  * kernels up to 64 tokens, a row kernel beyond and for the shapes those do
  * not cover.  X: [M][K] bf16, 16-byte aligned; Y: [M][N]
  * (fp32: 4-byte aligned, bf16: 2-byte aligned), must not overlap the inputs.
+ * K == 0 is allowed: every output is an empty sum and Y is set to +0.
  * workspace: at least tq_workspace_bytes(M, N, K, G) bytes of device scratch
  * (NULL allowed when that is 0), 256-byte aligned.
  * Ordering: the kernels are launched as programmatic dependents of the work
@@ -129,7 +135,10 @@ TQ_API tq_status tq_unpack_bf16(const uint8_t *codes, const void *scales_f16, in
  * codes and scales (the weights) may be read while it is still finishing, so
  * they must not be written by the kernel launched immediately before this
  * call on the same stream (write them earlier, or on another stream and
- * join with an event).
+ * join with an event).  The one exception is this library's own
+ * tq_quantize_pack / tq2_quantize_pack: they never release their dependents
+ * early and make their stores visible device-wide before their blocks exit,
+ * so a matmul may directly follow them on the same buffers and stream.
  */
 TQ_API tq_status tq_gemv(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
                   int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,
@@ -174,6 +183,32 @@ TQ_API tq_status tq2_unpack_bf16(const uint8_t *codes, const void *scales_f16, i
 TQ_API tq_status tq2_gemv(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
                    int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,
                    size_t ws_bytes, uint32_t *d_err, tq_stream_t stream);
+
+/*
+ * The W4A16 affine format (tiny-llm "Week 2 Day 3: Quantize the Model",
+ * "Group-Wise Affine Quantization", "Reconstruct a Stored Group", "Packed
+ * Storage Layout"), a second weight format next to the ternary codes:
+ * unsigned 4-bit codes q, eight per 32-bit word, code j of a row in bits
+ * 4 (j mod 8) .. 4 (j mod 8) + 3 of word j / 8 (first code in the low nibble);
+ * per group of G columns (G a multiple of 8) a signed bf16 scale s and a
+ * bf16 bias b; the weight is w = q * s + b.  Buffers: codes uint32 [N][K/8]
+ * (4-byte aligned; 16-byte aligned for the fast kernel), scales and biases
+ * bf16 [N][K/G] (2-byte aligned), X bf16 [M][K] (16-byte aligned), Y as for
+ * tq_gemv.  There are no invalid codes and no data-error bits.
+ */
+/* Bytes of the W4 codes buffer: N * (K/8) * 4.  0 for invalid shapes or G % 8 != 0. */
+TQ_API size_t tq_w4_codes_bytes(int64_t N, int64_t K, int G);
+/* Decode matmul on the W4 format, CUDA cores, any M >= 1 (eight tokens per
+ * launch): Y[m][n] = sum_g (s[n][g] * sum_{j in g} q[n][j] X[m][j] + b[n][g] *
+ * sum_{j in g} X[m][j]) with fp32 accumulation ("Stage 2: SIMD Matvec" factors
+ * the bias out of the group's dot product), written as fp32 or RNE bf16.
+ * Ordering rule as tq_gemv.  G % 32 == 0 with K % 32 == 0 and K <= 4096 take
+ * the streaming kernel, other shapes a plain one-warp-per-row kernel.
+ * Errors: TQ_ERR_INVALID_ARG (shapes, G % 8, nulls, Y overlapping an input),
+ * TQ_ERR_ALIGNMENT, TQ_ERR_CUDA. */
+TQ_API tq_status tq_w4_gemv(const void *X_bf16, int64_t M, const uint32_t *codes, const void *scales_bf16,
+                     const void *biases_bf16, int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype,
+                     tq_stream_t stream);
 
 /* Human-readable name of a status code (static string). */
 TQ_API const char *tq_status_string(tq_status s);

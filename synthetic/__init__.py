@@ -102,3 +102,18 @@ def random_bf16_bits(shape, seed: int, finite_only: bool = True) -> np.ndarray:
         bad = (b & 0x7F80) == 0x7F80
         b[bad] &= 0xBFFF  # clear the top exponent bit: a finite pattern
     return b
+
+
+def w4_params(N: int, K: int, G: int, index: int = 0):
+    """Seeded W4A16 affine parameters of an [N, K] matrix: codes uint32
+    [N, K/8] (eight uniform 4-bit codes per word), scales and biases as bf16
+    bit patterns [N, K/G].  Magnitudes follow an affine 4-bit quantization
+    of N(0, 0.02) weights over groups of G (scale ~ range / 15, bias ~ the
+    group minimum); scales carry random signs."""
+    rng = np.random.default_rng(SEED_W + 5000 + index)
+    codes = rng.integers(0, 1 << 32, size=(N, K // 8), dtype=np.uint64).astype(np.uint32)
+    mag = rng.uniform(0.004, 0.009, size=(N, K // G)).astype(np.float32)
+    sign = np.where(rng.random(size=(N, K // G)) < 0.5, -1.0, 1.0).astype(np.float32)
+    scales = to_bf16_bits(mag * sign)
+    biases = to_bf16_bits(rng.normal(0.0, 0.05, size=(N, K // G)).astype(np.float32))
+    return codes, scales, biases

@@ -68,6 +68,7 @@ struct Params {
     int CS;  // cluster size = split of K
     int y_bf16;
     uint32_t pad_base, pad_span;  // canonical range of a group's last code byte
+    WaitCfg wc;                   // wait bound and the withheld-load test hook
 };
 
 template <int NT, bool CODES_TMA>
@@ -86,11 +87,13 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
     const int nkl = kb_hi - kb_lo;  // stages of this CTA (>= 1)
     constexpr uint32_t kCols = NT < 32 ? 32 : NT;
     volatile int* abort_flag = &sm.abort_flag;
+    const uint64_t lim = p.wc.limit_ns;
 
     // Dependent launches may start now: only the X loads below wait for the
     // preceding kernel (codes and scales are weights, see tq_gemv's ordering
     // rule); every Y store follows MMAs that consumed X.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    cluster_arrive_relaxed();  // waited on before the first store into a peer's shared memory
     fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
@@ -113,6 +116,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    cluster_wait();  // every CTA of the cluster is running: the partial pushes below may target it
     const uint32_t tmem = sm.tmem_base;
 
     auto stage_geom = [&](int kb, int& g, int& c0, int& q_lo) {
@@ -128,11 +132,13 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
             int issued = 0;
             for (int i = 0; i < nkl; ++i) {
                 const int kb = kb_lo + i, st = i % STAGES, use = i / STAGES;
-                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
+                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
                 int g, c0, q_lo;
                 stage_geom(kb, g, c0, q_lo);
-                mbar_arrive_expect_tx(&sm.full_x[st], NT * 128);
-                tma_load_2d(sm.x[st], &tmap_x, kb * BK, 0, &sm.full_x[st]);
+                if (!(p.wc.withhold_x && i == 0)) {  // test hook: the first load left out
+                    mbar_arrive_expect_tx(&sm.full_x[st], NT * 128);
+                    tma_load_2d(sm.x[st], &tmap_x, kb * BK, 0, &sm.full_x[st]);
+                }
                 if (CODES_TMA) {
                     mbar_arrive_expect_tx(&sm.full_c[st], C_STAGE);
                     tma_load_2d(sm.c[st], &tmap_c, (g * p.B + q_lo) & ~15, (int)n0, &sm.full_c[st]);
@@ -142,10 +148,10 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
             for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
                 const int st = i % STAGES, use = i / STAGES;
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(&sm.full_x[st], use & 1) && globaltimer() - t0 < kTimeoutNs) {
+                while (!mbar_try_wait(&sm.full_x[st], use & 1) && globaltimer() - t0 < lim) {
                 }
                 if (CODES_TMA)
-                    while (!mbar_try_wait(&sm.full_c[st], use & 1) && globaltimer() - t0 < kTimeoutNs) {
+                    while (!mbar_try_wait(&sm.full_c[st], use & 1) && globaltimer() - t0 < lim) {
                     }
             }
         }
@@ -154,8 +160,8 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
             const uint32_t idesc = instr_desc(WM, NT);
             for (int i = 0; i < nkl; ++i) {
                 const int st = i % STAGES, use = i / STAGES;
-                if (!mbar_wait(&sm.full_x[st], use & 1, abort_flag)) break;
-                if (!mbar_wait(&sm.full_w[st], use & 1, abort_flag)) break;
+                if (!mbar_wait(&sm.full_x[st], use & 1, abort_flag, lim)) break;
+                if (!mbar_wait(&sm.full_w[st], use & 1, abort_flag, lim)) break;
                 tc_fence_after();
                 const uint32_t a0 = s32(sm.w[st]), b0 = s32(sm.x[st]);
 #pragma unroll
@@ -190,14 +196,14 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
             const int ql = p.B - 1 - q_lo;  // the group's last byte relative to q_lo
             uint32_t bytes[14], lastb = 0;
             if (CODES_TMA) {
-                if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag)) break;
+                if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag, lim)) break;
                 const int off = (g * p.B + q_lo) & 15;
                 const uint8_t* win = sm.c[st] + t * C_ROW;
                 window_bytes(win, off, bytes);
                 if (ql < 14) lastb = win[off + ql];
             } else {
                 if (i + 1 < nkl) load_global(kb + 1, nxt);  // next stage's bytes in flight
-                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
+                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
 #pragma unroll
                 for (int j = 0; j < 14; ++j) bytes[j] = cur[j];
                 if (ql < 14) lastb = __ldg(crow + (int64_t)g * p.B + p.B - 1);
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
     if (warp >= kDecodeWarp0) {
         const int q = warp - kDecodeWarp0;
         const int r = 32 * q + lane;  // W row of the tile = TMEM lane
-        const bool ok = mbar_wait(&sm.done, 0, abort_flag);
+        const bool ok = mbar_wait(&sm.done, 0, abort_flag, lim);
         tc_fence_after();
         uint32_t v[NT];
         if (NT == 16) {
@@ -232,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
                 tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 32u * h, v32);
             }
         }
-        if (!ok) {
+        if (!ok || *abort_flag) {  // a wait gave up: the partial is not defined
 #pragma unroll
             for (int j = 0; j < NT; ++j) v[j] = 0x7FC00000u;
         }
@@ -270,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
     __syncthreads();
     if (warp == 1 && lane == 0 && *abort_flag) {
         const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(&sm.done, 0) && globaltimer() - t0 < kTimeoutNs) {
+        while (!mbar_try_wait(&sm.done, 0) && globaltimer() - t0 < lim) {
         }
     }
     __syncthreads();
@@ -285,12 +291,8 @@ static cudaError_t launch_nt(const CUtensorMap& tx, const CUtensorMap& tc_, cons
                              cudaStream_t stream) {
     auto kern = gemm_small_kernel<NT, CT>;
     const size_t smem = sizeof(Smem<NT>) + 1024;
-    static std::atomic<int> smem_set{0};
-    if ((int)smem > smem_set.load()) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        smem_set.store((int)smem);
-    }
+    static SmemAttr smem_attr;
+    if (cudaError_t e = smem_attr.ensure(kern, (int)smem)) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(tiles * p.CS));
     cfg.blockDim = dim3(kThreads);
@@ -347,6 +349,7 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     if (CS == 1)  // no K split: the persistent kernel walks the tiles
         return launch_gemm_stream(X, M, codes, scales, N, K, G, Y, y_bf16, d_err, stream, sm_count, handled);
     Params p{};
+    p.wc = tc::wait_cfg_from_env();
     p.codes = codes;
     p.row_bytes = row_bytes;
     p.scales = scales;

@@ -66,6 +66,7 @@ struct Params {
     int tiles;
     int y_bf16;
     uint32_t pad_base, pad_span;  // canonical range of a group's last code byte
+    WaitCfg wc;                   // wait bound and the withheld-load test hook
 };
 
 __device__ __forceinline__ void cp_async16(uint8_t* dst, const uint8_t* src) {
@@ -116,6 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     const int total = my_tiles * nk;  // stages of this CTA
     constexpr uint32_t kCols = 2 * NT < 32 ? 32 : 2 * NT;
     volatile int* abort_flag = &sm.abort_flag;
+    const uint64_t lim = p.wc.limit_ns;
 
     // Dependent launches may start now: only the X loads below wait for the
     // preceding kernel (codes and scales are weights, see tq_gemv's ordering
@@ -154,16 +156,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
             int issued = 0;
             for (int i = 0; i < total; ++i) {
                 const int kb = i % nk, st = i % STAGES, use = i / STAGES;
-                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&sm.full_x[st], NT * 128);
-                tma_load_2d(sm.x[st], &tmap_x, kb * BK, 0, &sm.full_x[st]);
+                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
+                if (!(p.wc.withhold_x && i == 0)) {  // test hook: the first load left out
+                    mbar_arrive_expect_tx(&sm.full_x[st], NT * 128);
+                    tma_load_2d(sm.x[st], &tmap_x, kb * BK, 0, &sm.full_x[st]);
+                }
                 ++issued;
             }
             // loads still in flight after an abort must land before the CTA exits
             for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
                 const int st = i % STAGES, use = i / STAGES;
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(&sm.full_x[st], use & 1) && globaltimer() - t0 < kTimeoutNs) {
+                while (!mbar_try_wait(&sm.full_x[st], use & 1) && globaltimer() - t0 < lim) {
                 }
             }
         }
@@ -174,13 +178,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
             bool ok = true;
             for (int j = 0; j < my_tiles && ok; ++j) {
                 const int buf = j & 1;
-                if (j >= 2 && !mbar_wait(&sm.tempty[buf], ((j >> 1) - 1) & 1, abort_flag)) break;
+                if (j >= 2 && !mbar_wait(&sm.tempty[buf], ((j >> 1) - 1) & 1, abort_flag, lim)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + (uint32_t)(buf * NT);
                 for (int kb = 0; kb < nk; ++kb, ++i) {
                     const int st = i % STAGES, use = i / STAGES;
-                    if (!mbar_wait(&sm.full_x[st], use & 1, abort_flag) ||
-                        !mbar_wait(&sm.full_w[st], use & 1, abort_flag)) {
+                    if (!mbar_wait(&sm.full_x[st], use & 1, abort_flag, lim) ||
+                        !mbar_wait(&sm.full_w[st], use & 1, abort_flag, lim)) {
                         ok = false;
                         break;
                     }
@@ -242,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
             issue(s + CR - 1);  // its slot held own stage s - 1, decoded already
             asm volatile("cp.async.wait_group %0;" ::"n"(CR - 1) : "memory");
             const int i = grp + 2 * s, st = i % STAGES, use = i / STAGES;
-            if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
+            if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
             const int64_t n = row_of(pd);
             const int c0 = BK * pd.sub, q_lo = c0 / 5;
             const uintptr_t A = reinterpret_cast<uintptr_t>(p.codes + n * p.row_bytes + (int64_t)pd.g * p.B + q_lo);
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
         uint32_t err_acc = 0;
         for (int j = 0; j < my_tiles; ++j) {
             const int buf = j & 1;
-            if (!mbar_wait(&sm.tfull[buf], (j >> 1) & 1, abort_flag)) break;
+            if (!mbar_wait(&sm.tfull[buf], (j >> 1) & 1, abort_flag, lim)) break;
             tc_fence_after();
             uint32_t v[NT];
             const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * NT);
@@ -302,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     __syncthreads();
     if (warp == 1 && lane == 0 && *abort_flag) {
         const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(&sm.done, 0) && globaltimer() - t0 < kTimeoutNs) {
+        while (!mbar_try_wait(&sm.done, 0) && globaltimer() - t0 < lim) {
         }
     }
     __syncthreads();
@@ -316,12 +320,8 @@ template <int NT>
 static cudaError_t launch_nt(const CUtensorMap& tx, const Params& p, int grid, cudaStream_t stream) {
     auto kern = gemm_stream_kernel<NT>;
     const size_t smem = sizeof(Smem<NT>) + 1024;
-    static std::atomic<int> smem_set{0};
-    if ((int)smem > smem_set.load()) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        smem_set.store((int)smem);
-    }
+    static SmemAttr smem_attr;
+    if (cudaError_t e = smem_attr.ensure(kern, (int)smem)) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
@@ -354,6 +354,7 @@ cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* code
                         (uint64_t)K * 2, BK, (uint32_t)NT, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     Params p{};
+    p.wc = tc::wait_cfg_from_env();
     p.row_bytes = (K / G) * B;
     p.codes = codes;
     p.codes_end = codes + N * p.row_bytes;

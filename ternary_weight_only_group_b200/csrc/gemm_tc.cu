@@ -74,6 +74,7 @@ struct Params {
     int n_tiles;
     int y_bf16;
     uint32_t pad_base, pad_span;  // canonical range of a group's last code byte
+    WaitCfg wc;                   // wait bound and the withheld-load test hook
     int y_vec;  // Y rows allow 16-byte vector stores (base aligned, N a multiple of 16 bytes)
 };
 
@@ -90,6 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int64_t m0 = (int64_t)m_tile * BM, n0 = (int64_t)n_tile * TBN;
     const int nk = p.K / BK;
     volatile int* abort_flag = &sm.abort_flag;
+    const uint64_t lim = p.wc.limit_ns;
 
     fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
@@ -129,10 +131,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         if (lane == 0) {
             for (int kb = 0; kb < nk; ++kb) {
                 const int st = kb % STAGES, use = kb / STAGES;
-                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&sm.full_a[st], 2 * A_SUB);
-                tma_load_2d(sm.a[st][0], &tmap_x, kb * BK, (int)m0, &sm.full_a[st]);
-                tma_load_2d(sm.a[st][1], &tmap_x, kb * BK, (int)(m0 + UM), &sm.full_a[st]);
+                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
+                if (!(p.wc.withhold_x && kb == 0)) {  // test hook: the first load left out
+                    mbar_arrive_expect_tx(&sm.full_a[st], 2 * A_SUB);
+                    tma_load_2d(sm.a[st][0], &tmap_x, kb * BK, (int)m0, &sm.full_a[st]);
+                    tma_load_2d(sm.a[st][1], &tmap_x, kb * BK, (int)(m0 + UM), &sm.full_a[st]);
+                }
                 if (CODES_TMA) {
                     int g, c0, q_lo;
                     stage_geom(kb, g, c0, q_lo);
@@ -146,10 +150,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb) {
                 const int st = kb % STAGES, use = kb / STAGES;
                 const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(&sm.full_a[st], use & 1) && globaltimer() - t0 < kTimeoutNs) {
+                while (!mbar_try_wait(&sm.full_a[st], use & 1) && globaltimer() - t0 < lim) {
                 }
                 if (CODES_TMA)
-                    while (!mbar_try_wait(&sm.full_c[st], use & 1) && globaltimer() - t0 < kTimeoutNs) {
+                    while (!mbar_try_wait(&sm.full_c[st], use & 1) && globaltimer() - t0 < lim) {
                     }
             }
         }
@@ -159,8 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             const uint32_t idesc = instr_desc(UM, TBN);
             for (int kb = 0; kb < nk; ++kb) {
                 const int st = kb % STAGES, use = kb / STAGES;
-                if (!mbar_wait(&sm.full_a[st], use & 1, abort_flag)) break;
-                if (!mbar_wait(&sm.full_b[st], use & 1, abort_flag)) break;
+                if (!mbar_wait(&sm.full_a[st], use & 1, abort_flag, lim)) break;
+                if (!mbar_wait(&sm.full_b[st], use & 1, abort_flag, lim)) break;
                 tc_fence_after();
                 const uint32_t b0 = s32(sm.b[st]);
 #pragma unroll
@@ -201,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             const int ql = p.B - 1 - q_lo;  // the group's last byte relative to q_lo
             uint32_t bytes[14], lastb = 0;
             if (CODES_TMA) {
-                if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag)) break;
+                if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag, lim)) break;
                 const int gb = g * p.B + q_lo;
                 const uint8_t* win = sm.c[st] + t * C_ROW;
                 window_bytes(win, gb & 15, bytes);
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
                 for (int i = 0; i < 14; ++i) bytes[i] = nxt[i];
                 if (kb + 1 < nk) load_global(kb + 1, nxt);  // next stage's bytes in flight
-                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag)) break;
+                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
                 if (ql < 14) lastb = __ldg(crow + (int64_t)g * p.B + p.B - 1);
             }
             if (t < TBN)
@@ -224,9 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         if (warp < kDecodeWarp0 + 4) {
             const int q = warp - kDecodeWarp0;  // TMEM lanes 32q .. 32q+31
             uint32_t err_acc = 0;
-            const bool ok = mbar_wait(&sm.done, 0, abort_flag);
+            const bool ok = mbar_wait(&sm.done, 0, abort_flag, lim);
             tc_fence_after();
-            if (ok) {
+            if (ok && !*abort_flag) {  // after a wait gave up, Y is left as it was
                 for (int sub = 0; sub < 2; ++sub) {
                     const int64_t m = m0 + sub * UM + 32 * q + lane;
                     for (int c = 0; c < TBN / 32; ++c) {
@@ -291,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         // The commit after the issue loop tracks every MMA this CTA issued:
         // wait for it (bounded) before tensor memory is freed.
         const uint64_t t0 = globaltimer();
-        while (!mbar_try_wait(&sm.done, 0) && globaltimer() - t0 < kTimeoutNs) {
+        while (!mbar_try_wait(&sm.done, 0) && globaltimer() - t0 < lim) {
         }
     }
     __syncthreads();
@@ -369,6 +373,7 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
                                      CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     Params p{};
+    p.wc = tc::wait_cfg_from_env();
     p.codes = codes;
     p.scales = scales;
     p.Y = Y;
@@ -389,13 +394,8 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
     const size_t smem = gemm_smem_bytes();
     auto kern = codes_tma ? (tbn == 224 ? gemm_tc_kernel<true, 224> : gemm_tc_kernel<true, 256>)
                           : (tbn == 224 ? gemm_tc_kernel<false, 224> : gemm_tc_kernel<false, 256>);
-    static std::atomic<int> smem_set[4];
-    std::atomic<int>& slot = smem_set[(codes_tma ? 2 : 0) + (tbn == 224 ? 1 : 0)];
-    if ((int)smem > slot.load()) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        slot.store((int)smem);
-    }
+    static SmemAttr smem_attr[4];
+    if (cudaError_t e = smem_attr[(codes_tma ? 2 : 0) + (tbn == 224 ? 1 : 0)].ensure(kern, (int)smem)) return e;
     kern<<<(unsigned)grid, kThreads, smem, stream>>>(tmap_x, tmap_c, p);
     *handled = true;
     return cudaGetLastError();

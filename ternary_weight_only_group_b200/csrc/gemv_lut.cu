@@ -207,6 +207,7 @@ __global__ void __launch_bounds__(kLutThreads, 512 / kLutThreads) gemv_lut_kerne
     const uint32_t ssc_s = smem_u32(ssc);
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    cluster_arrive_relaxed();  // waited on before the first store into a peer's shared memory
 
     for (int pass = 0; pass < p.P; ++pass) {
         const int gg0 = (crank * p.P + pass) * ngl;  // first group of this pass
@@ -322,6 +323,7 @@ __global__ void __launch_bounds__(kLutThreads, 512 / kLutThreads) gemv_lut_kerne
             if (lane_on) build_part<B>(a, tab, sl, m, j, gg0, part);
         }
         __syncthreads();
+        if (pass == 0) cluster_wait();  // every CTA of the cluster is running: partial rows may be pushed
 
         int bt = warp;
         while (bt < nbatch) {
@@ -436,12 +438,8 @@ static bool make_plan(int64_t N, int K, int G, int MT, int sm_count, size_t smem
 template <int B, int MT, int NS, int T>
 static cudaError_t launch_lut(const LutArgs& a, cudaStream_t stream) {
     auto kern = gemv_lut_kernel<B, MT, NS, T>;
-    static std::atomic<int> smem_set{0};
-    if ((int)a.p.smem > smem_set.load()) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)a.p.smem);
-        if (e != cudaSuccess) return e;
-        smem_set.store((int)a.p.smem);
-    }
+    static SmemAttr smem_attr;
+    if (cudaError_t e = smem_attr.ensure(kern, (int)a.p.smem)) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.p.RB * a.p.CS));
     cfg.blockDim = dim3(T);

@@ -1,0 +1,500 @@
+// gemv_lut_stream.cu -- one-token decode GEMV over large matrices at HBM rate
+// (CUDA cores, sm_100a).
+//
+// Computes Y[n] = sum_g RNE_bf16(s[n,g]) * sum_{j in g} t[n,j] X[j] (tiny-llm
+// "Week 2 Day 3: Quantize the Model", "Mathematical Formulation", bias 0, the
+// group scale applied once per group as in "Stage 2: SIMD Matvec") for the
+// base-3 codes of "precisit/pack-unpack-run" (codec.py: five digits per byte,
+// each group byte-aligned) with G = 64 or 128, M = 1, fp32 accumulation.
+//
+// Lookup tables.  A code byte b covers five activations x_0..x_4 of its group;
+// the table of its chunk holds the 243 sums sum_i (d_i(b) - 1) x_i (NaN for
+// the 13 invalid byte values and for padding digits other than 1), so one
+// byte costs a table load and an add.  512 columns are 104 code bytes at both
+// group sizes; a CTA keeps the tables of one such K slice, and the K slices
+// of a row are spread over the CTAs of a thread-block cluster whose partial
+// rows are added in rank order through distributed shared memory.
+//
+// Table layout.  Entry b of a table sits at byte 256 b + 4 slot of its block
+// (64 slots of fp32 per entry row, 64 KB per block, two blocks at absolute
+// shared address 0x10000), so slot s lives in bank s mod 32 whatever b is.
+// A PRMT builds the whole lookup address in one instruction: it places the
+// code byte in bits 8..15 and the lane's slot offset (4 x bank, from a
+// per-lane constant register) in bits 0..7; the block and the upper half of
+// the slots come from the load's immediate offset.
+//
+// Lanes.  Each lane reads one code word of a row's K slice with a single
+// global load and owns the bytes of ONE group in it, so one scale per lane
+// and row suffices: words that straddle a group boundary are read by two
+// lanes, each of which masks the other group's bytes by pointing their
+// lookups at an all-zero table column.
+//   G = 128: 8-byte words, 13 words + 3 straddling copies = 16 lanes per
+//            row, two rows per warp step; the second row's lanes take their
+//            bytes in the order 4..7, 0..3 so that the 32 lookups of an
+//            instruction hit 32 different banks.
+//   G = 64:  4-byte words, 26 words + 6 straddling copies = 32 lanes, one
+//            row per warp step.
+// A warp handles 32 rows per chunk (16 or 32 steps); its per-row partials
+// are summed across lanes by a transposing butterfly.  Code words are
+// requested U steps ahead (ld.global.nc, no L1 allocation).
+//
+// Codes and scales do not depend on earlier kernels: the first steps' loads
+// are issued before griddepcontrol.wait; the activations (and therefore the
+// tables) only after it.  A NaN output row (invalid byte, bad padding, bad
+// scale) is rescanned for its error bits.
+#include <cooperative_groups.h>
+
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "tq_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace tq {
+
+namespace {
+
+constexpr int kLsThreads = 512;
+constexpr int kLsWarps = kLsThreads / 32;
+constexpr uint32_t kLsTableAbs = 0x10000u;   // absolute shared address of the tables
+constexpr uint32_t kLsBlockBytes = 0x10000u; // one block: 256 entry rows x 64 slots x 4 B
+constexpr uint32_t kLsSmemBytes = 0x30000u;  // dynamic request: covers [base, 0x30000) for any base <= 0x10000
+constexpr int kLsSliceCols = 512;            // K columns per CTA
+constexpr int kLsSliceBytes = 104;           // their code bytes (G = 64 or 128)
+constexpr int kLsRound = 6144;               // rows per cluster round (partials in shared memory)
+constexpr int kLsFreeBank = 26;              // banks 26..31: all-zero columns for masked lookups
+constexpr int kLsChunkRows = 32;             // rows per warp chunk
+
+template <int G>
+struct LsCfg;
+template <>
+struct LsCfg<128> {
+    static constexpr int B = 26;    // code bytes per group
+    static constexpr int GPS = 4;   // groups per slice
+    static constexpr int RPS = 2;   // rows per warp step
+    static constexpr int SPC = 16;  // steps per chunk
+    static constexpr int U = 8;     // steps of code loads in flight
+};
+template <>
+struct LsCfg<64> {
+    static constexpr int B = 13;
+    static constexpr int GPS = 8;
+    static constexpr int RPS = 1;
+    static constexpr int SPC = 32;
+    static constexpr int U = 16;
+};
+
+// shared memory below the tables: per-warp decoded scales, then the partial rows
+template <int G>
+__host__ __device__ constexpr uint32_t ls_scale_bytes() {
+    return (uint32_t)kLsWarps * kLsChunkRows * LsCfg<G>::GPS * 4;
+}
+template <int G>
+__host__ __device__ constexpr uint32_t ls_misc_bytes() {
+    return ls_scale_bytes<G>() + (uint32_t)kLsRound * 4;
+}
+
+struct LsArgs {
+    const uint16_t* X;
+    const uint8_t* codes;
+    const uint16_t* scales;
+    int64_t N;
+    int K, ng, CS;
+    int64_t row_bytes;
+    int64_t rows_per_cluster;
+    void* Y;
+    int y_bf16;
+    uint32_t* d_err;
+};
+
+// Table slot of chunk position p of a slice (0 <= p < 104), as the lanes below
+// read it: G = 128: p = 8 w + j -> block (j & 3) >> 1, upper slots j & 1, bank
+// 2 w + (j >> 2); G = 64: p = 4 w + j -> block j >> 1, upper slots j & 1,
+// bank w.  The table build needs the inverse: the position held at (block,
+// sub, bank < 26).
+template <int G>
+__device__ __forceinline__ int ls_slot_position(int block, int sub, int bank) {
+    if constexpr (G == 128) return 8 * (bank >> 1) + 4 * (bank & 1) + 2 * block + sub;
+    else return 4 * bank + 2 * block + sub;
+}
+
+// Per-lane constants: offset of the lane's word in the slice, the row within
+// the step, the lane's group in the slice and the slot offsets (4 x bank) of
+// its lookups, one byte per step (lb0: steps 0..3, lb1: steps 4..7).
+struct LsLane {
+    uint32_t wofs;
+    int h, grp;
+    uint32_t lb0, lb1;
+};
+
+template <int G>
+__device__ __forceinline__ LsLane ls_lane(int lane) {
+    LsLane L{};
+    if constexpr (G == 128) {
+        const int h = lane >> 4, q = lane & 15;
+        const int w = q < 13 ? q : 3 * (q - 12);  // copies of the straddling words 3, 6, 9
+        const bool copy = q >= 13;
+        const int si = (w == 3 || w == 6 || w == 9) ? w / 3 - 1 : 0;
+        const int grp = copy ? (8 * w + 7) / 26 : (8 * w) / 26;
+        uint32_t lb[2] = {0u, 0u};
+        for (int k = 0; k < 8; ++k) {
+            const int j = h ? ((k + 4) & 7) : k;
+            const bool live = (8 * w + j) / 26 == grp;
+            const int bank = live ? 2 * w + (j >> 2) : kLsFreeBank + 2 * si + h;
+            lb[k >> 2] |= (uint32_t)(4 * bank) << (8 * (k & 3));
+        }
+        L.wofs = 8u * w;
+        L.h = h;
+        L.grp = grp;
+        L.lb0 = lb[0];
+        L.lb1 = lb[1];
+    } else {
+        // straddling words 3, 6, 9, 16, 19, 22 (copy i = lane - 26)
+        const bool copy = lane >= 26;
+        const int w = copy ? (lane < 29 ? 3 * (lane - 25) : 3 * (lane - 26) + 7) : lane;
+        const int si = w <= 9 ? w / 3 - 1 : (w - 7) / 3;
+        const int grp = copy ? (4 * w + 3) / 13 : (4 * w) / 13;
+        uint32_t lb = 0;
+        for (int k = 0; k < 4; ++k) {
+            const bool live = (4 * w + k) / 13 == grp;
+            const int bank = live ? w : kLsFreeBank + si;
+            lb |= (uint32_t)(4 * bank) << (8 * k);
+        }
+        L.wofs = 4u * w;
+        L.h = 0;
+        L.grp = grp;
+        L.lb0 = lb;
+        L.lb1 = 0;
+    }
+    return L;
+}
+
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+template <uint32_t IMM>
+__device__ __forceinline__ float lds_imm(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(IMM));
+    return v;
+}
+__device__ __forceinline__ uint2 ldg_nc_u2(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// Decoded scale as the matmul uses it: fp32 of RNE_bf16(binary16 s); NaN for
+// a rejected scale (sign bit set, Inf or NaN: every pattern >= 0x7C00).
+__device__ __forceinline__ float ls_scale(uint32_t s) {
+    const float r = __bfloat162float(__float2bfloat16_rn(__half2float(__ushort_as_half((unsigned short)s))));
+    return s >= 0x7C00u ? __uint_as_float(0x7FC00000u) : r;
+}
+
+// Transposing butterfly within aligned groups of NV lanes (NV = 16 or 32):
+// on exit lane l holds the sum over its group of v[l mod NV].
+template <int NV>
+__device__ __forceinline__ float ls_transpose_reduce(float (&v)[NV], int lane) {
+#pragma unroll
+    for (int n = NV / 2; n >= 1; n >>= 1) {
+        const bool upper = (lane & n) != 0;
+#pragma unroll
+        for (int i = 0; i < n; ++i) {
+            const float keep = upper ? v[n + i] : v[i];
+            const float send = upper ? v[i] : v[n + i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, n);
+        }
+    }
+    return v[0];
+}
+
+// One lookup: byte k of word `a` plus the slot byte k of `lb`, at the
+// immediate offset of block / upper slots.
+template <int G, int K>
+__device__ __forceinline__ float ls_lookup(uint32_t a, uint32_t lb) {
+    constexpr uint32_t kk = (uint32_t)(K & 3);
+    constexpr uint32_t sel = 0xCC00u | (kk << 4) | (4u + kk);
+    constexpr uint32_t block = G == 128 ? (uint32_t)((K & 3) >> 1) : (uint32_t)(K >> 1);
+    constexpr uint32_t imm = kLsTableAbs + block * kLsBlockBytes + 128u * (uint32_t)(K & 1);
+    return lds_imm<imm>(prmt32(a, lb, sel));
+}
+
+template <int G>
+__global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const LsArgs a) {
+    using C = LsCfg<G>;
+    constexpr int SPC = C::SPC, U = C::U, RPS = C::RPS, GPS = C::GPS;
+    using Word = typename std::conditional<G == 128, uint2, uint32_t>::type;
+    extern __shared__ __align__(16) unsigned char smem[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int crank = (int)cluster.block_rank();
+    const int cid = (int)(blockIdx.x / (unsigned)a.CS);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // Shared-memory window: the tables at [0x10000, 0x30000), the scales and
+    // partials just below 0x10000.
+    const uint32_t dyn = (uint32_t)__cvta_generic_to_shared(smem);
+    const uint32_t misc = kLsTableAbs - ls_misc_bytes<G>();
+    if (dyn > misc) {  // cannot happen with no static shared memory; fail closed
+        if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
+        return;
+    }
+    float* ssc_all = reinterpret_cast<float*>(smem + (misc - dyn));
+    float* part = reinterpret_cast<float*>(smem + (misc - dyn) + ls_scale_bytes<G>());
+    float* ssc = ssc_all + warp * kLsChunkRows * GPS;
+
+    const LsLane L = ls_lane<G>(lane);
+    const int64_t crow0 = (int64_t)cid * a.rows_per_cluster;
+    const int64_t crow1 = min(a.N, crow0 + a.rows_per_cluster);
+    const uint8_t* cbase = a.codes + (int64_t)crank * kLsSliceBytes + L.wofs;
+    const uint16_t* sbase = a.scales + (int64_t)crank * GPS;
+    const uint32_t ssc_lane = (uint32_t)__cvta_generic_to_shared(ssc) + 4u * (uint32_t)(L.h * GPS + L.grp);
+    uint32_t err_acc = 0;
+    bool tables_built = false;
+
+    for (int64_t rr0 = crow0; rr0 < crow1; rr0 += kLsRound) {
+        const int nround = (int)(crow1 - rr0 < (int64_t)kLsRound ? crow1 - rr0 : (int64_t)kLsRound);
+        // this warp's rows of the round
+        int per = (nround + kLsWarps - 1) / kLsWarps;
+        per = (per + RPS - 1) / RPS * RPS;
+        const int wlo = min(nround, warp * per), whi = min(nround, wlo + per);
+        const int nr = whi - wlo;
+        const int64_t wr0 = rr0 + wlo;
+        const int T = (nr + RPS - 1) / RPS;
+        const int nch = (T + SPC - 1) / SPC;
+
+        auto code_ptr = [&](int t) -> const uint8_t* {
+            int r = RPS * t + L.h;
+            r = r < nr ? r : nr - 1;
+            return cbase + (wr0 + r) * a.row_bytes;
+        };
+        auto load_code = [&](int t) -> Word {
+            if constexpr (G == 128) return ldg_nc_u2(code_ptr(t));
+            else return ldg_nc_u32(code_ptr(t));
+        };
+        using SRaw = typename std::conditional<G == 128, uint2, uint4>::type;
+        auto load_scales = [&](int ch) -> SRaw {
+            int r = ch * kLsChunkRows + lane;
+            r = r < nr ? r : nr - 1;
+            const uint16_t* p = sbase + (wr0 + r) * a.ng;
+            if constexpr (G == 128) return __ldg(reinterpret_cast<const uint2*>(p));
+            else return __ldg(reinterpret_cast<const uint4*>(p));
+        };
+
+        Word cb[U];
+        SRaw sraw{};
+        if (nr > 0) {
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (u < T) cb[u] = load_code(u);
+            sraw = load_scales(0);
+        }
+
+        if (!tables_built) {
+            // Activations come from the preceding kernel: everything above ran
+            // before this wait.
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            const int col_base = crank * kLsSliceCols;
+            const float nan = __uint_as_float(0x7FC00000u);
+            // warp item (block, sub, d3 + 3 d4): the 27 entries b = d0 + 3 d1 + 9 d2 + 27 (d3 + 3 d4)
+            // of one table row per lane (lane = bank)
+            for (int it = warp; it < 36; it += kLsWarps) {
+                const int bs = it / 9, d34 = it - 9 * bs;
+                const int block = bs >> 1, sub = bs & 1;
+                const uint32_t base = kLsTableAbs + block * kLsBlockBytes + 27u * d34 * 256u +
+                                      4u * (uint32_t)(lane + 32 * sub);
+                if (lane >= kLsFreeBank) {
+#pragma unroll
+                    for (int e = 0; e < 27; ++e) sts_f32(base + 256u * e, 0.f);
+                    continue;
+                }
+                const int p = ls_slot_position<G>(block, sub, lane);
+                const int g = p / C::B, j = p - g * C::B;
+                const int real = min(5, G - 5 * j);
+                const uint16_t* xp = a.X + col_base + g * G + 5 * j;
+                float x[5];
+#pragma unroll
+                for (int i = 0; i < 5; ++i) x[i] = i < real ? __uint_as_float((uint32_t)__ldcg(xp + i) << 16) : 0.f;
+                const int d3 = d34 % 3, d4 = d34 / 3;
+                const bool bad34 = (3 >= real && d3 != 1) || (4 >= real && d4 != 1);
+                const float h34 = bad34 ? nan : (float)(d3 - 1) * x[3] + (float)(d4 - 1) * x[4];
+                float P[9];
+#pragma unroll
+                for (int d1 = 0; d1 < 3; ++d1)
+#pragma unroll
+                    for (int d0 = 0; d0 < 3; ++d0) {
+                        const bool bad = (1 >= real && d1 != 1) || (0 >= real && d0 != 1);
+                        P[d0 + 3 * d1] = bad ? nan : (float)(d0 - 1) * x[0] + (float)(d1 - 1) * x[1];
+                    }
+#pragma unroll
+                for (int d2 = 0; d2 < 3; ++d2) {
+                    const bool bad2 = 2 >= real && d2 != 1;
+                    const float q2 = bad2 ? nan : h34 + (float)(d2 - 1) * x[2];
+#pragma unroll
+                    for (int e = 0; e < 9; ++e) sts_f32(base + 256u * (9 * d2 + e), P[e] + q2);
+                }
+            }
+            // entry rows 243..255: NaN (invalid bytes) in table columns, 0 in the free ones
+            for (int it = warp; it < 4; it += kLsWarps) {
+                const int block = it >> 1, sub = it & 1;
+                const uint32_t base = kLsTableAbs + block * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * sub);
+                const float v = lane < kLsFreeBank ? nan : 0.f;
+#pragma unroll
+                for (int b = 243; b < 256; ++b) sts_f32(base + 256u * b, v);
+            }
+            __syncthreads();
+            tables_built = true;
+        }
+
+        for (int ch = 0; ch < nch; ++ch) {
+            // decoded scales of this chunk's 32 rows: lane = row
+            {
+                const uint32_t* sw = reinterpret_cast<const uint32_t*>(&sraw);
+                float4* dst = reinterpret_cast<float4*>(ssc + lane * GPS);
+#pragma unroll
+                for (int q = 0; q < GPS / 4; ++q)
+                    dst[q] = make_float4(ls_scale(sw[2 * q] & 0xFFFFu), ls_scale(sw[2 * q] >> 16),
+                                         ls_scale(sw[2 * q + 1] & 0xFFFFu), ls_scale(sw[2 * q + 1] >> 16));
+                if (ch + 1 < nch) sraw = load_scales(ch + 1);
+                __syncwarp();
+            }
+            float v[SPC];
+#pragma unroll
+            for (int s = 0; s < SPC; ++s) {
+                const int t = ch * SPC + s;
+                const Word cw = cb[s % U];
+                if (t + U < T) cb[s % U] = load_code(t + U);
+                if (t < T) {
+                    float sc;
+                    asm volatile("ld.shared.f32 %0, [%1];"
+                                 : "=f"(sc)
+                                 : "r"(ssc_lane + 4u * (uint32_t)(RPS * s * GPS)));
+                    if constexpr (G == 128) {
+                        const uint32_t w0 = L.h ? cw.y : cw.x;
+                        const uint32_t w1 = L.h ? cw.x : cw.y;
+                        const float t0 = ls_lookup<G, 0>(w0, L.lb0);
+                        const float t1 = ls_lookup<G, 1>(w0, L.lb0);
+                        const float t2 = ls_lookup<G, 2>(w0, L.lb0);
+                        const float t3 = ls_lookup<G, 3>(w0, L.lb0);
+                        const float t4 = ls_lookup<G, 4>(w1, L.lb1);
+                        const float t5 = ls_lookup<G, 5>(w1, L.lb1);
+                        const float t6 = ls_lookup<G, 6>(w1, L.lb1);
+                        const float t7 = ls_lookup<G, 7>(w1, L.lb1);
+                        v[s] = (((t0 + t1) + (t2 + t3)) + ((t4 + t5) + (t6 + t7))) * sc;
+                    } else {
+                        const float t0 = ls_lookup<G, 0>(cw, L.lb0);
+                        const float t1 = ls_lookup<G, 1>(cw, L.lb0);
+                        const float t2 = ls_lookup<G, 2>(cw, L.lb0);
+                        const float t3 = ls_lookup<G, 3>(cw, L.lb0);
+                        v[s] = ((t0 + t1) + (t2 + t3)) * sc;
+                    }
+                } else {
+                    v[s] = 0.f;
+                }
+            }
+            __syncwarp();  // this chunk's scales are consumed before the next chunk rewrites them
+            const float tot = ls_transpose_reduce<SPC>(v, lane);
+            const int r = ch * kLsChunkRows + (G == 128 ? 2 * (lane & 15) + (lane >> 4) : lane);
+            if (r < nr) part[wlo + r] = tot;
+        }
+
+        // K slices: every rank's partial rows are complete and visible, then
+        // rank q adds the ranks' partials of its share of rows in rank order.
+        __syncthreads();
+        cluster.sync();
+        const int share = (nround + a.CS - 1) / a.CS;
+        const int lo = min(nround, crank * share), hi = min(nround, lo + share);
+        for (int r = lo + (int)threadIdx.x; r < hi; r += kLsThreads) {
+            float y = 0.f;
+            for (int q = 0; q < a.CS; ++q) y += *cluster.map_shared_rank(part + r, q);
+            const int64_t n = rr0 + r;
+            if (y != y)
+                err_acc |= scan_row_errors(a.codes + n * a.row_bytes, a.scales + n * a.ng, a.ng, G, C::B);
+            if (a.y_bf16) reinterpret_cast<__nv_bfloat16*>(a.Y)[n] = __float2bfloat16_rn(y);
+            else reinterpret_cast<float*>(a.Y)[n] = y;
+        }
+        cluster.sync();  // the peers are done reading this CTA's partials
+    }
+    if (!tables_built) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (err_acc && a.d_err) atomicOr(a.d_err, err_acc);
+}
+
+template <int G>
+cudaError_t launch_ls(const LsArgs& a0, cudaStream_t stream, int sm_count) {
+    auto kern = gemv_lut_stream_kernel<G>;
+    static SmemAttr smem_attr;
+    static int max_clusters[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+    static std::mutex mu;
+    if (cudaError_t e = smem_attr.ensure(kern, (int)kLsSmemBytes)) return e;
+    LsArgs a = a0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kLsThreads);
+    cfg.dynamicSmemBytes = kLsSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = a.CS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    int ncl;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (max_clusters[a.CS] == 0) {
+            cfg.gridDim = dim3((unsigned)(a.CS * (sm_count / a.CS)));
+            int n = 0;
+            cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+            if (e != cudaSuccess) return e;
+            max_clusters[a.CS] = n > 0 ? n : 1;
+        }
+        ncl = max_clusters[a.CS];
+    }
+    const int64_t want = (a.N + 63) / 64;  // at least 64 rows per cluster
+    if (want < ncl) ncl = (int)(want < 1 ? 1 : want);
+    a.rows_per_cluster = (a.N + ncl - 1) / ncl;
+    cfg.gridDim = dim3((unsigned)(ncl * a.CS));
+    static const bool debug = getenv("TQ_DEBUG_PLAN") != nullptr;
+    if (debug)
+        fprintf(stderr, "tq gemv_lut_stream N=%lld K=%d G=%d: CS=%d clusters=%d rows/cluster=%lld\n",
+                (long long)a.N, a.K, G, a.CS, ncl, (long long)a.rows_per_cluster);
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+}  // namespace
+
+// Returns cudaErrorNotSupported when the shape is not covered: M != 1, G not
+// 64 or 128, K not a multiple of 512 or above 4096, or unaligned codes/scales.
+cudaError_t launch_gemv_lut_stream(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
+                                   int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
+                                   cudaStream_t stream, int sm_count) {
+    if (M != 1 || (G != 64 && G != 128) || K % kLsSliceCols != 0 || K > 8 * kLsSliceCols || N < 1)
+        return cudaErrorNotSupported;
+    const uintptr_t ca = reinterpret_cast<uintptr_t>(codes), sa = reinterpret_cast<uintptr_t>(scales);
+    if ((ca & (G == 128 ? 7 : 3)) || (sa & (G == 128 ? 7 : 15))) return cudaErrorNotSupported;
+    LsArgs a{};
+    a.X = X;
+    a.codes = codes;
+    a.scales = scales;
+    a.N = N;
+    a.K = (int)K;
+    a.ng = (int)(K / G);
+    a.CS = (int)(K / kLsSliceCols);
+    a.row_bytes = (int64_t)a.ng * bytes_per_group(G);
+    a.Y = Y;
+    a.y_bf16 = y_bf16;
+    a.d_err = d_err;
+    return G == 128 ? launch_ls<128>(a, stream, sm_count) : launch_ls<64>(a, stream, sm_count);
+}
+
+}  // namespace tq

@@ -342,12 +342,8 @@ static cudaError_t launch_pd(const uint16_t* X, int M, const uint8_t* codes, con
                              int K, int R, int grid, size_t smem, void* Y, int y_bf16, uint32_t* d_err,
                              cudaStream_t stream) {
     auto kern = gemv_predecode_kernel<G, MT>;
-    static std::atomic<int> smem_set{0};
-    if ((int)smem > smem_set.load()) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        smem_set.store((int)smem);
-    }
+    static SmemAttr smem_attr;
+    if (cudaError_t e = smem_attr.ensure(kern, (int)smem)) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kPdThreads);

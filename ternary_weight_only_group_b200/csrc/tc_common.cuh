@@ -6,12 +6,35 @@
 
 #include <cuda.h>
 
+#include <cstdlib>
+
 #include "tq_internal.cuh"
 
 namespace tq {
 namespace tc {
 
-constexpr uint64_t kTimeoutNs = 2000000000ull;  // bound of every mbarrier wait: 2 s
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // default bound of every mbarrier wait: 2 s
+
+// Bound of the kernels' mbarrier waits, and a test hook: with withhold_x set,
+// the TMA producer of every CTA leaves out its first activation load, so the
+// consumer waiting for it gives up after limit_ns (TQ_DERR_TIMEOUT) and the
+// whole CTA winds down through the abort path.  Read from the environment at
+// every launch (TQ_DEBUG_WAIT_LIMIT_NS, TQ_DEBUG_WITHHOLD_X_LOAD); unset, the
+// limit is 2 s and nothing is withheld.
+struct WaitCfg {
+    uint64_t limit_ns;
+    int withhold_x;
+};
+
+inline WaitCfg wait_cfg_from_env() {
+    WaitCfg w{kTimeoutNs, 0};
+    if (const char* e = getenv("TQ_DEBUG_WAIT_LIMIT_NS")) {
+        const unsigned long long v = strtoull(e, nullptr, 10);
+        if (v > 0 && v < kTimeoutNs) w.limit_ns = v;
+    }
+    if (const char* e = getenv("TQ_DEBUG_WITHHOLD_X_LOAD")) w.withhold_x = atoi(e) != 0;
+    return w;
+}
 
 __device__ __forceinline__ uint32_t s32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -39,15 +62,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: false when the deadline passed or another role gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// Bounded wait: false when the deadline (limit ns) passed or another role gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint64_t limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > kTimeoutNs) {
+            if (globaltimer() - t0 > limit) {
                 *abort_flag = 1;
                 return false;
             }

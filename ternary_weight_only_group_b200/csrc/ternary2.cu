@@ -300,12 +300,9 @@ cudaError_t launch_gemv2_t(const uint16_t* X, int M, const uint32_t* codes, cons
                            void* Y, int y_bf16, uint32_t* d_err, cudaStream_t stream, int sm_count) {
     auto kern = gemv2_kernel<MT, WPG>;
     const size_t smem = (size_t)MT * K * 2;
-    static std::atomic<int> smem_set{0};
-    if ((int)smem > 48 * 1024 && (int)smem > smem_set.load()) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        smem_set.store((int)smem);
-    }
+    static SmemAttr smem_attr;
+    if ((int)smem > 48 * 1024)
+        if (cudaError_t e = smem_attr.ensure(kern, (int)smem)) return e;
     constexpr int RB = MT <= 2 ? 4 : 2;
     const int64_t nbatch = (N + RB - 1) / RB;
     const int64_t want = (nbatch + kG2Warps - 1) / kG2Warps;

@@ -21,6 +21,12 @@ cudaError_t launch_gemv_rows(const uint16_t* X, int64_t M, const uint8_t* codes,
 cudaError_t launch_gemv_lut(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                             int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                             cudaStream_t stream, int sm_count, size_t smem_limit);
+cudaError_t launch_gemv_lut_stream(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
+                                   int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
+                                   cudaStream_t stream, int sm_count);
+cudaError_t launch_gemv_w4(const uint16_t* X, int64_t M, const uint32_t* codes, const uint16_t* scales,
+                           const uint16_t* biases, int64_t N, int64_t K, int G, void* Y, int y_bf16,
+                           cudaStream_t stream, int sm_count);
 cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                   int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                                   cudaStream_t stream, int sm_count);
@@ -129,6 +135,12 @@ tq_status check_matmul(const MatmulArgs& a) {
     return TQ_OK;
 }
 
+// Y for K == 0: every output is an empty sum, +0.
+tq_status zero_output(const MatmulArgs& a, cudaStream_t stream) {
+    const size_t yb = (size_t)a.M * (size_t)a.N * (a.yt == TQ_OUT_F32 ? 4 : 2);
+    return from_cuda(cudaMemsetAsync(a.Y, 0, yb, stream));
+}
+
 }  // namespace
 }  // namespace tq
 
@@ -191,7 +203,7 @@ tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* sc
     const MatmulArgs a{X, M, codes, scales, N, K, G, Y, yt};
     if (tq_status st = check_matmul(a)) return st;
     if (M == 0 || N == 0) return TQ_OK;
-    if (K == 0) return TQ_ERR_UNSUPPORTED;
+    if (K == 0) return zero_output(a, (cudaStream_t)stream);  // empty sums
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
     // 1..8 tokens, matrix small enough for one or two CTAs per SM to hold its
@@ -201,6 +213,14 @@ tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* sc
                                           d_err, (cudaStream_t)stream, d->sm_count);
     if (e != cudaErrorNotSupported) return from_cuda(e);
     cudaGetLastError();
+    // one token over a larger matrix: lookup tables of one 512-column K slice
+    // per CTA, slices spread over a cluster, code words streamed per lane
+    if (M == 1) {
+        e = launch_gemv_lut_stream(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
+                                   N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count);
+        if (e != cudaErrorNotSupported) return from_cuda(e);
+        cudaGetLastError();
+    }
     auto lut = [&]() {
         return launch_gemv_lut(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales), N,
                                K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, d->smem_optin);
@@ -241,7 +261,7 @@ tq_status tq_gemm(const void* X, int64_t M, const uint8_t* codes, const void* sc
     const MatmulArgs a{X, M, codes, scales, N, K, G, Y, yt};
     if (tq_status st = check_matmul(a)) return st;
     if (M == 0 || N == 0) return TQ_OK;
-    if (K == 0) return TQ_ERR_UNSUPPORTED;
+    if (K == 0) return zero_output(a, (cudaStream_t)stream);  // empty sums
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
     bool handled = false;
@@ -306,11 +326,43 @@ tq_status tq2_gemv(const void* X, int64_t M, const uint8_t* codes, const void* s
     a.fmt = 2;
     if (tq_status st = check_matmul(a)) return st;
     if (M == 0 || N == 0) return TQ_OK;
-    if (K == 0) return TQ_ERR_UNSUPPORTED;
+    if (K == 0) return zero_output(a, (cudaStream_t)stream);  // empty sums
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
     const cudaError_t e = launch_gemv2(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
                                        N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count);
+    if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
+    return from_cuda(e);
+}
+
+// ---- W4A16 affine format
+
+size_t tq_w4_codes_bytes(int64_t N, int64_t K, int G) {
+    if (!shape_ok(N, K, G) || G % 8 != 0) return 0;
+    return (size_t)N * (size_t)(K / 8) * 4;
+}
+
+tq_status tq_w4_gemv(const void* X, int64_t M, const uint32_t* codes, const void* scales, const void* biases,
+                     int64_t N, int64_t K, int G, void* Y, tq_out_dtype yt, tq_stream_t stream) {
+    if (!shape_ok(N, K, G) || G % 8 != 0 || M < 0) return TQ_ERR_INVALID_ARG;
+    if (yt != TQ_OUT_F32 && yt != TQ_OUT_BF16) return TQ_ERR_INVALID_ARG;
+    if (M > 0 && (K > (int64_t(1) << 62) / M || N > (int64_t(1) << 62) / M)) return TQ_ERR_INVALID_ARG;
+    const size_t cb = tq_w4_codes_bytes(N, K, G), sb = tq_scales_bytes(N, K, G);
+    const size_t xb = (size_t)M * (size_t)K * 2;
+    const size_t yb = (size_t)M * (size_t)N * (yt == TQ_OUT_F32 ? 4 : 2);
+    if ((xb && !X) || (cb && !codes) || (sb && (!scales || !biases)) || (yb && !Y)) return TQ_ERR_INVALID_ARG;
+    if (overlap(Y, yb, X, xb) || overlap(Y, yb, codes, cb) || overlap(Y, yb, scales, sb) || overlap(Y, yb, biases, sb))
+        return TQ_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(codes, 4) || !aligned(scales, 2) || !aligned(biases, 2) ||
+        !aligned(Y, yt == TQ_OUT_F32 ? 4 : 2))
+        return TQ_ERR_ALIGNMENT;
+    if (M == 0 || N == 0) return TQ_OK;
+    if (K == 0) return from_cuda(cudaMemsetAsync(Y, 0, yb, (cudaStream_t)stream));  // empty sums
+    const DeviceInfo* d = nullptr;
+    if (tq_status st = device_info(&d)) return st;
+    const cudaError_t e = launch_gemv_w4(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
+                                         static_cast<const uint16_t*>(biases), N, K, G, Y, yt == TQ_OUT_BF16,
+                                         (cudaStream_t)stream, d->sm_count);
     if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
     return from_cuda(e);
 }

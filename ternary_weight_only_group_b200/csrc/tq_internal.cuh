@@ -8,11 +8,42 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <atomic>
+#include <mutex>
 
 #include "tq.h"
 
 namespace tq {
+
+// Split cluster barrier.  Every thread of every CTA of the cluster arrives
+// once (relaxed) and later waits; once the wait returns, all CTAs of the
+// cluster are known to be running, so their shared memory may be written
+// through distributed shared memory.  Both calls must be reached by all
+// threads, warp-converged.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// A kernel's dynamic shared-memory limit, raised on demand and never lowered:
+// the check and the raise happen under one lock, so two host threads asking
+// for different sizes cannot leave the attribute below what either launches.
+struct SmemAttr {
+    std::mutex mu;
+    std::atomic<int> cur{0};
+    template <typename Kern>
+    cudaError_t ensure(Kern kern, int bytes) {
+        if (bytes <= cur.load(std::memory_order_acquire)) return cudaSuccess;
+        std::lock_guard<std::mutex> lk(mu);
+        if (bytes <= cur.load(std::memory_order_relaxed)) return cudaSuccess;
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e == cudaSuccess) cur.store(bytes, std::memory_order_release);
+        return e;
+    }
+};
 
 __host__ __device__ constexpr int bytes_per_group(int G) { return (G + 4) / 5; }
 

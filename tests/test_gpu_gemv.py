@@ -132,3 +132,18 @@ def test_small_m_tensor_path(M, N, K, G):
     W = synthetic.weights(N, K, index=M * 7 + N)
     X = synthetic.activations(M, K)
     check(X, W, G)
+
+
+@pytest.mark.parametrize("fn", [tq.gemv, tq.gemm, tq.gemv2])
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_empty_sum_k0(fn, dt):
+    """K = 0: every output is an empty sum, +0 (the output starts as NaN)."""
+    M, N, G = 3, 77, 64
+    X = torch.empty((M, 0), dtype=torch.bfloat16, device="cuda")
+    codes = torch.empty((N, 0, 13), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((N, 0), dtype=torch.float16, device="cuda")
+    Y = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
+    fn(X, codes, scales, N, 0, G, out=Y)
+    torch.cuda.synchronize()
+    y = Y.float().cpu().numpy()
+    assert np.all(y == 0) and not np.any(np.signbit(y))

@@ -1,0 +1,70 @@
+"""GPU parity of tq_w4_gemv (the W4A16 affine format, CUDA cores) against the
+oracle's binary64 reconstruction w = q * s + b and matmul.
+
+fp32 outputs: max_n |gpu - oracle| <= 1e-3 * max_n |oracle| per output row;
+bf16 outputs: |gpu - oracle| <= 2e-2 + 2e-2 |oracle|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+import ternary_weight_only_group_b200 as tq
+from tests.parity import assert_close_bf16, assert_rows_close_f32, to_dev_bf16, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def dev_params(codes, scales, biases):
+    c = torch.from_numpy(codes.view(np.int32)).cuda()
+    return c, to_dev_bf16(scales), to_dev_bf16(biases)
+
+
+def check(N, K, G, M, index=0, dtypes=(torch.float32, torch.bfloat16)):
+    codes, scales, biases = synthetic.w4_params(N, K, G, index=index)
+    X = synthetic.activations(M, K, offset=800)
+    ref = oracle.linear_w4(X, codes, scales, biases, N, K, G)
+    dc, ds, db = dev_params(codes, scales, biases)
+    for dt in dtypes:
+        Y = tq.w4_gemv(to_dev_bf16(X), dc, ds, db, N, K, G, out_dtype=dt)
+        torch.cuda.synchronize()
+        if dt == torch.float32:
+            assert_rows_close_f32(to_f64(Y), ref)
+        else:
+            assert_close_bf16(to_f64(Y), ref)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 8, 11])
+@pytest.mark.parametrize("N,K,G", [(3584, 1024, 128), (1024, 3584, 128), (1536, 1536, 64), (4096, 1536, 32)])
+def test_w4_gemv_shapes(N, K, G, M):
+    """Streaming kernel: one to four 32-column chunks per lane and row, one to
+    eight tokens per launch, two launches past eight tokens."""
+    check(N, K, G, M, index=N + K + G)
+
+
+@pytest.mark.parametrize("N,K,G", [(77, 4096, 128), (9, 96, 32), (2001, 512, 512)])
+def test_w4_gemv_ragged_rows(N, K, G):
+    check(N, K, G, 1, index=N)
+
+
+@pytest.mark.parametrize("N,K,G", [(300, 1024, 8), (129, 960, 48), (64, 8192, 128), (50, 1000, 40)])
+@pytest.mark.parametrize("M", [1, 5])
+def test_w4_gemv_generic_shapes(N, K, G, M):
+    """Group sizes that are not multiples of 32, and K beyond the streaming
+    kernel's 4096: the one-warp-per-row kernel."""
+    check(N, K, G, M, index=G + 7)
+
+
+def test_w4_gemv_every_code_value():
+    """Each code value 0..15 in every nibble position: rows of constant words."""
+    N, K, G = 64, 1024, 128
+    codes, scales, biases = synthetic.w4_params(N, K, G, index=3)
+    for q in range(16):
+        codes[q] = np.uint32(sum(q << (4 * k) for k in range(8)))
+    X = synthetic.activations(1, K, offset=801)
+    ref = oracle.linear_w4(X, codes, scales, biases, N, K, G)
+    dc, ds, db = dev_params(codes, scales, biases)
+    Y = tq.w4_gemv(to_dev_bf16(X), dc, ds, db, N, K, G, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert_rows_close_f32(to_f64(Y), ref)
