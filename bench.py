@@ -38,9 +38,12 @@ METRIC = "ternary x bf16 GEMV HBM GB/s (% of peak); prefill GEMM TFLOP/s; pack G
 # DRAM bytes (read + write) of one gemv_predecode_kernel launch per decode
 # shape (N, K, G), M=1, from an ncu capture of dram__bytes_read.sum +
 # dram__bytes_write.sum on `bench.py --only gemv` (one launch per shape).
-# Valid for the kernel as captured; set to None when it changes.
+# Valid only for the kernel source they were captured on: the SHA-256 of
+# gemv_predecode.cu at capture time is recorded beside them, and the figures
+# are reported only while the current source still has that hash.
 PREDECODE_DRAM_BYTES = {(3584, 1024, 64): 906496, (1024, 3584, 64): 911104,
                         (3584, 1024, 128): 848896, (1024, 3584, 128): 854528}
+PREDECODE_DRAM_SRC_SHA256 = None
 FFN = {"gate": (3584, 1024), "up": (3584, 1024), "down": (1024, 3584)}
 MSWEEP = {"q": (1536, 1536), "o": (1536, 1536), "gate": (4096, 1536), "up": (4096, 1536), "down": (1536, 4096)}
 MSWEEP_LAYERS = 28
@@ -59,6 +62,36 @@ def load_peaks():
                 "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
+
+
+def source_sha256(rel):
+    import hashlib
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def traffic_valid() -> bool:
+    """True while gemv_predecode.cu is the source the recorded DRAM bytes were captured on."""
+    return (PREDECODE_DRAM_SRC_SHA256 is not None and
+            source_sha256("ternary_weight_only_group_b200/csrc/gemv_predecode.cu") == PREDECODE_DRAM_SRC_SHA256)
+
+
+def host_cpu():
+    """Model name, logical CPUs and the CPUs this process may run on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        affinity = len(os.sched_getaffinity(0))
+    except AttributeError:
+        affinity = os.cpu_count()
+    return {"model": model, "logical_cpus": os.cpu_count(), "affinity_cpus": affinity}
 
 
 def packed_bytes(N, K, G):
@@ -306,6 +339,7 @@ def run_ours(args, rank, world, local):
     with ClockSampler(local) as clocks:
         ms = timed(graph.replay, K_steps, W_steps, world)
         ms_e2e = timed(graph_e2e.replay, K_steps, W_steps, world)
+        results["fused_gateup"] = bench_fused_gateup(tq, args, world, peaks, packs)
         results["stream"] = bench_gemv_stream(tq, args, world, peaks)
         results["pack"], results["unpack"] = bench_bulk_codec(tq, args, world, peaks)
         results["prefill"] = bench_prefill(tq, args, world, peaks)
@@ -319,7 +353,7 @@ def run_ours(args, rank, world, local):
     per_launch_us = ms_step * 1e3 / launches_per_step
     avg_bytes = step_bytes / launches_per_step
     traffic = None  # measured DRAM bytes per launch, averaged like avg_bytes
-    if PREDECODE_DRAM_BYTES is not None and all((N, K, G) in PREDECODE_DRAM_BYTES for (G, l, name, N, K, xo, yo) in calls):
+    if traffic_valid() and all((N, K, G) in PREDECODE_DRAM_BYTES for (G, l, name, N, K, xo, yo) in calls):
         traffic = round(sum(PREDECODE_DRAM_BYTES[(N, K, G)] for (G, l, name, N, K, xo, yo) in calls) / len(calls), 1)
     achieved = avg_bytes / (per_launch_us * 1e-6) / 1e9
     if rank != 0:
@@ -360,6 +394,7 @@ def run_ours(args, rank, world, local):
                 "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2},
         "gpu_launches": launches_per_step * K_steps * 2 + count_launches(results),
         "clocks": clk,
+        "fused_gateup": results["fused_gateup"],
         "gemv_stream": results["stream"],
         "pack": results["pack"],
         "unpack": results["unpack"],
@@ -368,6 +403,48 @@ def run_ours(args, rank, world, local):
         "ternary2": results["ternary2"],
     }
     print(json.dumps(line), flush=True)
+
+
+def bench_fused_gateup(tq, args, world, peaks, packs):
+    """The headline's decode chain with gate and up of every layer stacked
+    into one [7168 x 1024] matrix (one launch sharing the activations) and
+    down after it: 48 layers x 2 launches x 2 group sizes = 192 tq_gemv
+    launches per step from one CUDA graph, the same weights and bytes."""
+    import torch
+    calls = []
+    x_elems = y_elems = 0
+    fused = {}
+    for G in GROUPS:
+        for l in range(LAYERS):
+            cg_, sg = packs[(G, l, "gate")]
+            cu, su = packs[(G, l, "up")]
+            fused[(G, l)] = (torch.cat([cg_, cu]), torch.cat([sg, su]))
+            for name, (N, K) in (("gateup", (2 * FFN["gate"][0], FFN["gate"][1])), ("down", FFN["down"])):
+                calls.append((G, l, name, N, K, x_elems, y_elems))
+                x_elems += K
+                y_elems += N
+    X = device_acts(1, x_elems, seed=2002).view(-1)
+    Y = torch.empty(y_elems, dtype=torch.bfloat16, device="cuda")
+    step_bytes = sum(packed_bytes(N, K, G) + 2 * K + 2 * N for (G, l, name, N, K, xo, yo) in calls)
+
+    def step():
+        for (G, l, name, N, K, xo, yo) in calls:
+            c, s_ = fused[(G, l)] if name == "gateup" else packs[(G, l, "down")]
+            tq.gemv(X[xo:xo + K].view(1, K), c, s_, N, K, G, out=Y[yo:yo + N].view(1, N))
+    step()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+        step()
+    ms = timed(graph.replay, args.steps, args.warmup, world)
+    us = ms * 1e3 / args.steps
+    gbs = step_bytes / us / 1e3
+    del graph, fused
+    return {"launches_per_step": len(calls), "us_per_step": round(us, 1),
+            "us_per_launch": round(us / len(calls), 3), "GB/s": round(gbs, 1),
+            "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": step_bytes,
+            "launches": args.steps * len(calls),
+            "note": "gate and up of each layer as one [7168 x 1024] launch, then down; both G"}
 
 
 def count_launches(obj) -> int:
@@ -402,7 +479,7 @@ def bench_gemv_stream(tq, args, world, peaks):
     gbs = byts * reps / (ms * 1e-3) / 1e9
     return {"shape": [N, K], "G": G, "us": round(ms * 1e3 / reps, 2), "GB/s": round(gbs, 1),
             "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": reps,
-            "kernel": "gemv_lut_kernel (lookup tables; M=1 matrices too large for the pre-decode kernel)",
+            "kernel": "gemv_lut_stream_kernel<128> (lookup tables of one 512-column slice per CTA, 2-CTA clusters)",
             "note": "four copies of 38.5 MB used in turn (154 MB > L2)"}
 
 
@@ -674,21 +751,77 @@ def oracle_sample_step():
     return nbytes
 
 
-def cpu_baseline(args, budget_s=10.0):
-    """The oracle as it stands, single-threaded C, timed on this host on a
-    bounded sample: repeated decode GEMVs of the layer-0 projections."""
-    oracle_mats()
+def _oracle_pool_init(mats):
+    global _ORACLE_MATS
+    _ORACLE_MATS = mats
+
+
+def _oracle_rows_pass(job):
+    """Worker: decode GEMV (decode to bf16 + binary64 matmul) of rows
+    [N*part/nparts, N*(part+1)/nparts) of every sampled matrix."""
+    import oracle
+    part, nparts = job
+    for X, codes, scales, N, K, G in _ORACLE_MATS:
+        lo, hi = N * part // nparts, N * (part + 1) // nparts
+        if hi > lo:
+            oracle.linear(X, codes[lo:hi], scales[lo:hi], hi - lo, K, G)
+    return part
+
+
+class OraclePool:
+    """The single-threaded C oracle run by one spawned process per host CPU
+    (rows split evenly), for the all-core baseline.  Spawned, not forked, so
+    no child inherits a CUDA context."""
+
+    def __init__(self, n=None):
+        import multiprocessing as mp
+        self.n = n or host_cpu()["affinity_cpus"] or 1
+        self.pool = mp.get_context("spawn").Pool(self.n, initializer=_oracle_pool_init,
+                                                  initargs=(oracle_mats(),))
+        self.jobs = [(i, self.n) for i in range(self.n)]
+        self.pool.map(_oracle_rows_pass, self.jobs)  # workers up and warm
+
+    def step(self):
+        """One pass over the whole sample; returns its algorithmic bytes."""
+        self.pool.map(_oracle_rows_pass, self.jobs)
+        return sum(packed_bytes(N, K, G) + 2 * K + 2 * N for (_, _, _, N, K, G) in oracle_mats())
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def _timed_passes(step, budget_s):
     t0 = time.perf_counter()
     nbytes = reps = 0
     while True:
-        nbytes += oracle_sample_step()
+        nbytes += step()
         reps += 1
         if time.perf_counter() - t0 > budget_s:
             break
-    sec = time.perf_counter() - t0
-    return {"value": round(nbytes / sec / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{reps} passes of the decode GEMV (decode to bf16 + binary64 matmul) over "
-                      f"layer-0 gate/up/down for G=64 and G=128, M=1, {sec:.1f} s"}
+    return nbytes, reps, time.perf_counter() - t0
+
+
+SAMPLE_DESC = "decode GEMV (decode to bf16 + binary64 matmul) over layer-0 gate/up/down for G=64 and G=128, M=1"
+
+
+def cpu_baseline(args, budget_s=10.0):
+    """The oracle as it stands (plain C, binary64) timed on this host on a
+    bounded sample -- repeated decode GEMVs of the layer-0 projections --
+    on every host CPU (one spawned process per CPU, rows split) and on one."""
+    oracle_mats()
+    host = host_cpu()
+    pool = OraclePool()
+    try:
+        nb, reps, sec = _timed_passes(pool.step, budget_s)
+    finally:
+        pool.close()
+    nb1, reps1, sec1 = _timed_passes(oracle_sample_step, budget_s)
+    return {"value": round(nb / sec / 1e9, 4), "unit": "GB/s", "cores": pool.n, "kind": "oracle",
+            "sample": f"{reps} passes of the {SAMPLE_DESC}, rows split over {pool.n} processes, {sec:.1f} s",
+            "host": host,
+            "single_thread": {"value": round(nb1 / sec1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                              "sample": f"{reps1} passes of the same sample, {sec1:.1f} s"}}
 
 
 def run_reference(args, rank, world):
@@ -697,12 +830,16 @@ def run_reference(args, rank, world):
     t = []
     nbytes = 0
     oracle_mats()
-    for _ in range(args.warmup):
-        oracle_sample_step()
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        nbytes = oracle_sample_step()
-        t.append(time.perf_counter() - t0)
+    pool = OraclePool()
+    try:
+        for _ in range(args.warmup):
+            pool.step()
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            nbytes = pool.step()
+            t.append(time.perf_counter() - t0)
+    finally:
+        pool.close()
     total = sum(t)
     value = nbytes * len(t) / total / 1e9
     line = {
@@ -713,8 +850,9 @@ def run_reference(args, rank, world):
         "config": {"workload": "decode GEMV, M=1, Qwen3.5-0.8B-shaped FFN gate/up 3584x1024 and "
                                "down 1024x3584, G in {64,128}; each step a bounded sample: layer 0's "
                                "three projections for both G (decode to bf16 + binary64 matmul)"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": "layer-0 gate/up/down, G=64 and 128, M=1, per step"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": pool.n, "kind": "oracle",
+                         "sample": f"layer-0 gate/up/down, G=64 and 128, M=1, per step, rows split over "
+                                   f"{pool.n} spawned processes", "host": host_cpu()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
