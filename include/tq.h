@@ -173,14 +173,23 @@ TQ_API tq_status tq2_quantize_pack(const void *W_bf16, int64_t N, int64_t K, int
 /* Decode the 2-bit format to bf16; as tq_unpack_bf16 (rejected groups NaN). */
 TQ_API tq_status tq2_unpack_bf16(const uint8_t *codes, const void *scales_f16, int64_t N, int64_t K,
                           int G, void *W_bf16_out, uint32_t *d_err, tq_stream_t stream);
-/* Fused unpack-and-scale matmul on the 2-bit format, CUDA cores, any M >= 1
- * (eight tokens per launch); result definition, arguments, alignment and
- * ordering rule as tq_gemv (X is read after the preceding work has
- * completed; codes and scales may be read before, so the kernel launched
- * immediately before on the same stream must not write them).  Covers G in
- * {16, 32, 64, 128, 256} and K <= 49152; other shapes return
- * TQ_ERR_UNSUPPORTED. */
+/* Fused unpack-and-scale matmul on the 2-bit format for decode; result
+ * definition, arguments, alignment and ordering rule as tq_gemv (X is read
+ * after the preceding work has completed; codes and scales may be read
+ * before, so the kernel launched immediately before on the same stream must
+ * not write them).  3..64 tokens with K % 64 == 0 and G % 64 == 0 take the
+ * tensor-core small-M kernels (2-bit codes decoded on chip); otherwise the
+ * CUDA-core kernel, eight tokens per launch, which covers G in {16, 32, 64,
+ * 128, 256} and K <= 49152; other shapes return TQ_ERR_UNSUPPORTED. */
 TQ_API tq_status tq2_gemv(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
+                   int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,
+                   size_t ws_bytes, uint32_t *d_err, tq_stream_t stream);
+/* Fused unpack-and-scale matmul on the 2-bit format for prefill, on the
+ * tensor cores (tcgen05, fp32 accumulators in tensor memory), What decoded on
+ * chip from the 2-bit codes: the result definition, arguments and ordering
+ * rule of tq_gemm.  Needs K % 64 == 0 and G % 64 == 0 (a 64-column stage is
+ * 16 whole code bytes of one group), else TQ_ERR_UNSUPPORTED. */
+TQ_API tq_status tq2_gemm(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
                    int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,
                    size_t ws_bytes, uint32_t *d_err, tq_stream_t stream);
 
@@ -207,6 +216,16 @@ TQ_API size_t tq_w4_codes_bytes(int64_t N, int64_t K, int G);
  * Errors: TQ_ERR_INVALID_ARG (shapes, G % 8, nulls, Y overlapping an input),
  * TQ_ERR_ALIGNMENT, TQ_ERR_CUDA. */
 TQ_API tq_status tq_w4_gemv(const void *X_bf16, int64_t M, const uint32_t *codes, const void *scales_bf16,
+                     const void *biases_bf16, int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype,
+                     tq_stream_t stream);
+
+/* Fused matmul on the W4 format for prefill, on the tensor cores (tcgen05,
+ * fp32 accumulators in tensor memory): the same result definition as
+ * tq_w4_gemv.  Each weight w = q * s + b is formed with one fp32 FMA and fed
+ * to the MMA as two bf16 terms, RNE_bf16(w) and RNE_bf16 of the remainder,
+ * so the products keep w to about 2^-17 relative.  Needs K % 64 == 0 and
+ * G % 64 == 0, else TQ_ERR_UNSUPPORTED; other arguments as tq_w4_gemv. */
+TQ_API tq_status tq_w4_gemm(const void *X_bf16, int64_t M, const uint32_t *codes, const void *scales_bf16,
                      const void *biases_bf16, int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype,
                      tq_stream_t stream);
 

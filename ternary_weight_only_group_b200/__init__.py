@@ -26,7 +26,7 @@ MAX_G = 4096
 
 EXPORTS = ("tq_codes_bytes", "tq_scales_bytes", "tq_workspace_bytes", "tq_quantize_pack",
            "tq_unpack_bf16", "tq_gemv", "tq_gemm", "tq2_codes_bytes", "tq2_quantize_pack",
-           "tq2_unpack_bf16", "tq2_gemv", "tq_w4_codes_bytes", "tq_w4_gemv", "tq_status_string",
+           "tq2_unpack_bf16", "tq2_gemv", "tq2_gemm", "tq_w4_codes_bytes", "tq_w4_gemv", "tq_w4_gemm", "tq_status_string",
            "tq_version")
 
 _lock = threading.Lock()
@@ -72,10 +72,14 @@ def lib() -> ctypes.CDLL:
             L.tq2_unpack_bf16.restype = i32
             L.tq2_gemv.argtypes = mm
             L.tq2_gemv.restype = i32
+            L.tq2_gemm.argtypes = mm
+            L.tq2_gemm.restype = i32
             L.tq_w4_codes_bytes.argtypes = [i64, i64, i32]
             L.tq_w4_codes_bytes.restype = sz
             L.tq_w4_gemv.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, vp, i32, vp]
             L.tq_w4_gemv.restype = i32
+            L.tq_w4_gemm.argtypes = [vp, i64, vp, vp, vp, i64, i64, i32, vp, i32, vp]
+            L.tq_w4_gemm.restype = i32
             L.tq_status_string.argtypes = [i32]
             L.tq_status_string.restype = ctypes.c_char_p
             L.tq_version.argtypes = []
@@ -249,12 +253,31 @@ def gemv2(X, codes, scales, N: int, K: int, G: int, out_dtype=None, out=None, d_
                    out_dtype or torch.float32, out, d_err, stream, workspace)
 
 
+def gemm2(X, codes, scales, N: int, K: int, G: int, out_dtype=None, out=None, d_err=None,
+          stream=None, workspace=None):
+    """Prefill matmul on the 2-bit format (tensor cores): Y[M, N] = X . What^T."""
+    torch = _torch()
+    return _matmul(lib().tq2_gemm, "tq2_gemm", X, codes, scales, N, K, G,
+                   out_dtype or torch.bfloat16, out, d_err, stream, workspace)
+
+
 # ----------------------------------------------------------------------------
 # the W4A16 affine format (uint4 codes, bf16 scale and bias per group)
 
 def w4_gemv(X, codes, scales, biases, N: int, K: int, G: int, out_dtype=None, out=None, stream=None):
     """Decode matmul on the W4 format (CUDA cores): Y[M, N] = X . (q * s + b)^T.
     codes: int32/uint32 [N, K/8]; scales, biases: bf16 [N, K/G]."""
+    return _w4_matmul(lib().tq_w4_gemv, "tq_w4_gemv", X, codes, scales, biases, N, K, G,
+                      out_dtype, out, stream)
+
+
+def w4_gemm(X, codes, scales, biases, N: int, K: int, G: int, out_dtype=None, out=None, stream=None):
+    """Prefill matmul on the W4 format (tensor cores): Y[M, N] = X . (q * s + b)^T."""
+    return _w4_matmul(lib().tq_w4_gemm, "tq_w4_gemm", X, codes, scales, biases, N, K, G,
+                      out_dtype, out, stream)
+
+
+def _w4_matmul(fn, name, X, codes, scales, biases, N, K, G, out_dtype, out, stream):
     torch = _torch()
     X = _as_cuda(X, torch.bfloat16, "X")
     if not isinstance(codes, torch.Tensor) or not codes.is_cuda or codes.dtype not in (torch.int32, torch.uint32):
@@ -269,6 +292,6 @@ def w4_gemv(X, codes, scales, biases, N: int, K: int, G: int, out_dtype=None, ou
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype or torch.float32, device=X.device)
     yt = TQ_OUT_BF16 if out.dtype == torch.bfloat16 else TQ_OUT_F32
-    _check(lib().tq_w4_gemv(_ptr(X), M, _ptr(codes), _ptr(scales), _ptr(biases), N, K, G, _ptr(out), yt,
-                            _stream(stream)), "tq_w4_gemv")
+    _check(fn(_ptr(X), M, _ptr(codes), _ptr(scales), _ptr(biases), N, K, G, _ptr(out), yt,
+              _stream(stream)), name)
     return out

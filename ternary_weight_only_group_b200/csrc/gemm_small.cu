@@ -71,7 +71,9 @@ struct Params {
     WaitCfg wc;                   // wait bound and the withheld-load test hook
 };
 
-template <int NT, bool CODES_TMA>
+// FMT 3: base-3 codes (five digits per byte); FMT 2: the 2-bit format (four
+// codes per byte, G a multiple of 64: a stage's 64 codes are 16 whole bytes).
+template <int NT, bool CODES_TMA, int FMT>
 __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                  const __grid_constant__ CUtensorMap tmap_c,
                                                                  const Params p) {
@@ -94,7 +96,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
     // rule); every Y store follows MMAs that consumed X.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     cluster_arrive_relaxed();  // waited on before the first store into a peer's shared memory
-    fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
+    if (FMT == 3) fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(&sm.full_x[st], 1);
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
         const int k0 = kb * BK;
         g = k0 / p.G;
         c0 = k0 - g * p.G;
-        q_lo = c0 / 5;
+        q_lo = FMT == 3 ? c0 / 5 : c0 / 4;
     };
 
     if (warp == 0) {
@@ -185,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
             for (int j = 0; j < 14; ++j) bytes[j] = (q_lo + j < p.B) ? (uint32_t)__ldg(cb + q_lo + j) : kZeroByte;
         };
         uint32_t cur[14], nxt[14];
-        if (!CODES_TMA && nkl > 0) load_global(kb_lo, cur);
+        if (!CODES_TMA && FMT == 3 && nkl > 0) load_global(kb_lo, cur);
         uint32_t sc_nxt = nkl > 0 ? __ldg(srow + (kb_lo * BK) / p.G) : 0u;
         for (int i = 0; i < nkl; ++i) {
             const int kb = kb_lo + i, st = i % STAGES, use = i / STAGES;
@@ -193,6 +195,21 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
             stage_geom(kb, g, c0, q_lo);
             const uint32_t sc = sc_nxt;
             if (i + 1 < nkl) sc_nxt = __ldg(srow + ((kb + 1) * BK) / p.G);  // next stage's scale in flight
+            if constexpr (FMT == 2) {
+                // the stage's 16 code bytes start on a 16-byte boundary of the row
+                uint32_t wd[4];
+                if (CODES_TMA) {
+                    if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag, lim)) break;
+                    const uint4 v = *reinterpret_cast<const uint4*>(sm.c[st] + t * C_ROW);
+                    wd[0] = v.x, wd[1] = v.y, wd[2] = v.z, wd[3] = v.w;
+                } else {
+                    if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
+                    const uint32_t* cw = reinterpret_cast<const uint32_t*>(crow + (int64_t)g * p.B + q_lo);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) wd[j] = __ldg(cw + j);
+                }
+                decode_stage64_2bit(wd, sc, sm.w[st] + t * 128, t & 7);
+            } else {
             const int ql = p.B - 1 - q_lo;  // the group's last byte relative to q_lo
             uint32_t bytes[14], lastb = 0;
             if (CODES_TMA) {
@@ -210,10 +227,11 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
             }
             decode_stage64(sm.lut, bytes, c0 - 5 * q_lo, ql < 14, lastb, p.pad_base, p.pad_span, sc,
                            sm.w[st] + t * 128, t & 7);
+            }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_w[st]);
-            if (!CODES_TMA) {
+            if (!CODES_TMA && FMT == 3) {
 #pragma unroll
                 for (int j = 0; j < 14; ++j) cur[j] = nxt[j];
             }
@@ -262,7 +280,8 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
         const int64_t n = n0 + crank * RPQ + rr;
         if (n < p.N) {
             if (m == 0 && acc != acc)  // NaN output of the first token: rescan that W row
-                err_acc |= scan_row_errors(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G, p.B);
+                err_acc |= FMT == 3 ? scan_row_errors(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G, p.B)
+                                    : scan_row_errors2(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G);
             const int64_t o = (int64_t)m * p.N + n;
             if (p.y_bf16) reinterpret_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(acc);
             else reinterpret_cast<float*>(p.Y)[o] = acc;
@@ -286,10 +305,10 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
     if (threadIdx.x == 0 && *abort_flag && p.d_err) atomicOr(p.d_err, TQ_DERR_TIMEOUT);
 }
 
-template <int NT, bool CT>
+template <int NT, bool CT, int FMT>
 static cudaError_t launch_nt(const CUtensorMap& tx, const CUtensorMap& tc_, const Params& p, int tiles,
                              cudaStream_t stream) {
-    auto kern = gemm_small_kernel<NT, CT>;
+    auto kern = gemm_small_kernel<NT, CT, FMT>;
     const size_t smem = sizeof(Smem<NT>) + 1024;
     static SmemAttr smem_attr;
     if (cudaError_t e = smem_attr.ensure(kern, (int)smem)) return e;
@@ -314,16 +333,16 @@ static cudaError_t launch_nt(const CUtensorMap& tx, const CUtensorMap& tc_, cons
 
 cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                               cudaStream_t stream, int sm_count, bool* handled);
+                               cudaStream_t stream, int sm_count, bool* handled, int fmt);
 
 // Covered shapes: 1 <= M <= 64, K % 64 == 0, G % 64 == 0.  Otherwise *handled is
-// left false and nothing is launched.
+// left false and nothing is launched.  fmt: 3 base-3 codes, 2 the 2-bit format.
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                               int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                              cudaStream_t stream, int sm_count, bool* handled) {
+                              cudaStream_t stream, int sm_count, bool* handled, int fmt) {
     using namespace small;
     *handled = false;
-    const int B = bytes_per_group(G);
+    const int B = fmt == 3 ? bytes_per_group(G) : G / 4;
     const int64_t row_bytes = (int64_t)(K / G) * B;
     if (M < 1 || M > 64 || K % BK != 0 || G % 64 != 0 || N > (int64_t(1) << 31) || K > (1 << 30))
         return cudaSuccess;
@@ -347,7 +366,7 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     const int64_t slots = (M <= 32 ? 2 : 1) * (int64_t)sm_count;  // resident CTAs (16/32-token tiles: two per SM)
     while (CS < kMaxCS && tiles * CS * 2 <= slots && nk / (CS * 2) >= 2) CS *= 2;
     if (CS == 1)  // no K split: the persistent kernel walks the tiles
-        return launch_gemm_stream(X, M, codes, scales, N, K, G, Y, y_bf16, d_err, stream, sm_count, handled);
+        return launch_gemm_stream(X, M, codes, scales, N, K, G, Y, y_bf16, d_err, stream, sm_count, handled, fmt);
     Params p{};
     p.wc = tc::wait_cfg_from_env();
     p.codes = codes;
@@ -365,14 +384,24 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     p.y_bf16 = y_bf16;
     padding_range(G, p.pad_base, p.pad_span);
     cudaError_t e;
-    if (codes_tma) {
-        if (NT == 16) e = launch_nt<16, true>(tx, tcm, p, (int)tiles, stream);
-        else if (NT == 32) e = launch_nt<32, true>(tx, tcm, p, (int)tiles, stream);
-        else e = launch_nt<64, true>(tx, tcm, p, (int)tiles, stream);
+    if (fmt == 2) {
+        if (codes_tma) {
+            if (NT == 16) e = launch_nt<16, true, 2>(tx, tcm, p, (int)tiles, stream);
+            else if (NT == 32) e = launch_nt<32, true, 2>(tx, tcm, p, (int)tiles, stream);
+            else e = launch_nt<64, true, 2>(tx, tcm, p, (int)tiles, stream);
+        } else {
+            if (NT == 16) e = launch_nt<16, false, 2>(tx, tcm, p, (int)tiles, stream);
+            else if (NT == 32) e = launch_nt<32, false, 2>(tx, tcm, p, (int)tiles, stream);
+            else e = launch_nt<64, false, 2>(tx, tcm, p, (int)tiles, stream);
+        }
+    } else if (codes_tma) {
+        if (NT == 16) e = launch_nt<16, true, 3>(tx, tcm, p, (int)tiles, stream);
+        else if (NT == 32) e = launch_nt<32, true, 3>(tx, tcm, p, (int)tiles, stream);
+        else e = launch_nt<64, true, 3>(tx, tcm, p, (int)tiles, stream);
     } else {
-        if (NT == 16) e = launch_nt<16, false>(tx, tcm, p, (int)tiles, stream);
-        else if (NT == 32) e = launch_nt<32, false>(tx, tcm, p, (int)tiles, stream);
-        else e = launch_nt<64, false>(tx, tcm, p, (int)tiles, stream);
+        if (NT == 16) e = launch_nt<16, false, 3>(tx, tcm, p, (int)tiles, stream);
+        else if (NT == 32) e = launch_nt<32, false, 3>(tx, tcm, p, (int)tiles, stream);
+        else e = launch_nt<64, false, 3>(tx, tcm, p, (int)tiles, stream);
     }
     if (e == cudaSuccess) *handled = true;
     return e;

@@ -106,7 +106,9 @@ __device__ __forceinline__ void fetch_scale(uint8_t* dst, const uint16_t* S, con
         *reinterpret_cast<uint16_t*>(dst + (reinterpret_cast<uintptr_t>(S) & 2)) = *S;
 }
 
-template <int NT>
+// FMT 3: base-3 codes; FMT 2: the 2-bit format (a stage's 64 codes are the 16
+// bytes at the 16-byte-aligned offset G/4 * g + 16 * sub of the row).
+template <int NT, int FMT>
 __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                   const Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     // preceding kernel (codes and scales are weights, see tq_gemv's ordering
     // rule); every Y store follows MMAs that consumed X.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    fill_digit_selector_lut4_lanes(sm.lut, threadIdx.x, kThreads);
+    if (FMT == 3) fill_digit_selector_lut4_lanes(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(&sm.full_x[st], 1);
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
         auto issue = [&](int s) {
             if (grp + 2 * s < total) {
                 const int64_t n = row_of(pi);
-                const int q_lo = (BK * pi.sub) / 5;
+                const int q_lo = FMT == 3 ? (BK * pi.sub) / 5 : (BK * pi.sub) / 4;
                 uint8_t* slot = sm.win[grp][s % CR] + t * WIN;
                 fetch_window(slot, p.codes + n * p.row_bytes + (int64_t)pi.g * p.B + q_lo, p.codes, p.codes_end);
                 fetch_scale(slot + 32, p.scales + n * p.ng + pi.g, p.scales, p.scales_end);
@@ -248,18 +250,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
             const int i = grp + 2 * s, st = i % STAGES, use = i / STAGES;
             if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
             const int64_t n = row_of(pd);
-            const int c0 = BK * pd.sub, q_lo = c0 / 5;
+            const int c0 = BK * pd.sub, q_lo = FMT == 3 ? c0 / 5 : c0 / 4;
             const uintptr_t A = reinterpret_cast<uintptr_t>(p.codes + n * p.row_bytes + (int64_t)pd.g * p.B + q_lo);
             const uintptr_t S = reinterpret_cast<uintptr_t>(p.scales + n * p.ng + pd.g);
             const uint8_t* slot = sm.win[grp][s % CR] + t * WIN;
             const uint8_t* cb = slot + (A & 15);
             const uint32_t sc = *reinterpret_cast<const uint16_t*>(slot + 32 + (S & 2));
+            if constexpr (FMT == 2) {  // codes 4-byte aligned: cb is a word boundary of the window
+                const uint32_t* cw = reinterpret_cast<const uint32_t*>(cb);
+                const uint32_t wd[4] = {cw[0], cw[1], cw[2], cw[3]};
+                decode_stage64_2bit(wd, sc, sm.w[st] + t * 128, t & 7);
+            } else {
             uint32_t bytes[14];
 #pragma unroll
             for (int b = 0; b < 14; ++b) bytes[b] = cb[b];
             const int ql = p.B - 1 - q_lo;  // the group's last byte, relative to cb
             decode_stage64<32>(sm.lut + (t & 31), bytes, c0 - 5 * q_lo, ql < 14, ql < 14 ? cb[ql] : 0u, p.pad_base, p.pad_span,
                            sc, sm.w[st] + t * 128, t & 7);
+            }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_w[st]);
@@ -287,7 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
             const int64_t n = ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * WM + 32 * q + lane;
             if (n < p.N) {
                 if (__uint_as_float(v[0]) != __uint_as_float(v[0]))  // NaN for the first token: rescan the row
-                    err_acc |= scan_row_errors(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G, p.B);
+                    err_acc |= FMT == 3 ? scan_row_errors(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G, p.B)
+                                        : scan_row_errors2(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G);
 #pragma unroll
                 for (int m = 0; m < NT; ++m) {
                     if (m < p.M) {
@@ -316,9 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     if (threadIdx.x == 0 && *abort_flag && p.d_err) atomicOr(p.d_err, TQ_DERR_TIMEOUT);
 }
 
-template <int NT>
+template <int NT, int FMT>
 static cudaError_t launch_nt(const CUtensorMap& tx, const Params& p, int grid, cudaStream_t stream) {
-    auto kern = gemm_stream_kernel<NT>;
+    auto kern = gemm_stream_kernel<NT, FMT>;
     const size_t smem = sizeof(Smem<NT>) + 1024;
     static SmemAttr smem_attr;
     if (cudaError_t e = smem_attr.ensure(kern, (int)smem)) return e;
@@ -341,13 +350,13 @@ static cudaError_t launch_nt(const CUtensorMap& tx, const Params& p, int grid, c
 // *handled is left false and nothing is launched.
 cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                               cudaStream_t stream, int sm_count, bool* handled) {
+                               cudaStream_t stream, int sm_count, bool* handled, int fmt) {
     using namespace stream;
     *handled = false;
     if (M < 1 || M > 64 || K % BK != 0 || G % 64 != 0 || N < 1 || K > (1 << 30)) return cudaSuccess;
     const int64_t tiles = (N + WM - 1) / WM;
     if (tiles > 0x7FFFFFFF / (K / BK)) return cudaSuccess;
-    const int B = bytes_per_group(G);
+    const int B = fmt == 3 ? bytes_per_group(G) : G / 4;
     const int NT = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
     CUtensorMap tx;
     if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<uint16_t*>(X), (uint64_t)K, (uint64_t)M,
@@ -373,9 +382,15 @@ cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* code
     padding_range(G, p.pad_base, p.pad_span);
     const int grid = (int)(tiles < sm_count ? tiles : sm_count);
     cudaError_t e;
-    if (NT == 16) e = launch_nt<16>(tx, p, grid, stream);
-    else if (NT == 32) e = launch_nt<32>(tx, p, grid, stream);
-    else e = launch_nt<64>(tx, p, grid, stream);
+    if (fmt == 2) {
+        if (NT == 16) e = launch_nt<16, 2>(tx, p, grid, stream);
+        else if (NT == 32) e = launch_nt<32, 2>(tx, p, grid, stream);
+        else e = launch_nt<64, 2>(tx, p, grid, stream);
+    } else {
+        if (NT == 16) e = launch_nt<16, 3>(tx, p, grid, stream);
+        else if (NT == 32) e = launch_nt<32, 3>(tx, p, grid, stream);
+        else e = launch_nt<64, 3>(tx, p, grid, stream);
+    }
     if (e == cudaSuccess) *handled = true;
     return e;
 }

@@ -66,6 +66,7 @@ struct Smem {
 struct Params {
     const uint8_t* codes;
     const uint16_t* scales;
+    const uint16_t* biases;  // W4A16 only
     void* Y;
     uint32_t* d_err;
     int64_t M, N;
@@ -80,7 +81,15 @@ struct Params {
 
 // TBN: W rows per tile (256, or 224 when that leaves a fuller last wave);
 // buffers and tensor memory are laid out for 256.
-template <bool CODES_TMA, int TBN>
+// FMT 3: base-3 codes; FMT 2: the 2-bit format (a stage's 64 codes are 16
+// whole bytes at a 16-byte boundary of the row); FMT 4: the W4A16 affine
+// format (TBN = 128).  A W4 weight w = q * s + b (one fp32 FMA) is held as
+// two bf16 tiles, hi = RNE_bf16(w) and lo = RNE_bf16(w - hi), which share
+// the 32 KB W buffer of a stage; each k-step issues the MMA of both into the
+// same accumulator, so the products carry w to about 2^-17 relative (one
+// bf16 tile alone would carry only 2^-9).  Two threads decode a row, 32
+// columns each.
+template <bool CODES_TMA, int TBN, int FMT>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                               const __grid_constant__ CUtensorMap tmap_c,
                                                               const Params p) {
@@ -93,7 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     volatile int* abort_flag = &sm.abort_flag;
     const uint64_t lim = p.wc.limit_ns;
 
-    fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
+    if (FMT == 3) fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
+    static_assert(FMT != 4 || TBN == 128, "W4 tiles are 128 rows (hi and lo share the W buffer)");
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
             mbar_init(&sm.full_a[st], 1);
@@ -122,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         const int k0 = kb * BK;
         g = k0 / p.G;
         c0 = k0 - g * p.G;
-        q_lo = c0 / 5;
+        q_lo = FMT == 3 ? c0 / 5 : (FMT == 2 ? c0 / 4 : c0 / 2);
     };
 
     if (warp == 0) {
@@ -171,9 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                 for (int sub = 0; sub < 2; ++sub) {
                     const uint32_t a0 = s32(sm.a[st][sub]);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
+                    for (int k = 0; k < BK / 16; ++k) {
                         mma_bf16(tmem + (uint32_t)(sub * BN), smem_desc_sw128(a0 + 32 * k),
                                  smem_desc_sw128(b0 + 32 * k), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                        if (FMT == 4)  // the lo tile, 128 rows after hi
+                            mma_bf16(tmem + (uint32_t)(sub * BN), smem_desc_sw128(a0 + 32 * k),
+                                     smem_desc_sw128(b0 + TBN * 128 + 32 * k), idesc, 1u);
+                    }
                 }
                 mma_commit(&sm.empty[st]);  // stage free once these MMAs have read it
             }
@@ -182,10 +196,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     } else if (warp >= kDecodeWarp0) {
         // ---------------- decoders: thread -> one W row of the tile
         const int t = threadIdx.x - kDecodeWarp0 * 32;  // 0..255
-        const int64_t n = n0 + t;
+        const int64_t n = n0 + (FMT == 4 ? (t & (TBN - 1)) : t);  // W4: two threads per row
         const bool row_ok = n < p.N;
         const uint8_t* crow = p.codes + (row_ok ? n : 0) * p.row_bytes;
         const uint16_t* srow = p.scales + (row_ok ? n : 0) * p.ng;
+        const uint16_t* brow = FMT == 4 ? p.biases + (row_ok ? n : 0) * p.ng : nullptr;
+        const uint8_t* w4row = crow;
         auto load_global = [&](int kb, uint32_t (&bytes)[14]) {  // code bytes of a stage, by loads
             int g, c0, q_lo;
             stage_geom(kb, g, c0, q_lo);
@@ -194,14 +210,68 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             for (int i = 0; i < 14; ++i) bytes[i] = (q_lo + i < p.B) ? (uint32_t)__ldg(cb + q_lo + i) : kZeroByte;
         };
         uint32_t nxt[14];
-        if (!CODES_TMA) load_global(0, nxt);
+        if (!CODES_TMA && FMT == 3) load_global(0, nxt);
         uint32_t sc_nxt = __ldg(srow);  // scale of stage 0 (group 0)
+        uint32_t bi_nxt = FMT == 4 ? __ldg(brow) : 0u;
         for (int kb = 0; kb < nk; ++kb) {
             const int st = kb % STAGES, use = kb / STAGES;
             int g, c0, q_lo;
             stage_geom(kb, g, c0, q_lo);
             const uint32_t sc = sc_nxt;
             if (kb + 1 < nk) sc_nxt = __ldg(srow + ((kb + 1) * BK) / p.G);  // next stage's scale in flight
+            const uint32_t bi = bi_nxt;
+            if (FMT == 4 && kb + 1 < nk) bi_nxt = __ldg(brow + ((kb + 1) * BK) / p.G);
+            if constexpr (FMT == 4) {
+                // thread -> row t % 128, columns 32 (t / 128) .. + 31 of the stage
+                const int r = t & (TBN - 1), hh = t / TBN;
+                uint32_t wd[4];
+                if (CODES_TMA) {
+                    if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag, lim)) break;
+                    const uint4 v = *reinterpret_cast<const uint4*>(sm.c[st] + r * C_ROW + 16 * hh);
+                    wd[0] = v.x, wd[1] = v.y, wd[2] = v.z, wd[3] = v.w;
+                } else {
+                    if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
+                    const uint32_t* cw = reinterpret_cast<const uint32_t*>(w4row + 32 * kb + 16 * hh);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) wd[i] = __ldg(cw + i);
+                }
+                const float s = __uint_as_float(sc << 16), b = __uint_as_float(bi << 16);
+                uint32_t hi[16], lo[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {  // columns 2j, 2j+1: nibbles of word j / 4
+                    const uint32_t wv = wd[j >> 2] >> (8 * (j & 3));
+                    const float q0 = __uint_as_float(0x4B000000u | (wv & 0xFu)) - 8388608.f;
+                    const float q1 = __uint_as_float(0x4B000000u | ((wv >> 4) & 0xFu)) - 8388608.f;
+                    const float w0 = fmaf(q0, s, b), w1 = fmaf(q1, s, b);
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(w0, w1);
+                    const uint32_t hv = *reinterpret_cast<const uint32_t*>(&h2);
+                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(w0 - __uint_as_float(hv << 16),
+                                                                    w1 - __uint_as_float(hv & 0xFFFF0000u));
+                    hi[j] = hv;
+                    lo[j] = *reinterpret_cast<const uint32_t*>(&l2);
+                }
+                uint8_t* rh = sm.b[st] + r * 128;
+                uint8_t* rl = sm.b[st] + TBN * 128 + r * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int ch = ((4 * hh + c) ^ (r & 7)) << 4;
+                    *reinterpret_cast<uint4*>(rh + ch) = make_uint4(hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+                    *reinterpret_cast<uint4*>(rl + ch) = make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
+                }
+            } else if constexpr (FMT == 2) {
+                uint32_t wd[4];
+                if (CODES_TMA) {
+                    if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag, lim)) break;
+                    const uint4 v = *reinterpret_cast<const uint4*>(sm.c[st] + t * C_ROW);
+                    wd[0] = v.x, wd[1] = v.y, wd[2] = v.z, wd[3] = v.w;
+                } else {
+                    if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
+                    const uint32_t* cw = reinterpret_cast<const uint32_t*>(crow + (int64_t)g * p.B + q_lo);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) wd[i] = __ldg(cw + i);
+                }
+                if (t < TBN) decode_stage64_2bit(wd, sc, sm.b[st] + t * 128, t & 7);
+            } else {
             const int ql = p.B - 1 - q_lo;  // the group's last byte relative to q_lo
             uint32_t bytes[14], lastb = 0;
             if (CODES_TMA) {
@@ -220,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             if (t < TBN)
                 decode_stage64(sm.lut, bytes, c0 - 5 * q_lo, ql < 14, lastb, p.pad_base, p.pad_span, sc,
                                sm.b[st] + t * 128, t & 7);
+            }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor core
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_b[st]);
@@ -239,12 +310,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                         const int64_t nb = n0 + 32 * c;
                         if (m < p.M && nb < p.N) {
                             const int cnt = (int)(p.N - nb < 32 ? p.N - nb : 32);
-                            if (m == 0) {  // a NaN output of the first X row: rescan that W row's groups
+                            if (m == 0 && FMT != 4) {  // a NaN output of the first X row: rescan that W row's groups
 #pragma unroll
                                 for (int j = 0; j < 32; ++j)
                                     if (j < cnt && __uint_as_float(r[j]) != __uint_as_float(r[j]))
-                                        err_acc |= scan_row_errors(p.codes + (nb + j) * p.row_bytes,
-                                                                   p.scales + (nb + j) * p.ng, p.ng, p.G, p.B);
+                                        err_acc |= FMT == 3 ? scan_row_errors(p.codes + (nb + j) * p.row_bytes,
+                                                                              p.scales + (nb + j) * p.ng, p.ng, p.G, p.B)
+                                                            : scan_row_errors2(p.codes + (nb + j) * p.row_bytes,
+                                                                               p.scales + (nb + j) * p.ng, p.ng, p.G);
                             }
                             if (p.y_bf16) {
                                 __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.Y) + m * p.N + nb;
@@ -344,14 +417,14 @@ size_t gemm_smem_bytes() { return sizeof(gemm::Smem) + 1024; }
 
 cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales, int64_t N,
                            int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err, cudaStream_t stream,
-                           int sm_count, bool* handled) {
+                           int sm_count, bool* handled, int fmt, const uint16_t* biases) {
     using namespace gemm;
     *handled = false;
     // Shapes this kernel covers: K a multiple of the 64-column stage, G a
     // multiple of 64 (a stage never crosses a group).
     if (K % BK != 0 || G % 64 != 0 || M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (1 << 30))
         return cudaSuccess;
-    const int B = bytes_per_group(G);
+    const int B = fmt == 3 ? bytes_per_group(G) : (fmt == 2 ? G / 4 : G / 2);
     const int64_t row_bytes = (int64_t)(K / G) * B;
     CUtensorMap tmap_x, tmap_c;
     std::memset(&tmap_c, 0, sizeof(tmap_c));
@@ -367,7 +440,7 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
         const int64_t tiles = m_tiles * ((N + bn - 1) / bn);
         return ((tiles + sm_count - 1) / sm_count) * bn;
     };
-    const int tbn = cost(224) < cost(256) ? 224 : 256;
+    const int tbn = fmt == 4 ? 128 : (cost(224) < cost(256) ? 224 : 256);
     if (codes_tma && !encode_tmap_2d(&tmap_c, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<uint8_t*>(codes),
                                      (uint64_t)row_bytes, (uint64_t)N, (uint64_t)row_bytes, C_ROW, (uint32_t)tbn,
                                      CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -376,6 +449,7 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
     p.wc = tc::wait_cfg_from_env();
     p.codes = codes;
     p.scales = scales;
+    p.biases = biases;
     p.Y = Y;
     p.d_err = d_err;
     p.M = M;
@@ -392,10 +466,14 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes, c
     const int64_t grid = m_tiles * p.n_tiles;
     if (grid > 0x7FFFFFFF) return cudaSuccess;
     const size_t smem = gemm_smem_bytes();
-    auto kern = codes_tma ? (tbn == 224 ? gemm_tc_kernel<true, 224> : gemm_tc_kernel<true, 256>)
-                          : (tbn == 224 ? gemm_tc_kernel<false, 224> : gemm_tc_kernel<false, 256>);
-    static SmemAttr smem_attr[4];
-    if (cudaError_t e = smem_attr[(codes_tma ? 2 : 0) + (tbn == 224 ? 1 : 0)].ensure(kern, (int)smem)) return e;
+    auto kern = fmt == 4   ? (codes_tma ? gemm_tc_kernel<true, 128, 4> : gemm_tc_kernel<false, 128, 4>)
+                : fmt == 2 ? (codes_tma ? (tbn == 224 ? gemm_tc_kernel<true, 224, 2> : gemm_tc_kernel<true, 256, 2>)
+                                        : (tbn == 224 ? gemm_tc_kernel<false, 224, 2> : gemm_tc_kernel<false, 256, 2>))
+                           : (codes_tma ? (tbn == 224 ? gemm_tc_kernel<true, 224, 3> : gemm_tc_kernel<true, 256, 3>)
+                                        : (tbn == 224 ? gemm_tc_kernel<false, 224, 3> : gemm_tc_kernel<false, 256, 3>));
+    static SmemAttr smem_attr[10];
+    const int slot = fmt == 4 ? 8 + (codes_tma ? 1 : 0) : (fmt == 2 ? 4 : 0) + (codes_tma ? 2 : 0) + (tbn == 224 ? 1 : 0);
+    if (cudaError_t e = smem_attr[slot].ensure(kern, (int)smem)) return e;
     kern<<<(unsigned)grid, kThreads, smem, stream>>>(tmap_x, tmap_c, p);
     *handled = true;
     return cudaGetLastError();

@@ -16,12 +16,14 @@
 // rows are added in rank order through distributed shared memory.
 //
 // Table layout.  Entry b of a table sits at byte 256 b + 4 slot of its block
-// (64 slots of fp32 per entry row, 64 KB per block, two blocks at absolute
-// shared address 0x10000), so slot s lives in bank s mod 32 whatever b is.
-// A PRMT builds the whole lookup address in one instruction: it places the
-// code byte in bits 8..15 and the lane's slot offset (4 x bank, from a
-// per-lane constant register) in bits 0..7; the block and the upper half of
-// the slots come from the load's immediate offset.
+// (64 slots of fp32 per entry row, 64 KB per block, two blocks at offset
+// 0x10000 of the CTA's shared-memory window), so slot s lives in bank s mod 32
+// whatever b is.  A PRMT builds the whole lookup address in one instruction:
+// it places the code byte in bits 8..15, the lane's slot offset (4 x bank,
+// from a per-lane constant register) in bits 0..7, and the window's base in
+// bits 24..31 (in a cluster, a CTA's shared-memory window starts at rank x
+// 2^24: the address of rank 1's first dynamic byte is 0x1000400); the block
+// and the upper half of the slots come from the load's immediate offset.
 //
 // Lanes.  Each lane reads one code word of a row's K slice with a single
 // global load and owns the bytes of ONE group in it, so one scale per lane
@@ -58,7 +60,7 @@ namespace {
 
 constexpr int kLsThreads = 512;
 constexpr int kLsWarps = kLsThreads / 32;
-constexpr uint32_t kLsTableAbs = 0x10000u;   // absolute shared address of the tables
+constexpr uint32_t kLsTableAbs = 0x10000u;   // offset of the tables in the CTA's shared-memory window
 constexpr uint32_t kLsBlockBytes = 0x10000u; // one block: 256 entry rows x 64 slots x 4 B
 constexpr uint32_t kLsSmemBytes = 0x30000u;  // dynamic request: covers [base, 0x30000) for any base <= 0x10000
 constexpr int kLsSliceCols = 512;            // K columns per CTA
@@ -121,52 +123,48 @@ __device__ __forceinline__ int ls_slot_position(int block, int sub, int bank) {
 }
 
 // Per-lane constants: offset of the lane's word in the slice, the row within
-// the step, the lane's group in the slice and the slot offsets (4 x bank) of
-// its lookups, one byte per step (lb0: steps 0..3, lb1: steps 4..7).
+// the step, the lane's group in the slice and the PRMT source words of its
+// lookups: lb[i] = {slot offset (4 x bank) of step 2i, of step 2i + 1, 0,
+// window base >> 24}.
 struct LsLane {
     uint32_t wofs;
     int h, grp;
-    uint32_t lb0, lb1;
+    uint32_t lb[4];
 };
 
 template <int G>
-__device__ __forceinline__ LsLane ls_lane(int lane) {
+__device__ __forceinline__ LsLane ls_lane(int lane, uint32_t win_base) {
     LsLane L{};
+    for (int i = 0; i < 4; ++i) L.lb[i] = win_base & 0xFF000000u;
     if constexpr (G == 128) {
         const int h = lane >> 4, q = lane & 15;
         const int w = q < 13 ? q : 3 * (q - 12);  // copies of the straddling words 3, 6, 9
         const bool copy = q >= 13;
         const int si = (w == 3 || w == 6 || w == 9) ? w / 3 - 1 : 0;
         const int grp = copy ? (8 * w + 7) / 26 : (8 * w) / 26;
-        uint32_t lb[2] = {0u, 0u};
         for (int k = 0; k < 8; ++k) {
             const int j = h ? ((k + 4) & 7) : k;
             const bool live = (8 * w + j) / 26 == grp;
             const int bank = live ? 2 * w + (j >> 2) : kLsFreeBank + 2 * si + h;
-            lb[k >> 2] |= (uint32_t)(4 * bank) << (8 * (k & 3));
+            L.lb[k >> 1] |= (uint32_t)(4 * bank) << (8 * (k & 1));
         }
         L.wofs = 8u * w;
         L.h = h;
         L.grp = grp;
-        L.lb0 = lb[0];
-        L.lb1 = lb[1];
     } else {
         // straddling words 3, 6, 9, 16, 19, 22 (copy i = lane - 26)
         const bool copy = lane >= 26;
         const int w = copy ? (lane < 29 ? 3 * (lane - 25) : 3 * (lane - 26) + 7) : lane;
         const int si = w <= 9 ? w / 3 - 1 : (w - 7) / 3;
         const int grp = copy ? (4 * w + 3) / 13 : (4 * w) / 13;
-        uint32_t lb = 0;
         for (int k = 0; k < 4; ++k) {
             const bool live = (4 * w + k) / 13 == grp;
             const int bank = live ? w : kLsFreeBank + si;
-            lb |= (uint32_t)(4 * bank) << (8 * k);
+            L.lb[k >> 1] |= (uint32_t)(4 * bank) << (8 * (k & 1));
         }
         L.wofs = 4u * w;
         L.h = 0;
         L.grp = grp;
-        L.lb0 = lb;
-        L.lb1 = 0;
     }
     return L;
 }
@@ -215,12 +213,13 @@ __device__ __forceinline__ float ls_transpose_reduce(float (&v)[NV], int lane) {
     return v[0];
 }
 
-// One lookup: byte k of word `a` plus the slot byte k of `lb`, at the
-// immediate offset of block / upper slots.
+// One lookup: byte K mod 4 of word `a` as bits 8..15, the slot byte K mod 2
+// of `lb` as bits 0..7, byte 2 of `lb` (0) and its byte 3 (the window base)
+// above; the block and the upper slots in the immediate offset.
 template <int G, int K>
 __device__ __forceinline__ float ls_lookup(uint32_t a, uint32_t lb) {
     constexpr uint32_t kk = (uint32_t)(K & 3);
-    constexpr uint32_t sel = 0xCC00u | (kk << 4) | (4u + kk);
+    constexpr uint32_t sel = 0x7600u | (kk << 4) | (4u + (uint32_t)(K & 1));
     constexpr uint32_t block = G == 128 ? (uint32_t)((K & 3) >> 1) : (uint32_t)(K >> 1);
     constexpr uint32_t imm = kLsTableAbs + block * kLsBlockBytes + 128u * (uint32_t)(K & 1);
     return lds_imm<imm>(prmt32(a, lb, sel));
@@ -239,19 +238,22 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    // Shared-memory window: the tables at [0x10000, 0x30000), the scales and
-    // partials just below 0x10000.
+    // Shared-memory window (base: the top byte of the dynamic region's
+    // address, the CTA's rank in the cluster): the tables at offsets
+    // [0x10000, 0x30000), the scales and partials just below 0x10000.
     const uint32_t dyn = (uint32_t)__cvta_generic_to_shared(smem);
+    const uint32_t wbase = dyn & 0xFF000000u, doff = dyn - wbase;
     const uint32_t misc = kLsTableAbs - ls_misc_bytes<G>();
-    if (dyn > misc) {  // cannot happen with no static shared memory; fail closed
+    if (doff > misc) {  // the same offset in every CTA: all of them leave here, none waits on a peer
         if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
         return;
     }
-    float* ssc_all = reinterpret_cast<float*>(smem + (misc - dyn));
-    float* part = reinterpret_cast<float*>(smem + (misc - dyn) + ls_scale_bytes<G>());
+    float* ssc_all = reinterpret_cast<float*>(smem + (misc - doff));
+    float* part = reinterpret_cast<float*>(smem + (misc - doff) + ls_scale_bytes<G>());
     float* ssc = ssc_all + warp * kLsChunkRows * GPS;
+    const uint32_t tabs = wbase + kLsTableAbs;  // the tables, for the stores of the build
 
-    const LsLane L = ls_lane<G>(lane);
+    const LsLane L = ls_lane<G>(lane, wbase);
     const int64_t crow0 = (int64_t)cid * a.rows_per_cluster;
     const int64_t crow1 = min(a.N, crow0 + a.rows_per_cluster);
     const uint8_t* cbase = a.codes + (int64_t)crank * kLsSliceBytes + L.wofs;
@@ -309,7 +311,7 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
             for (int it = warp; it < 36; it += kLsWarps) {
                 const int bs = it / 9, d34 = it - 9 * bs;
                 const int block = bs >> 1, sub = bs & 1;
-                const uint32_t base = kLsTableAbs + block * kLsBlockBytes + 27u * d34 * 256u +
+                const uint32_t base = tabs + block * kLsBlockBytes + 27u * d34 * 256u +
                                       4u * (uint32_t)(lane + 32 * sub);
                 if (lane >= kLsFreeBank) {
 #pragma unroll
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
             // entry rows 243..255: NaN (invalid bytes) in table columns, 0 in the free ones
             for (int it = warp; it < 4; it += kLsWarps) {
                 const int block = it >> 1, sub = it & 1;
-                const uint32_t base = kLsTableAbs + block * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * sub);
+                const uint32_t base = tabs + block * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * sub);
                 const float v = lane < kLsFreeBank ? nan : 0.f;
 #pragma unroll
                 for (int b = 243; b < 256; ++b) sts_f32(base + 256u * b, v);
@@ -380,20 +382,20 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
                     if constexpr (G == 128) {
                         const uint32_t w0 = L.h ? cw.y : cw.x;
                         const uint32_t w1 = L.h ? cw.x : cw.y;
-                        const float t0 = ls_lookup<G, 0>(w0, L.lb0);
-                        const float t1 = ls_lookup<G, 1>(w0, L.lb0);
-                        const float t2 = ls_lookup<G, 2>(w0, L.lb0);
-                        const float t3 = ls_lookup<G, 3>(w0, L.lb0);
-                        const float t4 = ls_lookup<G, 4>(w1, L.lb1);
-                        const float t5 = ls_lookup<G, 5>(w1, L.lb1);
-                        const float t6 = ls_lookup<G, 6>(w1, L.lb1);
-                        const float t7 = ls_lookup<G, 7>(w1, L.lb1);
+                        const float t0 = ls_lookup<G, 0>(w0, L.lb[0]);
+                        const float t1 = ls_lookup<G, 1>(w0, L.lb[0]);
+                        const float t2 = ls_lookup<G, 2>(w0, L.lb[1]);
+                        const float t3 = ls_lookup<G, 3>(w0, L.lb[1]);
+                        const float t4 = ls_lookup<G, 4>(w1, L.lb[2]);
+                        const float t5 = ls_lookup<G, 5>(w1, L.lb[2]);
+                        const float t6 = ls_lookup<G, 6>(w1, L.lb[3]);
+                        const float t7 = ls_lookup<G, 7>(w1, L.lb[3]);
                         v[s] = (((t0 + t1) + (t2 + t3)) + ((t4 + t5) + (t6 + t7))) * sc;
                     } else {
-                        const float t0 = ls_lookup<G, 0>(cw, L.lb0);
-                        const float t1 = ls_lookup<G, 1>(cw, L.lb0);
-                        const float t2 = ls_lookup<G, 2>(cw, L.lb0);
-                        const float t3 = ls_lookup<G, 3>(cw, L.lb0);
+                        const float t0 = ls_lookup<G, 0>(cw, L.lb[0]);
+                        const float t1 = ls_lookup<G, 1>(cw, L.lb[0]);
+                        const float t2 = ls_lookup<G, 2>(cw, L.lb[1]);
+                        const float t3 = ls_lookup<G, 3>(cw, L.lb[1]);
                         v[s] = ((t0 + t1) + (t2 + t3)) * sc;
                     }
                 } else {

@@ -233,6 +233,41 @@ __device__ __forceinline__ void decode_stage64(const uint32_t* lut4, const uint3
     }
 }
 
+// Decoder of one row's 64 weights for a stage in the 2-bit format (code c =
+// t + 1 of weight j in bits 2 (j mod 4) of byte j / 4; code 3 invalid): the
+// four 32-bit words w[] hold the stage's 64 codes in column order (G a
+// multiple of 64, so the stage lies in one group and has no padding).
+// (w >> 2k) & 0x03030303 holds the codes of columns k, k+4, k+8, k+12 in its
+// bytes; mapped to selector bytes 0x10 + 0x22 c over V = {-s, 0}, Z = {+s,
+// NaN} and interleaved by PRMT into the selector pairs of adjacent columns,
+// one PRMT per column pair picks the bf16 values.  Code 3 and a rejected
+// scale give NaN.  Writes the 128-byte swizzled K-major tile row.
+__device__ __forceinline__ void decode_stage64_2bit(const uint32_t (&w)[4], uint32_t scale_bits, uint8_t* tile_row,
+                                                    int row_in_atom) {
+    uint32_t V, Z;
+    if (scale_is_bad(scale_bits)) {
+        V = Z = 0x7FC07FC0u;
+    } else {
+        const uint32_t mag = scale_bits == 0 ? 0u : scale_to_bf16_bits((uint16_t)scale_bits);
+        V = mag ? (mag | 0x8000u) : 0u;  // {-s, 0}
+        Z = mag | 0x7FC00000u;           // {+s, NaN}
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // columns 16 q .. 16 q + 15
+        uint32_t s[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) s[k] = 0x10101010u + 0x22u * ((w[q] >> (2 * k)) & 0x03030303u);
+        const uint32_t p01a = prmt(s[0], s[1], 0x5140u);  // columns (0,1) low half, (4,5) high half
+        const uint32_t p23a = prmt(s[2], s[3], 0x5140u);  // (2,3), (6,7)
+        const uint32_t p01b = prmt(s[0], s[1], 0x7362u);  // (8,9), (12,13)
+        const uint32_t p23b = prmt(s[2], s[3], 0x7362u);  // (10,11), (14,15)
+        *reinterpret_cast<uint4*>(tile_row + (((2 * q) ^ row_in_atom) << 4)) =
+            make_uint4(prmt(V, Z, p01a), prmt(V, Z, p23a), prmt(V, Z, p01a >> 16), prmt(V, Z, p23a >> 16));
+        *reinterpret_cast<uint4*>(tile_row + (((2 * q + 1) ^ row_in_atom) << 4)) =
+            make_uint4(prmt(V, Z, p01b), prmt(V, Z, p23b), prmt(V, Z, p01b >> 16), prmt(V, Z, p23b >> 16));
+    }
+}
+
 // Canonical range of a group's last code byte: digits REAL..4 equal to 1,
 // i.e. [base, base + 3^REAL) with base = sum_{i=REAL}^{4} 3^i (REAL < 5);
 // every byte below 243 when REAL == 5.

@@ -32,7 +32,7 @@ cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* c
                                   cudaStream_t stream, int sm_count);
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                               int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                              cudaStream_t stream, int sm_count, bool* handled);
+                              cudaStream_t stream, int sm_count, bool* handled, int fmt);
 cudaError_t launch_quantize_pack2(const uint16_t* W, int64_t N, int64_t K, int G, uint8_t* codes,
                                   uint16_t* scales, uint32_t* d_err, cudaStream_t stream, int sm_count);
 cudaError_t launch_unpack2(const uint8_t* codes, const uint16_t* scales, int64_t N, int64_t K, int G, uint16_t* out,
@@ -42,7 +42,7 @@ cudaError_t launch_gemv2(const uint16_t* X, int64_t M, const uint8_t* codes, con
 cudaError_t launch_gemm_tc(const uint16_t* X, int64_t M, const uint8_t* codes,
                            const uint16_t* scales, int64_t N, int64_t K, int G, void* Y,
                            int y_bf16, uint32_t* d_err, cudaStream_t stream, int sm_count,
-                           bool* handled);
+                           bool* handled, int fmt, const uint16_t* biases = nullptr);
 
 namespace {
 
@@ -237,7 +237,7 @@ tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* sc
     {
         bool handled = false;
         e = launch_gemm_small(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales), N,
-                              K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, &handled);
+                              K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, &handled, 3);
         if (e != cudaSuccess) return from_cuda(e);
         if (handled) return TQ_OK;
     }
@@ -268,12 +268,12 @@ tq_status tq_gemm(const void* X, int64_t M, const uint8_t* codes, const void* sc
     cudaError_t e = cudaSuccess;
     if (M <= 64)
         e = launch_gemm_small(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales), N,
-                              K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, &handled);
+                              K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, &handled, 3);
     if (e == cudaSuccess && !handled)
         e = launch_gemm_tc(static_cast<const uint16_t*>(X), M, codes,
                            static_cast<const uint16_t*>(scales), N, K, G, Y,
                            yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count,
-                           &handled);
+                           &handled, 3);
     if (e != cudaSuccess) return from_cuda(e);
     if (!handled) return TQ_ERR_UNSUPPORTED;
     return TQ_OK;
@@ -329,10 +329,43 @@ tq_status tq2_gemv(const void* X, int64_t M, const uint8_t* codes, const void* s
     if (K == 0) return zero_output(a, (cudaStream_t)stream);  // empty sums
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
+    // 3..64 tokens: the tensor-core small-M kernels on the 2-bit codes
+    if (M >= 3) {
+        bool handled = false;
+        const cudaError_t e = launch_gemm_small(static_cast<const uint16_t*>(X), M, codes,
+                                                static_cast<const uint16_t*>(scales), N, K, G, Y, yt == TQ_OUT_BF16,
+                                                d_err, (cudaStream_t)stream, d->sm_count, &handled, 2);
+        if (e != cudaSuccess) return from_cuda(e);
+        if (handled) return TQ_OK;
+    }
     const cudaError_t e = launch_gemv2(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
                                        N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count);
     if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
     return from_cuda(e);
+}
+
+tq_status tq2_gemm(const void* X, int64_t M, const uint8_t* codes, const void* scales, int64_t N, int64_t K, int G,
+                   void* Y, tq_out_dtype yt, void* workspace, size_t ws_bytes, uint32_t* d_err,
+                   tq_stream_t stream) {
+    (void)workspace; (void)ws_bytes;
+    MatmulArgs a{X, M, codes, scales, N, K, G, Y, yt};
+    a.fmt = 2;
+    if (tq_status st = check_matmul(a)) return st;
+    if (M == 0 || N == 0) return TQ_OK;
+    if (K == 0) return zero_output(a, (cudaStream_t)stream);  // empty sums
+    const DeviceInfo* d = nullptr;
+    if (tq_status st = device_info(&d)) return st;
+    bool handled = false;
+    cudaError_t e = cudaSuccess;
+    if (M <= 64)
+        e = launch_gemm_small(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales), N, K, G,
+                              Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, &handled, 2);
+    if (e == cudaSuccess && !handled)
+        e = launch_gemm_tc(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales), N, K, G, Y,
+                           yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, &handled, 2);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (!handled) return TQ_ERR_UNSUPPORTED;
+    return TQ_OK;
 }
 
 // ---- W4A16 affine format
@@ -365,6 +398,33 @@ tq_status tq_w4_gemv(const void* X, int64_t M, const uint32_t* codes, const void
                                          (cudaStream_t)stream, d->sm_count);
     if (e == cudaErrorNotSupported) return TQ_ERR_UNSUPPORTED;
     return from_cuda(e);
+}
+
+tq_status tq_w4_gemm(const void* X, int64_t M, const uint32_t* codes, const void* scales, const void* biases,
+                     int64_t N, int64_t K, int G, void* Y, tq_out_dtype yt, tq_stream_t stream) {
+    if (!shape_ok(N, K, G) || G % 8 != 0 || M < 0) return TQ_ERR_INVALID_ARG;
+    if (yt != TQ_OUT_F32 && yt != TQ_OUT_BF16) return TQ_ERR_INVALID_ARG;
+    if (M > 0 && (K > (int64_t(1) << 62) / M || N > (int64_t(1) << 62) / M)) return TQ_ERR_INVALID_ARG;
+    const size_t cb = tq_w4_codes_bytes(N, K, G), sb = tq_scales_bytes(N, K, G);
+    const size_t xb = (size_t)M * (size_t)K * 2;
+    const size_t yb = (size_t)M * (size_t)N * (yt == TQ_OUT_F32 ? 4 : 2);
+    if ((xb && !X) || (cb && !codes) || (sb && (!scales || !biases)) || (yb && !Y)) return TQ_ERR_INVALID_ARG;
+    if (overlap(Y, yb, X, xb) || overlap(Y, yb, codes, cb) || overlap(Y, yb, scales, sb) || overlap(Y, yb, biases, sb))
+        return TQ_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(codes, 4) || !aligned(scales, 2) || !aligned(biases, 2) ||
+        !aligned(Y, yt == TQ_OUT_F32 ? 4 : 2))
+        return TQ_ERR_ALIGNMENT;
+    if (M == 0 || N == 0) return TQ_OK;
+    if (K == 0) return from_cuda(cudaMemsetAsync(Y, 0, yb, (cudaStream_t)stream));  // empty sums
+    const DeviceInfo* d = nullptr;
+    if (tq_status st = device_info(&d)) return st;
+    bool handled = false;
+    const cudaError_t e = launch_gemm_tc(static_cast<const uint16_t*>(X), M, reinterpret_cast<const uint8_t*>(codes),
+                                         static_cast<const uint16_t*>(scales), N, K, G, Y, yt == TQ_OUT_BF16, nullptr,
+                                         (cudaStream_t)stream, d->sm_count, &handled, 4,
+                                         static_cast<const uint16_t*>(biases));
+    if (e != cudaSuccess) return from_cuda(e);
+    return handled ? TQ_OK : TQ_ERR_UNSUPPORTED;
 }
 
 const char* tq_status_string(tq_status s) {

@@ -256,4 +256,21 @@ static __device__ __noinline__ uint32_t scan_row_errors(const uint8_t* crow, con
     return bad;
 }
 
+// The same for the 2-bit format (ceil(G/4) bytes per group, code c in bits
+// 2 (j mod 4) of byte j / 4): a code 3 sets TQ_DERR_BYTE (a padding position
+// included), a padding code other than 1 or 3 TQ_DERR_PADDING.
+static __device__ __noinline__ uint32_t scan_row_errors2(const uint8_t* crow, const uint16_t* srow, int ng, int G) {
+    const int B = (G + 3) / 4;
+    uint32_t bad = 0;
+    for (int g = 0; g < ng; ++g) {
+        if (scale_is_bad(srow[g])) bad |= TQ_DERR_SCALE;
+        for (int j = 0; j < 4 * B; ++j) {
+            const uint32_t c = (crow[g * B + j / 4] >> (2 * (j % 4))) & 3u;
+            if (c == 3u) bad |= TQ_DERR_BYTE;
+            else if (j >= G && c != 1u) bad |= TQ_DERR_PADDING;
+        }
+    }
+    return bad;
+}
+
 }  // namespace tq

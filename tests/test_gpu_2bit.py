@@ -165,3 +165,52 @@ def test_gemv2_unsupported_group_size():
     codes, scales, _ = oracle.quantize_pack2(W, G)
     with pytest.raises(tq.TQError, match="UNSUPPORTED"):
         run_gemv2(synthetic.activations(1, K), codes, scales, N, K, G, torch.float32)
+
+
+def run_mm2(fn, X, codes, scales, N, K, G, out_dtype):
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Y = fn(to_dev_bf16(X), to_dev_u8(codes), to_dev_f16(scales), N, K, G, out_dtype=out_dtype, d_err=err)
+    torch.cuda.synchronize()
+    return to_f64(Y), int(err.item())
+
+
+@pytest.mark.parametrize("M", [3, 16, 40, 64, 100, 300])
+@pytest.mark.parametrize("N,K,G", [(300, 1024, 128), (1536, 4096, 64), (9601, 1024, 128), (515, 2048, 256)])
+def test_gemm2_tensor_paths(N, K, G, M):
+    """The 2-bit codes through the tensor-core kernels: split-K and persistent
+    small-M kernels (tq2_gemv and tq2_gemm up to 64 tokens), the prefill
+    kernel beyond; sampled token rows compared over every output column."""
+    W = synthetic.weights(N, K, index=N + K + G)
+    codes, scales, _ = oracle.quantize_pack2(W, G)
+    X = synthetic.activations(M, K, offset=1100)
+    rows = sorted({0, M // 2, M - 1})
+    ref = oracle.linear2(X, codes, scales, N, K, G, rows=rows)
+    fns = (tq.gemm2, tq.gemv2) if M <= 64 else (tq.gemm2,)
+    for fn in fns:
+        Y, e = run_mm2(fn, X, codes, scales, N, K, G, torch.float32)
+        assert_rows_close_f32(Y[rows], ref)
+        assert e == 0
+    Yb, _ = run_mm2(tq.gemm2, X, codes, scales, N, K, G, torch.bfloat16)
+    assert_close_bf16(Yb[rows], ref)
+
+
+@pytest.mark.parametrize("M", [16, 256])
+def test_gemm2_rejected_groups(M):
+    """Code 3 and bad scales on the tensor paths: NaN output columns and the
+    oracle's error bits."""
+    N, K, G = 9601, 1024, 128
+    W = synthetic.weights(N, K, index=13)
+    codes, scales, _ = oracle.quantize_pack2(W, G)
+    codes[5, 2, 7] |= 0xC0       # code 3
+    codes[4000, 7, 31] = 0xFF    # four codes 3 in a group's last byte
+    scales[9600, 1] = 0x7C00     # Inf scale, last row
+    scales[130, 0] = 0x8000      # -0 scale
+    scales[7777, 3] = 0          # zero group: finite
+    X = synthetic.activations(M, K, offset=1101)
+    rows = [0, M - 1]
+    ref = oracle.linear2(X, codes, scales, N, K, G, rows=rows)
+    _, e_ref = oracle.unpack2_bf16(codes, scales, N, K, G)
+    Y, e = run_mm2(tq.gemm2, X, codes, scales, N, K, G, torch.float32)
+    assert_rows_close_f32(Y[rows], ref)
+    assert np.all(np.isnan(Y[:, [5, 4000, 9600, 130]])) and np.all(np.isfinite(Y[:, 7777]))
+    assert e == e_ref == tq.DERR_BYTE | tq.DERR_SCALE

@@ -68,3 +68,29 @@ def test_w4_gemv_every_code_value():
     Y = tq.w4_gemv(to_dev_bf16(X), dc, ds, db, N, K, G, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert_rows_close_f32(to_f64(Y), ref)
+
+
+@pytest.mark.parametrize("M", [1, 16, 256, 300])
+@pytest.mark.parametrize("N,K,G", [(512, 1024, 128), (1000, 4096, 64), (4096, 1024, 128), (130, 2048, 256)])
+def test_w4_gemm_tensor_cores(N, K, G, M):
+    """tq_w4_gemm: the W4 weights as two bf16 terms (hi + remainder) on the
+    tensor cores; the fp32 per-row tolerance holds on every output."""
+    codes, scales, biases = synthetic.w4_params(N, K, G, index=N + 3 * K + G)
+    X = synthetic.activations(M, K, offset=802)
+    ref = oracle.linear_w4(X, codes, scales, biases, N, K, G)
+    dc, ds, db = dev_params(codes, scales, biases)
+    for dt in (torch.float32, torch.bfloat16):
+        Y = tq.w4_gemm(to_dev_bf16(X), dc, ds, db, N, K, G, out_dtype=dt)
+        torch.cuda.synchronize()
+        if dt == torch.float32:
+            assert_rows_close_f32(to_f64(Y), ref)
+        else:
+            assert_close_bf16(to_f64(Y), ref)
+
+
+def test_w4_gemm_unsupported_group_size():
+    N, K, G = 64, 1024, 32
+    codes, scales, biases = synthetic.w4_params(N, K, G, index=5)
+    dc, ds, db = dev_params(codes, scales, biases)
+    with pytest.raises(tq.TQError, match="UNSUPPORTED"):
+        tq.w4_gemm(to_dev_bf16(synthetic.activations(4, K)), dc, ds, db, N, K, G)
