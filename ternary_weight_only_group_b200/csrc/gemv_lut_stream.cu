@@ -13,17 +13,17 @@
 // byte costs a table load and an add.  512 columns are 104 code bytes at both
 // group sizes; a CTA keeps the tables of one such K slice, and the K slices
 // of a row are spread over the CTAs of a thread-block cluster whose partial
-// rows are added in rank order through distributed shared memory.
+// rows are added in rank order.
 //
 // Table layout.  Entry b of a table sits at byte 256 b + 4 slot of its block
 // (64 slots of fp32 per entry row, 64 KB per block, two blocks at offset
 // 0x10000 of the CTA's shared-memory window), so slot s lives in bank s mod 32
 // whatever b is.  A PRMT builds the whole lookup address in one instruction:
 // it places the code byte in bits 8..15, the lane's slot offset (4 x bank,
-// from a per-lane constant register) in bits 0..7, and the window's base in
-// bits 24..31 (in a cluster, a CTA's shared-memory window starts at rank x
-// 2^24: the address of rank 1's first dynamic byte is 0x1000400); the block
-// and the upper half of the slots come from the load's immediate offset.
+// +128 for the upper 32 slots) in bits 0..7, the block in bits 16..23 and the
+// window's base in bits 24..31 (in a cluster, a CTA's shared-memory window
+// starts at rank x 2^24: the address of rank 1's first dynamic byte is
+// 0x1000400), all from one per-lane constant register.
 //
 // Lanes.  Each lane reads one code word of a row's K slice with a single
 // global load and owns the bytes of ONE group in it, so one scale per lane
@@ -36,14 +36,25 @@
 //            instruction hit 32 different banks.
 //   G = 64:  4-byte words, 26 words + 6 straddling copies = 32 lanes, one
 //            row per warp step.
-// A warp handles 32 rows per chunk (16 or 32 steps); its per-row partials
-// are summed across lanes by a transposing butterfly.  Code words are
-// requested U steps ahead (ld.global.nc, no L1 allocation).
+// A warp handles 32 rows per chunk (16 or 32 steps) and keeps the code words
+// of U steps in flight (ld.global.nc, no L1 allocation); the row stride is a
+// compile-time constant (one kernel per cluster size), so the loads of a
+// chunk walk one pointer with immediate offsets.  Two steps are summed side
+// by side in packed fp32 pairs (add.rn.f32x2), in the same order as one step
+// alone.  A warp's per-row partials are summed across lanes by a transposing
+// butterfly; steps past the warp's last row compute rows that are never
+// stored, so no step is predicated.
 //
-// Codes and scales do not depend on earlier kernels: the first steps' loads
-// are issued before griddepcontrol.wait; the activations (and therefore the
-// tables) only after it.  A NaN output row (invalid byte, bad padding, bad
-// scale) is rescanned for its error bits.
+// K slices.  Row j of a cluster round belongs to rank j mod CS; each warp
+// stores the partial of its slice straight into the owner's shared memory
+// (st.shared::cluster), and after one cluster barrier per round the owner
+// adds the CS partials in rank order and writes Y.
+//
+// Ordering.  Codes and scales do not depend on earlier kernels: the first
+// steps' loads and the constant parts of the tables (the masking columns,
+// the invalid-byte rows) are issued before griddepcontrol.wait; the
+// activations, and therefore the table values, only after it.  A NaN output
+// row (invalid byte, bad padding, bad scale) is rescanned for its error bits.
 #include <cooperative_groups.h>
 
 #include <cstdio>
@@ -65,9 +76,11 @@ constexpr uint32_t kLsBlockBytes = 0x10000u; // one block: 256 entry rows x 64 s
 constexpr uint32_t kLsSmemBytes = 0x30000u;  // dynamic request: covers [base, 0x30000) for any base <= 0x10000
 constexpr int kLsSliceCols = 512;            // K columns per CTA
 constexpr int kLsSliceBytes = 104;           // their code bytes (G = 64 or 128)
-constexpr int kLsRound = 6144;               // rows per cluster round (partials in shared memory)
+constexpr int kLsRound = 4096;               // rows per cluster round (partials in shared memory)
 constexpr int kLsFreeBank = 26;              // banks 26..31: all-zero columns for masked lookups
 constexpr int kLsChunkRows = 32;             // rows per warp chunk
+constexpr int kLsScaleStride = 36;           // floats per group in a warp's scale block
+static_assert(kLsThreads == kLsSliceCols, "one thread per activation of the slice");
 
 template <int G>
 struct LsCfg;
@@ -88,14 +101,20 @@ struct LsCfg<64> {
     static constexpr int U = 16;
 };
 
-// shared memory below the tables: per-warp decoded scales, then the partial rows
+// Shared memory below the tables: per-warp decoded scales of a chunk (stored
+// group-major, and within a group in step order for each row of the step,
+// kLsScaleStride floats per group so that the float4 reads of lanes of
+// different groups and rows land in different banks), then two buffers of
+// partial rows (CS slots of kLsRound / CS rows each, alternating by round),
+// then the slice's activations in fp32.
+constexpr int kLsPartFloats = kLsRound + 8;
 template <int G>
 __host__ __device__ constexpr uint32_t ls_scale_bytes() {
-    return (uint32_t)kLsWarps * kLsChunkRows * LsCfg<G>::GPS * 4;
+    return (uint32_t)kLsWarps * LsCfg<G>::GPS * kLsScaleStride * 4;
 }
 template <int G>
 __host__ __device__ constexpr uint32_t ls_misc_bytes() {
-    return ls_scale_bytes<G>() + (uint32_t)kLsRound * 4;
+    return ls_scale_bytes<G>() + 2u * kLsPartFloats * 4 + (uint32_t)kLsSliceCols * 4;
 }
 
 struct LsArgs {
@@ -103,8 +122,7 @@ struct LsArgs {
     const uint8_t* codes;
     const uint16_t* scales;
     int64_t N;
-    int K, ng, CS;
-    int64_t row_bytes;
+    int K, CS;
     int64_t rows_per_cluster;
     void* Y;
     int y_bf16;
@@ -124,8 +142,9 @@ __device__ __forceinline__ int ls_slot_position(int block, int sub, int bank) {
 
 // Per-lane constants: offset of the lane's word in the slice, the row within
 // the step, the lane's group in the slice and the PRMT source words of its
-// lookups: lb[i] = {slot offset (4 x bank) of step 2i, of step 2i + 1, 0,
-// window base >> 24}.
+// lookups: lb[i] = {slot offset of lookup 2i (4 x bank), of lookup 2i + 1
+// (128 + 4 x bank: the upper slots), table block of both (bits 16..23 of the
+// address), window base >> 24}.
 struct LsLane {
     uint32_t wofs;
     int h, grp;
@@ -135,7 +154,10 @@ struct LsLane {
 template <int G>
 __device__ __forceinline__ LsLane ls_lane(int lane, uint32_t win_base) {
     LsLane L{};
-    for (int i = 0; i < 4; ++i) L.lb[i] = win_base & 0xFF000000u;
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t block = G == 128 ? (uint32_t)(i & 1) : (uint32_t)i;  // lookups 2i, 2i + 1
+        L.lb[i] = (win_base & 0xFF000000u) | (((kLsTableAbs + block * kLsBlockBytes) >> 16) << 16) | 0x8000u;
+    }
     if constexpr (G == 128) {
         const int h = lane >> 4, q = lane & 15;
         const int w = q < 13 ? q : 3 * (q - 12);  // copies of the straddling words 3, 6, 9
@@ -189,6 +211,16 @@ __device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
     return v;
 }
 
+// One lookup: the whole shared-memory address from one PRMT -- byte K mod 4
+// of word `a` as bits 8..15, the slot byte K mod 2 of `lb` as bits 0..7 and
+// bytes 2, 3 of `lb` (table block, window base) above.
+template <int G, int K>
+__device__ __forceinline__ float ls_lookup(uint32_t a, uint32_t lb) {
+    constexpr uint32_t kk = (uint32_t)(K & 3);
+    constexpr uint32_t sel = 0x7600u | (kk << 4) | (4u + (uint32_t)(K & 1));
+    return lds_imm<0>(prmt32(a, lb, sel));
+}
+
 // Decoded scale as the matmul uses it: fp32 of RNE_bf16(binary16 s); NaN for
 // a rejected scale (sign bit set, Inf or NaN: every pattern >= 0x7C00).
 __device__ __forceinline__ float ls_scale(uint32_t s) {
@@ -197,50 +229,97 @@ __device__ __forceinline__ float ls_scale(uint32_t s) {
 }
 
 // Transposing butterfly within aligned groups of NV lanes (NV = 16 or 32):
-// on exit lane l holds the sum over its group of v[l mod NV].
+// on exit lane l holds the sum over its group of v[l mod NV].  The adds of a
+// level run in packed pairs; each is the same single fp32 add as unpacked.
 template <int NV>
 __device__ __forceinline__ float ls_transpose_reduce(float (&v)[NV], int lane) {
 #pragma unroll
     for (int n = NV / 2; n >= 1; n >>= 1) {
         const bool upper = (lane & n) != 0;
+        float keep[NV / 2], recv[NV / 2];
 #pragma unroll
         for (int i = 0; i < n; ++i) {
-            const float keep = upper ? v[n + i] : v[i];
-            const float send = upper ? v[i] : v[n + i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, n);
+            keep[i] = upper ? v[n + i] : v[i];
+            recv[i] = __shfl_xor_sync(0xffffffffu, upper ? v[i] : v[n + i], n);
+        }
+        if (n >= 2) {
+#pragma unroll
+            for (int i = 0; i < n; i += 2) {
+                const float2 r = f2_unpack(f2_add(f2_pack(keep[i], keep[i + 1]), f2_pack(recv[i], recv[i + 1])));
+                v[i] = r.x;
+                v[i + 1] = r.y;
+            }
+        } else {
+            v[0] = keep[0] + recv[0];
         }
     }
     return v[0];
 }
 
-// One lookup: byte K mod 4 of word `a` as bits 8..15, the slot byte K mod 2
-// of `lb` as bits 0..7, byte 2 of `lb` (0) and its byte 3 (the window base)
-// above; the block and the upper slots in the immediate offset.
-template <int G, int K>
-__device__ __forceinline__ float ls_lookup(uint32_t a, uint32_t lb) {
-    constexpr uint32_t kk = (uint32_t)(K & 3);
-    constexpr uint32_t sel = 0x7600u | (kk << 4) | (4u + (uint32_t)(K & 1));
-    constexpr uint32_t block = G == 128 ? (uint32_t)((K & 3) >> 1) : (uint32_t)(K >> 1);
-    constexpr uint32_t imm = kLsTableAbs + block * kLsBlockBytes + 128u * (uint32_t)(K & 1);
-    return lds_imm<imm>(prmt32(a, lb, sel));
+// Code word of one lane and step.
+template <int G>
+using LsWord = typename std::conditional<G == 128, uint2, uint32_t>::type;
+template <int G>
+__device__ __forceinline__ LsWord<G> ls_load(const uint8_t* p) {
+    if constexpr (G == 128) return ldg_nc_u2(p);
+    else return ldg_nc_u32(p);
 }
 
+// The scaled sums of two steps' code words (wa, wb), side by side:
+// ((t0+t1)+(t2+t3)) + ((t4+t5)+(t6+t7)) per step, times the step's scale.
 template <int G>
+__device__ __forceinline__ float2 ls_two_steps(const LsWord<G>& wa, const LsWord<G>& wb, const LsLane& L,
+                                               float sca, float scb) {
+    if constexpr (G == 128) {
+        const uint32_t a0 = L.h ? wa.y : wa.x, a1 = L.h ? wa.x : wa.y;
+        const uint32_t b0 = L.h ? wb.y : wb.x, b1 = L.h ? wb.x : wb.y;
+        const uint64_t p0 = f2_pack(ls_lookup<G, 0>(a0, L.lb[0]), ls_lookup<G, 0>(b0, L.lb[0]));
+        const uint64_t p1 = f2_pack(ls_lookup<G, 1>(a0, L.lb[0]), ls_lookup<G, 1>(b0, L.lb[0]));
+        const uint64_t p2 = f2_pack(ls_lookup<G, 2>(a0, L.lb[1]), ls_lookup<G, 2>(b0, L.lb[1]));
+        const uint64_t p3 = f2_pack(ls_lookup<G, 3>(a0, L.lb[1]), ls_lookup<G, 3>(b0, L.lb[1]));
+        const uint64_t p4 = f2_pack(ls_lookup<G, 4>(a1, L.lb[2]), ls_lookup<G, 4>(b1, L.lb[2]));
+        const uint64_t p5 = f2_pack(ls_lookup<G, 5>(a1, L.lb[2]), ls_lookup<G, 5>(b1, L.lb[2]));
+        const uint64_t p6 = f2_pack(ls_lookup<G, 6>(a1, L.lb[3]), ls_lookup<G, 6>(b1, L.lb[3]));
+        const uint64_t p7 = f2_pack(ls_lookup<G, 7>(a1, L.lb[3]), ls_lookup<G, 7>(b1, L.lb[3]));
+        const uint64_t lo = f2_add(f2_add(p0, p1), f2_add(p2, p3));
+        const uint64_t hi = f2_add(f2_add(p4, p5), f2_add(p6, p7));
+        return f2_unpack(f2_mul(f2_add(lo, hi), f2_pack(sca, scb)));
+    } else {
+        const uint64_t p0 = f2_pack(ls_lookup<G, 0>(wa, L.lb[0]), ls_lookup<G, 0>(wb, L.lb[0]));
+        const uint64_t p1 = f2_pack(ls_lookup<G, 1>(wa, L.lb[0]), ls_lookup<G, 1>(wb, L.lb[0]));
+        const uint64_t p2 = f2_pack(ls_lookup<G, 2>(wa, L.lb[1]), ls_lookup<G, 2>(wb, L.lb[1]));
+        const uint64_t p3 = f2_pack(ls_lookup<G, 3>(wa, L.lb[1]), ls_lookup<G, 3>(wb, L.lb[1]));
+        return f2_unpack(f2_mul(f2_add(f2_add(p0, p1), f2_add(p2, p3)), f2_pack(sca, scb)));
+    }
+}
+
+__device__ __forceinline__ void st_cluster_f32(uint32_t local_addr, int rank, float v) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+
+template <int G, int CS>
 __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const LsArgs a) {
     using C = LsCfg<G>;
+    using Word = LsWord<G>;
     constexpr int SPC = C::SPC, U = C::U, RPS = C::RPS, GPS = C::GPS;
-    using Word = typename std::conditional<G == 128, uint2, uint32_t>::type;
+    constexpr int64_t RB = (int64_t)CS * kLsSliceBytes;  // code bytes per row
+    constexpr int NG = CS * GPS;                         // groups per row
+    constexpr int64_t STEP = RPS * RB;                   // code bytes between a lane's consecutive steps
+    constexpr int PS = (kLsRound + CS - 1) / CS;         // partial rows per rank slot
+    static_assert(U % 2 == 0 && SPC % U == 0, "steps run in pairs; the load ring divides a chunk");
+    static_assert(CS * PS <= kLsPartFloats, "partial buffer");
     extern __shared__ __align__(16) unsigned char smem[];
-    cg::cluster_group cluster = cg::this_cluster();
-    const int crank = (int)cluster.block_rank();
-    const int cid = (int)(blockIdx.x / (unsigned)a.CS);
+    const int crank = (int)cg::this_cluster().block_rank();
+    const int cid = (int)(blockIdx.x / (unsigned)CS);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // Shared-memory window (base: the top byte of the dynamic region's
     // address, the CTA's rank in the cluster): the tables at offsets
-    // [0x10000, 0x30000), the scales and partials just below 0x10000.
+    // [0x10000, 0x30000), the scales, partials and activations just below.
     const uint32_t dyn = (uint32_t)__cvta_generic_to_shared(smem);
     const uint32_t wbase = dyn & 0xFF000000u, doff = dyn - wbase;
     const uint32_t misc = kLsTableAbs - ls_misc_bytes<G>();
@@ -248,21 +327,45 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
         if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
         return;
     }
-    float* ssc_all = reinterpret_cast<float*>(smem + (misc - doff));
+    // peers store partial rows into this CTA only after the matching wait
+    cluster_arrive_relaxed();
+    float* ssc = reinterpret_cast<float*>(smem + (misc - doff)) + warp * GPS * kLsScaleStride;
     float* part = reinterpret_cast<float*>(smem + (misc - doff) + ls_scale_bytes<G>());
-    float* ssc = ssc_all + warp * kLsChunkRows * GPS;
+    float* xs = part + 2 * kLsPartFloats;
+    const uint32_t part_sa = (uint32_t)__cvta_generic_to_shared(part);
     const uint32_t tabs = wbase + kLsTableAbs;  // the tables, for the stores of the build
+    const float nan = __uint_as_float(0x7FC00000u);
+
+    // constant parts of the tables: the masking columns (banks 26..31) and
+    // the invalid-byte rows 243..255 (NaN in the table columns)
+    for (int it = warp; it < 36; it += kLsWarps) {
+        if (lane >= kLsFreeBank) {
+            const int bs = it / 9, d34 = it - 9 * bs;
+            const uint32_t base = tabs + (bs >> 1) * kLsBlockBytes + 27u * d34 * 256u + 4u * (uint32_t)(lane + 32 * (bs & 1));
+#pragma unroll
+            for (int e = 0; e < 27; ++e) sts_f32(base + 256u * e, 0.f);
+        }
+    }
+    for (int it = warp; it < 4; it += kLsWarps) {
+        const uint32_t base = tabs + (it >> 1) * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * (it & 1));
+        const float v = lane < kLsFreeBank ? nan : 0.f;
+#pragma unroll
+        for (int b = 243; b < 256; ++b) sts_f32(base + 256u * b, v);
+    }
 
     const LsLane L = ls_lane<G>(lane, wbase);
     const int64_t crow0 = (int64_t)cid * a.rows_per_cluster;
     const int64_t crow1 = min(a.N, crow0 + a.rows_per_cluster);
     const uint8_t* cbase = a.codes + (int64_t)crank * kLsSliceBytes + L.wofs;
     const uint16_t* sbase = a.scales + (int64_t)crank * GPS;
-    const uint32_t ssc_lane = (uint32_t)__cvta_generic_to_shared(ssc) + 4u * (uint32_t)(L.h * GPS + L.grp);
+    // this lane's scales in the warp's block: group L.grp, row L.h of each step, steps in order
+    const float4* ssc_lane = reinterpret_cast<const float4*>(ssc + L.grp * kLsScaleStride + (RPS == 2 ? 16 * L.h : 0));
+    const int res_row = G == 128 ? 2 * (lane & 15) + (lane >> 4) : lane;  // row of the reduced value, in the chunk
     uint32_t err_acc = 0;
     bool tables_built = false;
+    int round = 0;
 
-    for (int64_t rr0 = crow0; rr0 < crow1; rr0 += kLsRound) {
+    for (int64_t rr0 = crow0; rr0 < crow1; rr0 += kLsRound, ++round) {
         const int nround = (int)(crow1 - rr0 < (int64_t)kLsRound ? crow1 - rr0 : (int64_t)kLsRound);
         // this warp's rows of the round
         int per = (nround + kLsWarps - 1) / kLsWarps;
@@ -272,21 +375,19 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
         const int64_t wr0 = rr0 + wlo;
         const int T = (nr + RPS - 1) / RPS;
         const int nch = (T + SPC - 1) / SPC;
+        const uint32_t pbuf = part_sa + (uint32_t)(round & 1) * kLsPartFloats * 4u;
 
-        auto code_ptr = [&](int t) -> const uint8_t* {
+        // code word of step t, the row clamped to the warp's last
+        auto load_clamped = [&](int t) -> Word {
             int r = RPS * t + L.h;
             r = r < nr ? r : nr - 1;
-            return cbase + (wr0 + r) * a.row_bytes;
-        };
-        auto load_code = [&](int t) -> Word {
-            if constexpr (G == 128) return ldg_nc_u2(code_ptr(t));
-            else return ldg_nc_u32(code_ptr(t));
+            return ls_load<G>(cbase + (wr0 + r) * RB);
         };
         using SRaw = typename std::conditional<G == 128, uint2, uint4>::type;
         auto load_scales = [&](int ch) -> SRaw {
             int r = ch * kLsChunkRows + lane;
             r = r < nr ? r : nr - 1;
-            const uint16_t* p = sbase + (wr0 + r) * a.ng;
+            const uint16_t* p = sbase + (wr0 + r) * NG;
             if constexpr (G == 128) return __ldg(reinterpret_cast<const uint2*>(p));
             else return __ldg(reinterpret_cast<const uint4*>(p));
         };
@@ -295,145 +396,139 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
         SRaw sraw{};
         if (nr > 0) {
 #pragma unroll
-            for (int u = 0; u < U; ++u)
-                if (u < T) cb[u] = load_code(u);
+            for (int u = 0; u < U; ++u) cb[u] = load_clamped(u);
             sraw = load_scales(0);
         }
 
         if (!tables_built) {
             // Activations come from the preceding kernel: everything above ran
-            // before this wait.
+            // before this wait.  One coalesced read of the slice's 512
+            // activations (every CTA of the grid reads the same 1 KB, so the
+            // per-entry reads of the build go to shared memory).
             asm volatile("griddepcontrol.wait;" ::: "memory");
-            const int col_base = crank * kLsSliceCols;
-            const float nan = __uint_as_float(0x7FC00000u);
+            xs[threadIdx.x] = __uint_as_float((uint32_t)__ldcg(a.X + crank * kLsSliceCols + threadIdx.x) << 16);
+            __syncthreads();
             // warp item (block, sub, d3 + 3 d4): the 27 entries b = d0 + 3 d1 + 9 d2 + 27 (d3 + 3 d4)
             // of one table row per lane (lane = bank)
             for (int it = warp; it < 36; it += kLsWarps) {
-                const int bs = it / 9, d34 = it - 9 * bs;
-                const int block = bs >> 1, sub = bs & 1;
-                const uint32_t base = tabs + block * kLsBlockBytes + 27u * d34 * 256u +
-                                      4u * (uint32_t)(lane + 32 * sub);
-                if (lane >= kLsFreeBank) {
+                if (lane < kLsFreeBank) {
+                    const int bs = it / 9, d34 = it - 9 * bs;
+                    const int block = bs >> 1, sub = bs & 1;
+                    const uint32_t base = tabs + block * kLsBlockBytes + 27u * d34 * 256u +
+                                          4u * (uint32_t)(lane + 32 * sub);
+                    const int p = ls_slot_position<G>(block, sub, lane);
+                    const int g = p / C::B, j = p - g * C::B;
+                    const int real = min(5, G - 5 * j);
+                    const float* xp = xs + g * G + 5 * j;
+                    float x[5];
 #pragma unroll
-                    for (int e = 0; e < 27; ++e) sts_f32(base + 256u * e, 0.f);
-                    continue;
-                }
-                const int p = ls_slot_position<G>(block, sub, lane);
-                const int g = p / C::B, j = p - g * C::B;
-                const int real = min(5, G - 5 * j);
-                const uint16_t* xp = a.X + col_base + g * G + 5 * j;
-                float x[5];
+                    for (int i = 0; i < 5; ++i) x[i] = i < real ? xp[i] : 0.f;
+                    const int d3 = d34 % 3, d4 = d34 / 3;
+                    const bool bad34 = (3 >= real && d3 != 1) || (4 >= real && d4 != 1);
+                    const float h34 = bad34 ? nan : (float)(d3 - 1) * x[3] + (float)(d4 - 1) * x[4];
+                    float P[9];
 #pragma unroll
-                for (int i = 0; i < 5; ++i) x[i] = i < real ? __uint_as_float((uint32_t)__ldcg(xp + i) << 16) : 0.f;
-                const int d3 = d34 % 3, d4 = d34 / 3;
-                const bool bad34 = (3 >= real && d3 != 1) || (4 >= real && d4 != 1);
-                const float h34 = bad34 ? nan : (float)(d3 - 1) * x[3] + (float)(d4 - 1) * x[4];
-                float P[9];
+                    for (int d1 = 0; d1 < 3; ++d1)
 #pragma unroll
-                for (int d1 = 0; d1 < 3; ++d1)
+                        for (int d0 = 0; d0 < 3; ++d0) {
+                            const bool bad = (1 >= real && d1 != 1) || (0 >= real && d0 != 1);
+                            P[d0 + 3 * d1] = bad ? nan : (float)(d0 - 1) * x[0] + (float)(d1 - 1) * x[1];
+                        }
 #pragma unroll
-                    for (int d0 = 0; d0 < 3; ++d0) {
-                        const bool bad = (1 >= real && d1 != 1) || (0 >= real && d0 != 1);
-                        P[d0 + 3 * d1] = bad ? nan : (float)(d0 - 1) * x[0] + (float)(d1 - 1) * x[1];
+                    for (int d2 = 0; d2 < 3; ++d2) {
+                        const bool bad2 = 2 >= real && d2 != 1;
+                        const float q2 = bad2 ? nan : h34 + (float)(d2 - 1) * x[2];
+#pragma unroll
+                        for (int e = 0; e < 9; ++e) sts_f32(base + 256u * (9 * d2 + e), P[e] + q2);
                     }
-#pragma unroll
-                for (int d2 = 0; d2 < 3; ++d2) {
-                    const bool bad2 = 2 >= real && d2 != 1;
-                    const float q2 = bad2 ? nan : h34 + (float)(d2 - 1) * x[2];
-#pragma unroll
-                    for (int e = 0; e < 9; ++e) sts_f32(base + 256u * (9 * d2 + e), P[e] + q2);
                 }
-            }
-            // entry rows 243..255: NaN (invalid bytes) in table columns, 0 in the free ones
-            for (int it = warp; it < 4; it += kLsWarps) {
-                const int block = it >> 1, sub = it & 1;
-                const uint32_t base = tabs + block * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * sub);
-                const float v = lane < kLsFreeBank ? nan : 0.f;
-#pragma unroll
-                for (int b = 243; b < 256; ++b) sts_f32(base + 256u * b, v);
             }
             __syncthreads();
+            cluster_wait();  // every CTA of the cluster runs: partials may be stored into peers
             tables_built = true;
         }
 
-        for (int ch = 0; ch < nch; ++ch) {
-            // decoded scales of this chunk's 32 rows: lane = row
+        // Chunk ch of the warp.  WALK: every load the chunk issues (U steps
+        // ahead) stays inside the matrix, so the loads walk one pointer with
+        // immediate offsets (rows past the warp's own are read and their
+        // results never stored); otherwise each load is clamped to the warp's
+        // last row.
+        const uint8_t* lp = cbase + (wr0 + RPS * U + L.h) * RB;
+        auto run_chunk = [&](int ch, auto walk_tag) {
+            constexpr bool WALK = decltype(walk_tag)::value;
+            // decoded scales of this chunk's 32 rows (lane = row), stored by group
             {
                 const uint32_t* sw = reinterpret_cast<const uint32_t*>(&sraw);
-                float4* dst = reinterpret_cast<float4*>(ssc + lane * GPS);
+                const int col = RPS == 2 ? 16 * (lane & 1) + (lane >> 1) : lane;
 #pragma unroll
-                for (int q = 0; q < GPS / 4; ++q)
-                    dst[q] = make_float4(ls_scale(sw[2 * q] & 0xFFFFu), ls_scale(sw[2 * q] >> 16),
-                                         ls_scale(sw[2 * q + 1] & 0xFFFFu), ls_scale(sw[2 * q + 1] >> 16));
+                for (int g = 0; g < GPS; ++g)
+                    ssc[g * kLsScaleStride + col] = ls_scale(g & 1 ? sw[g >> 1] >> 16 : sw[g >> 1] & 0xFFFFu);
                 if (ch + 1 < nch) sraw = load_scales(ch + 1);
                 __syncwarp();
             }
             float v[SPC];
+            float4 sc4;
 #pragma unroll
-            for (int s = 0; s < SPC; ++s) {
-                const int t = ch * SPC + s;
-                const Word cw = cb[s % U];
-                if (t + U < T) cb[s % U] = load_code(t + U);
-                if (t < T) {
-                    float sc;
-                    asm volatile("ld.shared.f32 %0, [%1];"
-                                 : "=f"(sc)
-                                 : "r"(ssc_lane + 4u * (uint32_t)(RPS * s * GPS)));
-                    if constexpr (G == 128) {
-                        const uint32_t w0 = L.h ? cw.y : cw.x;
-                        const uint32_t w1 = L.h ? cw.x : cw.y;
-                        const float t0 = ls_lookup<G, 0>(w0, L.lb[0]);
-                        const float t1 = ls_lookup<G, 1>(w0, L.lb[0]);
-                        const float t2 = ls_lookup<G, 2>(w0, L.lb[1]);
-                        const float t3 = ls_lookup<G, 3>(w0, L.lb[1]);
-                        const float t4 = ls_lookup<G, 4>(w1, L.lb[2]);
-                        const float t5 = ls_lookup<G, 5>(w1, L.lb[2]);
-                        const float t6 = ls_lookup<G, 6>(w1, L.lb[3]);
-                        const float t7 = ls_lookup<G, 7>(w1, L.lb[3]);
-                        v[s] = (((t0 + t1) + (t2 + t3)) + ((t4 + t5) + (t6 + t7))) * sc;
-                    } else {
-                        const float t0 = ls_lookup<G, 0>(cw, L.lb[0]);
-                        const float t1 = ls_lookup<G, 1>(cw, L.lb[0]);
-                        const float t2 = ls_lookup<G, 2>(cw, L.lb[1]);
-                        const float t3 = ls_lookup<G, 3>(cw, L.lb[1]);
-                        v[s] = ((t0 + t1) + (t2 + t3)) * sc;
-                    }
+            for (int s = 0; s < SPC; s += 2) {
+                const Word wa = cb[s % U], wb = cb[(s + 1) % U];
+                if constexpr (WALK) {
+                    cb[s % U] = ls_load<G>(lp + s * STEP);
+                    cb[(s + 1) % U] = ls_load<G>(lp + (s + 1) * STEP);
                 } else {
-                    v[s] = 0.f;
+                    cb[s % U] = load_clamped(ch * SPC + s + U);
+                    cb[(s + 1) % U] = load_clamped(ch * SPC + s + 1 + U);
                 }
+                if (s % 4 == 0) sc4 = ssc_lane[s / 4];
+                const float2 r = s % 4 == 0 ? ls_two_steps<G>(wa, wb, L, sc4.x, sc4.y)
+                                            : ls_two_steps<G>(wa, wb, L, sc4.z, sc4.w);
+                v[s] = r.x;
+                v[s + 1] = r.y;
             }
+            if constexpr (WALK) lp += SPC * STEP;
             __syncwarp();  // this chunk's scales are consumed before the next chunk rewrites them
             const float tot = ls_transpose_reduce<SPC>(v, lane);
-            const int r = ch * kLsChunkRows + (G == 128 ? 2 * (lane & 15) + (lane >> 4) : lane);
-            if (r < nr) part[wlo + r] = tot;
-        }
+            const int r = ch * kLsChunkRows + res_row;
+            if (r < nr) {
+                const int j = wlo + r;  // row within the round: owner rank j mod CS, slot j / CS
+                st_cluster_f32(pbuf + 4u * (uint32_t)(crank * PS + j / CS), j % CS, tot);
+            }
+        };
+        // chunk ch walks while its last load, row wr0 + RPS ((ch + 1) SPC + U) - 1, is below N
+        const int64_t walk_rows = a.N - wr0 - (int64_t)RPS * U;
+        int ch = 0;
+        for (; ch < nch && (int64_t)RPS * (ch + 1) * SPC <= walk_rows; ++ch) run_chunk(ch, std::true_type{});
+        for (; ch < nch; ++ch) run_chunk(ch, std::false_type{});
 
-        // K slices: every rank's partial rows are complete and visible, then
-        // rank q adds the ranks' partials of its share of rows in rank order.
-        __syncthreads();
-        cluster.sync();
-        const int share = (nround + a.CS - 1) / a.CS;
-        const int lo = min(nround, crank * share), hi = min(nround, lo + share);
-        for (int r = lo + (int)threadIdx.x; r < hi; r += kLsThreads) {
+        // K slices: every rank's partials of the round are stored, then each
+        // rank adds the partials of its rows (j = crank mod CS) in rank order.
+        cluster_arrive();
+        cluster_wait();
+        const int own = (nround - crank + CS - 1) / CS;
+        const float* pb = reinterpret_cast<const float*>(smem + (misc - doff) + ls_scale_bytes<G>()) +
+                          (round & 1) * kLsPartFloats;
+        for (int i = (int)threadIdx.x; i < own; i += kLsThreads) {
             float y = 0.f;
-            for (int q = 0; q < a.CS; ++q) y += *cluster.map_shared_rank(part + r, q);
-            const int64_t n = rr0 + r;
+#pragma unroll
+            for (int q = 0; q < CS; ++q) y += pb[q * PS + i];
+            const int64_t n = rr0 + crank + (int64_t)CS * i;
             if (y != y)
-                err_acc |= scan_row_errors(a.codes + n * a.row_bytes, a.scales + n * a.ng, a.ng, G, C::B);
+                err_acc |= scan_row_errors(a.codes + n * RB, a.scales + n * NG, NG, G, C::B);
             if (a.y_bf16) reinterpret_cast<__nv_bfloat16*>(a.Y)[n] = __float2bfloat16_rn(y);
             else reinterpret_cast<float*>(a.Y)[n] = y;
         }
-        cluster.sync();  // the peers are done reading this CTA's partials
     }
-    if (!tables_built) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!tables_built) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        cluster_wait();
+    }
     if (err_acc && a.d_err) atomicOr(a.d_err, err_acc);
 }
 
-template <int G>
+template <int G, int CS>
 cudaError_t launch_ls(const LsArgs& a0, cudaStream_t stream, int sm_count) {
-    auto kern = gemv_lut_stream_kernel<G>;
+    auto kern = gemv_lut_stream_kernel<G, CS>;
     static SmemAttr smem_attr;
-    static int max_clusters[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+    static int max_clusters = 0;
     static std::mutex mu;
     if (cudaError_t e = smem_attr.ensure(kern, (int)kLsSmemBytes)) return e;
     LsArgs a = a0;
@@ -443,7 +538,7 @@ cudaError_t launch_ls(const LsArgs& a0, cudaStream_t stream, int sm_count) {
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = a.CS;
+    attr[0].val.clusterDim.x = CS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -453,24 +548,39 @@ cudaError_t launch_ls(const LsArgs& a0, cudaStream_t stream, int sm_count) {
     int ncl;
     {
         std::lock_guard<std::mutex> lk(mu);
-        if (max_clusters[a.CS] == 0) {
-            cfg.gridDim = dim3((unsigned)(a.CS * (sm_count / a.CS)));
+        if (max_clusters == 0) {
+            cfg.gridDim = dim3((unsigned)(CS * (sm_count / CS)));
             int n = 0;
             cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
             if (e != cudaSuccess) return e;
-            max_clusters[a.CS] = n > 0 ? n : 1;
+            max_clusters = n > 0 ? n : 1;
         }
-        ncl = max_clusters[a.CS];
+        ncl = max_clusters;
     }
     const int64_t want = (a.N + 63) / 64;  // at least 64 rows per cluster
     if (want < ncl) ncl = (int)(want < 1 ? 1 : want);
     a.rows_per_cluster = (a.N + ncl - 1) / ncl;
-    cfg.gridDim = dim3((unsigned)(ncl * a.CS));
+    cfg.gridDim = dim3((unsigned)(ncl * CS));
     static const bool debug = getenv("TQ_DEBUG_PLAN") != nullptr;
     if (debug)
         fprintf(stderr, "tq gemv_lut_stream N=%lld K=%d G=%d: CS=%d clusters=%d rows/cluster=%lld\n",
-                (long long)a.N, a.K, G, a.CS, ncl, (long long)a.rows_per_cluster);
+                (long long)a.N, a.K, G, CS, ncl, (long long)a.rows_per_cluster);
     return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <int G>
+cudaError_t launch_ls_cs(const LsArgs& a, cudaStream_t stream, int sm_count) {
+    switch (a.CS) {
+        case 1: return launch_ls<G, 1>(a, stream, sm_count);
+        case 2: return launch_ls<G, 2>(a, stream, sm_count);
+        case 3: return launch_ls<G, 3>(a, stream, sm_count);
+        case 4: return launch_ls<G, 4>(a, stream, sm_count);
+        case 5: return launch_ls<G, 5>(a, stream, sm_count);
+        case 6: return launch_ls<G, 6>(a, stream, sm_count);
+        case 7: return launch_ls<G, 7>(a, stream, sm_count);
+        case 8: return launch_ls<G, 8>(a, stream, sm_count);
+        default: return cudaErrorNotSupported;
+    }
 }
 
 }  // namespace
@@ -490,13 +600,11 @@ cudaError_t launch_gemv_lut_stream(const uint16_t* X, int64_t M, const uint8_t* 
     a.scales = scales;
     a.N = N;
     a.K = (int)K;
-    a.ng = (int)(K / G);
     a.CS = (int)(K / kLsSliceCols);
-    a.row_bytes = (int64_t)a.ng * bytes_per_group(G);
     a.Y = Y;
     a.y_bf16 = y_bf16;
     a.d_err = d_err;
-    return G == 128 ? launch_ls<128>(a, stream, sm_count) : launch_ls<64>(a, stream, sm_count);
+    return G == 128 ? launch_ls_cs<128>(a, stream, sm_count) : launch_ls_cs<64>(a, stream, sm_count);
 }
 
 }  // namespace tq
