@@ -345,6 +345,7 @@ def run_ours(args, rank, world, local):
         results["prefill"] = bench_prefill(tq, args, world, peaks)
         results["msweep"] = bench_msweep(tq, args, world, peaks)
         results["ternary2"] = bench_ternary2(tq, args, world, peaks)
+        results["w4"] = bench_w4(tq, args, world, peaks)
     clk = clocks.summary()
 
     ms_step = ms / K_steps
@@ -401,6 +402,7 @@ def run_ours(args, rank, world, local):
         "prefill_gemm": results["prefill"],
         "msweep": results["msweep"],
         "ternary2": results["ternary2"],
+        "w4": results["w4"],
     }
     print(json.dumps(line), flush=True)
 
@@ -454,33 +456,64 @@ def count_launches(obj) -> int:
     return 0
 
 
-def bench_gemv_stream(tq, args, world, peaks):
-    """One GEMV over the 24-layer gate/up stack as a single [172032 x 1024]
-    matrix (G=128, M=1): the streaming rate without launch gaps.  Four packed
-    copies (154 MB together, more than the 126 MB L2) are used in turn."""
+def graph_launch_us(launches, rounds, args, world):
+    """Capture `rounds` passes over `launches` (one kernel launch each) in one
+    CUDA graph and time its replays: microseconds per launch with launches
+    back to back (programmatic dependency edges between them), not limited
+    by the Python dispatcher."""
     import torch
-    N, K, G = 48 * 3584, 1024, 128
-    packs = []
-    for c in range(4):
-        W = device_weights(N, K, seed=77 + c)
-        packs.append(tq.quantize_pack(W, G))
-        del W
-    X = device_acts(1, K, seed=78)
-    Y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
-    reps = 4 * max(2, args.steps // 4)
-    state = {"i": 0}
+    for f in launches:
+        f()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+        for _ in range(rounds):
+            for f in launches:
+                f()
+    steps = max(3, args.steps)
+    ms = timed(graph.replay, steps, max(3, args.warmup), world)
+    del graph
+    return ms * 1e3 / (steps * rounds * len(launches))
 
-    def one():
-        c, s = packs[state["i"] % 4]
-        state["i"] += 1
-        tq.gemv(X, c, s, N, K, G, out=Y)
-    ms = timed(one, reps, max(4, args.warmup), world)
-    byts = packed_bytes(N, K, G) + 2 * K + 2 * N
-    gbs = byts * reps / (ms * 1e-3) / 1e9
-    return {"shape": [N, K], "G": G, "us": round(ms * 1e3 / reps, 2), "GB/s": round(gbs, 1),
-            "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": reps,
-            "kernel": "gemv_lut_stream_kernel<128> (lookup tables of one 512-column slice per CTA, 2-CTA clusters)",
-            "note": "four copies of 38.5 MB used in turn (154 MB > L2)"}
+
+def bench_gemv_stream(tq, args, world, peaks):
+    """One M=1 GEMV over the FFN gate/up projections stacked as one matrix:
+    24 layers, [172032 x 1024], at G=128 (top-level keys) and G=64, four
+    packed copies used in turn (154 and 165 MB, more than the 126 MB L2); and
+    48 layers, [344064 x 1024], G=128, two copies (155 MB).  Launches run
+    back to back from a CUDA graph: the streaming rate of the kernel with its
+    per-launch fixed costs (grid-dependency wait, table build, cluster
+    combine) included."""
+    import torch
+    K = 1024
+    res = {}
+    for layers, G, ncopy in [(24, 128, 4), (24, 64, 4), (48, 128, 2)]:
+        N = layers * 2 * 3584
+        packs = []
+        for c in range(ncopy):
+            W = device_weights(N, K, seed=77 + c)
+            packs.append(tq.quantize_pack(W, G))
+            del W
+        torch.cuda.empty_cache()
+        X = device_acts(1, K, seed=78)
+        Y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+        launches = [lambda c=c, s=s: tq.gemv(X, c, s, N, K, G, out=Y) for c, s in packs]
+        us = graph_launch_us(launches, 16 // ncopy, args, world)
+        byts = packed_bytes(N, K, G) + 2 * K + 2 * N
+        gbs = byts / (us * 1e-6) / 1e9
+        r = {"shape": [N, K], "G": G, "us": round(us, 2), "GB/s": round(gbs, 1),
+             "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": max(3, args.steps) * 16,
+             "kernel": f"gemv_lut_stream_kernel<{G}, 3, 2> (lookup tables of one 512-column slice per CTA, "
+                       "2-CTA clusters)",
+             "note": f"{ncopy} copies of {byts / 1e6:.1f} MB used in turn from one CUDA graph "
+                     f"({ncopy * byts / 1e6:.0f} MB > L2)"}
+        if layers == 24 and G == 128:
+            res.update(r)
+        else:
+            res[f"stack{layers}_G{G}"] = r
+        del packs, launches
+        torch.cuda.empty_cache()
+    return res
 
 
 def bench_gemv_shapes(tq, args, world, peaks):
@@ -645,19 +678,16 @@ def bench_ternary2(tq, args, world, peaks):
         del W
     X = device_acts(1, K, seed=78)
     Y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
-    sreps = 4 * max(2, args.steps // 4)
-    state = {"i": 0}
-
-    def one():
-        c, s = packs[state["i"] % 4]
-        state["i"] += 1
-        tq.gemv2(X, c, s, N, K, G, out=Y)
-    ms = timed(one, sreps, max(4, args.warmup), world)
+    launches = [lambda c=c, s=s: tq.gemv2(X, c, s, N, K, G, out=Y) for c, s in packs]
+    us = graph_launch_us(launches, 4, args, world)
     byts = packed2_bytes(N, K, G) + 2 * K + 2 * N
-    gbs = byts * sreps / (ms * 1e-3) / 1e9
-    res["gemv_stream"] = {"shape": [N, K], "G": G, "us": round(ms * 1e3 / sreps, 2), "GB/s": round(gbs, 1),
-                          "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": sreps,
-                          "kernel": "gemv2_kernel<1, 8>"}
+    gbs = byts / (us * 1e-6) / 1e9
+    res["gemv_stream"] = {"shape": [N, K], "G": G, "us": round(us, 2), "GB/s": round(gbs, 1),
+                          "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": max(3, args.steps) * 16,
+                          "kernel": "gemv_lut_stream_kernel<128, 2, 2> (lookup tables of 2-bit bytes, "
+                                    "one 512-column slice per CTA)",
+                          "note": "four copies used in turn from one CUDA graph"}
+    del launches
     del packs
     torch.cuda.empty_cache()
 
@@ -688,6 +718,83 @@ def bench_ternary2(tq, args, world, peaks):
                            "frac": round(step_bytes / us / 1e3 / peaks["hbm_gbs"], 4),
                            "launches": steps * len(calls), "bytes_per_step": step_bytes}
     del graph, packs2
+    torch.cuda.empty_cache()
+
+    # prefill on the tensor cores with 2-bit codes
+    M, N, K = 4096, 14336, 4096
+    W = device_weights(N, K, seed=904, outliers=False)
+    c2, s2 = tq.quantize_pack2(W, 128)
+    del W
+    X = device_acts(M, K, seed=905)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    tq.gemm2(X, c2, s2, N, K, 128, out=Y)
+    preps = max(3, args.steps // 4)
+    ms = timed_flushed(lambda: tq.gemm2(X, c2, s2, N, K, 128, out=Y), preps, max(3, args.warmup), world)
+    tflops = 2.0 * M * N * K * preps / (ms * 1e-3) / 1e12
+    res["prefill"] = {"M": M, "N": N, "K": K, "G": 128, "us": round(ms * 1e3 / preps, 1),
+                      "TFLOP/s": round(tflops, 1), "frac": round(tflops / peaks["bf16_tflops"], 4), "launches": preps}
+    del c2, s2, X, Y
+    torch.cuda.empty_cache()
+    return res
+
+
+def device_w4_params(N, K, G, seed):
+    """Seeded W4A16 parameters made on the device: uniform 4-bit codes, scale
+    magnitudes 0.004..0.009 with random signs, biases ~ N(0, 0.05) (an affine
+    4-bit quantization of N(0, 0.02) weights over groups of G)."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    codes = torch.randint(-(1 << 31), (1 << 31) - 1, (N, K // 8), generator=g, device="cuda", dtype=torch.int64)
+    codes = codes.to(torch.int32)
+    mag = torch.rand((N, K // G), generator=g, device="cuda") * 0.005 + 0.004
+    sign = torch.where(torch.rand((N, K // G), generator=g, device="cuda") < 0.5, -1.0, 1.0)
+    scales = (mag * sign).to(torch.bfloat16)
+    biases = (torch.randn((N, K // G), generator=g, device="cuda") * 0.05).to(torch.bfloat16)
+    return codes, scales, biases
+
+
+def w4_bytes(N, K, G):
+    return N * K // 2 + 4 * N * (K // G)
+
+
+def bench_w4(tq, args, world, peaks):
+    """The W4A16 affine format (the second weight format): the streaming
+    decode GEMV over the [172032 x 1024] gate/up-shaped stack at G=128 (two
+    copies, 182 MB > L2) and the tensor-core prefill GEMM at M=4096,
+    4096 -> 14336 (L2 flushed before every launch)."""
+    import torch
+    res = {}
+    N, K, G = 48 * 3584, 1024, 128
+    packs = [device_w4_params(N, K, G, seed=300 + c) for c in range(2)]
+    X = device_acts(1, K, seed=301)
+    Y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+    reps = 4 * max(2, args.steps // 4)
+    state = {"i": 0}
+
+    def one():
+        c, s_, b = packs[state["i"] % 2]
+        state["i"] += 1
+        tq.w4_gemv(X, c, s_, b, N, K, G, out=Y)
+    ms = timed(one, reps, max(4, args.warmup), world)
+    gbs = (w4_bytes(N, K, G) + 2 * K + 2 * N) * reps / (ms * 1e-3) / 1e9
+    res["gemv_stream"] = {"shape": [N, K], "G": G, "us": round(ms * 1e3 / reps, 2), "GB/s": round(gbs, 1),
+                          "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": reps,
+                          "kernel": "gemv_w4_kernel<1, 1>"}
+    del packs
+    torch.cuda.empty_cache()
+    M, N, K = 4096, 14336, 4096
+    c, s_, b = device_w4_params(N, K, G, seed=302)
+    X = device_acts(M, K, seed=303)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    tq.w4_gemm(X, c, s_, b, N, K, G, out=Y)
+    preps = max(3, args.steps // 4)
+    ms = timed_flushed(lambda: tq.w4_gemm(X, c, s_, b, N, K, G, out=Y), preps, max(3, args.warmup), world)
+    tflops = 2.0 * M * N * K * preps / (ms * 1e-3) / 1e12
+    res["prefill"] = {"M": M, "N": N, "K": K, "G": G, "us": round(ms * 1e3 / preps, 1), "TFLOP/s": round(tflops, 1),
+                      "frac": round(tflops / peaks["bf16_tflops"], 4), "launches": preps,
+                      "note": "each weight as two bf16 terms: two MMAs per product, so at most half the bf16 rate"}
+    del c, s_, b, X, Y
     torch.cuda.empty_cache()
     return res
 
@@ -865,7 +972,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
-    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv", "msweep", "ternary2"], default=None,
+    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv", "msweep", "ternary2", "w4"], default=None,
                     help="run one sub-benchmark alone and print its result (profiling aid)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -881,7 +988,7 @@ def main():
             torch.cuda.set_device(local)
             peaks = load_peaks()
             fn = {"stream": bench_gemv_stream, "codec": bench_bulk_codec, "prefill": bench_prefill,
-                  "gemv": bench_gemv_shapes, "msweep": bench_msweep, "ternary2": bench_ternary2}
+                  "gemv": bench_gemv_shapes, "msweep": bench_msweep, "ternary2": bench_ternary2, "w4": bench_w4}
             res = fn[args.only](tq, args, world, peaks)
             if rank == 0:
                 print(json.dumps({"only": args.only, "result": res}), flush=True)

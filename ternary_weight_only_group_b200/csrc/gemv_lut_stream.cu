@@ -75,31 +75,41 @@ constexpr uint32_t kLsTableAbs = 0x10000u;   // offset of the tables in the CTA'
 constexpr uint32_t kLsBlockBytes = 0x10000u; // one block: 256 entry rows x 64 slots x 4 B
 constexpr uint32_t kLsSmemBytes = 0x30000u;  // dynamic request: covers [base, 0x30000) for any base <= 0x10000
 constexpr int kLsSliceCols = 512;            // K columns per CTA
-constexpr int kLsSliceBytes = 104;           // their code bytes (G = 64 or 128)
 constexpr int kLsRound = 4096;               // rows per cluster round (partials in shared memory)
 constexpr int kLsFreeBank = 26;              // banks 26..31: all-zero columns for masked lookups
 constexpr int kLsChunkRows = 32;             // rows per warp chunk
 constexpr int kLsScaleStride = 36;           // floats per group in a warp's scale block
 static_assert(kLsThreads == kLsSliceCols, "one thread per activation of the slice");
 
-template <int G>
+// FMT 3: base-3 codes (five digits per byte, 104 bytes per 512 columns);
+// FMT 2: 2-bit codes (four per byte, 128 bytes per 512 columns, groups of
+// 64 or 128 columns are whole 8-byte words).
+template <int G, int FMT>
 struct LsCfg;
 template <>
-struct LsCfg<128> {
+struct LsCfg<128, 3> {
     static constexpr int B = 26;    // code bytes per group
+    static constexpr int SB = 104;  // code bytes per slice
     static constexpr int GPS = 4;   // groups per slice
     static constexpr int RPS = 2;   // rows per warp step
     static constexpr int SPC = 16;  // steps per chunk
     static constexpr int U = 8;     // steps of code loads in flight
 };
 template <>
-struct LsCfg<64> {
-    static constexpr int B = 13;
-    static constexpr int GPS = 8;
-    static constexpr int RPS = 1;
-    static constexpr int SPC = 32;
-    static constexpr int U = 16;
+struct LsCfg<64, 3> {
+    static constexpr int B = 13, SB = 104, GPS = 8, RPS = 1, SPC = 32, U = 8;
 };
+template <>
+struct LsCfg<128, 2> {
+    static constexpr int B = 32, SB = 128, GPS = 4, RPS = 2, SPC = 16, U = 8;
+};
+template <>
+struct LsCfg<64, 2> {
+    static constexpr int B = 16, SB = 128, GPS = 8, RPS = 2, SPC = 16, U = 8;
+};
+// 8-byte code words, two rows per step
+template <int G, int FMT>
+constexpr bool ls_wide() { return LsCfg<G, FMT>::RPS == 2; }
 
 // Shared memory below the tables: per-warp decoded scales of a chunk (stored
 // group-major, and within a group in step order for each row of the step,
@@ -108,13 +118,13 @@ struct LsCfg<64> {
 // partial rows (CS slots of kLsRound / CS rows each, alternating by round),
 // then the slice's activations in fp32.
 constexpr int kLsPartFloats = kLsRound + 8;
-template <int G>
+template <int G, int FMT>
 __host__ __device__ constexpr uint32_t ls_scale_bytes() {
-    return (uint32_t)kLsWarps * LsCfg<G>::GPS * kLsScaleStride * 4;
+    return (uint32_t)kLsWarps * LsCfg<G, FMT>::GPS * kLsScaleStride * 4;
 }
-template <int G>
+template <int G, int FMT>
 __host__ __device__ constexpr uint32_t ls_misc_bytes() {
-    return ls_scale_bytes<G>() + 2u * kLsPartFloats * 4 + (uint32_t)kLsSliceCols * 4;
+    return ls_scale_bytes<G, FMT>() + 2u * kLsPartFloats * 4 + (uint32_t)kLsSliceCols * 4;
 }
 
 struct LsArgs {
@@ -129,14 +139,14 @@ struct LsArgs {
     uint32_t* d_err;
 };
 
-// Table slot of chunk position p of a slice (0 <= p < 104), as the lanes below
-// read it: G = 128: p = 8 w + j -> block (j & 3) >> 1, upper slots j & 1, bank
-// 2 w + (j >> 2); G = 64: p = 4 w + j -> block j >> 1, upper slots j & 1,
-// bank w.  The table build needs the inverse: the position held at (block,
-// sub, bank < 26).
-template <int G>
+// Table slot of chunk position p of a slice (p < 104 base-3, < 128 2-bit), as
+// the lanes below read it: 8-byte words: p = 8 w + j -> block (j & 3) >> 1,
+// upper slots j & 1, bank 2 w + (j >> 2); 4-byte words (base-3, G = 64):
+// p = 4 w + j -> block j >> 1, upper slots j & 1, bank w.  The table build
+// needs the inverse: the position held at (block, sub, bank).
+template <int G, int FMT>
 __device__ __forceinline__ int ls_slot_position(int block, int sub, int bank) {
-    if constexpr (G == 128) return 8 * (bank >> 1) + 4 * (bank & 1) + 2 * block + sub;
+    if constexpr (ls_wide<G, FMT>()) return 8 * (bank >> 1) + 4 * (bank & 1) + 2 * block + sub;
     else return 4 * bank + 2 * block + sub;
 }
 
@@ -151,14 +161,24 @@ struct LsLane {
     uint32_t lb[4];
 };
 
-template <int G>
+template <int G, int FMT>
 __device__ __forceinline__ LsLane ls_lane(int lane, uint32_t win_base) {
     LsLane L{};
     for (int i = 0; i < 4; ++i) {
-        const uint32_t block = G == 128 ? (uint32_t)(i & 1) : (uint32_t)i;  // lookups 2i, 2i + 1
+        const uint32_t block = ls_wide<G, FMT>() ? (uint32_t)(i & 1) : (uint32_t)i;  // lookups 2i, 2i + 1
         L.lb[i] = (win_base & 0xFF000000u) | (((kLsTableAbs + block * kLsBlockBytes) >> 16) << 16) | 0x8000u;
     }
-    if constexpr (G == 128) {
+    if constexpr (FMT == 2) {
+        // 16 words per row, no group straddles a word: every lookup is live
+        const int h = lane >> 4, w = lane & 15;
+        for (int k = 0; k < 8; ++k) {
+            const int j = h ? ((k + 4) & 7) : k;
+            L.lb[k >> 1] |= (uint32_t)(4 * (2 * w + (j >> 2))) << (8 * (k & 1));
+        }
+        L.wofs = 8u * w;
+        L.h = h;
+        L.grp = 8 * w / LsCfg<G, FMT>::B;
+    } else if constexpr (G == 128) {
         const int h = lane >> 4, q = lane & 15;
         const int w = q < 13 ? q : 3 * (q - 12);  // copies of the straddling words 3, 6, 9
         const bool copy = q >= 13;
@@ -214,7 +234,7 @@ __device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
 // One lookup: the whole shared-memory address from one PRMT -- byte K mod 4
 // of word `a` as bits 8..15, the slot byte K mod 2 of `lb` as bits 0..7 and
 // bytes 2, 3 of `lb` (table block, window base) above.
-template <int G, int K>
+template <int K>
 __device__ __forceinline__ float ls_lookup(uint32_t a, uint32_t lb) {
     constexpr uint32_t kk = (uint32_t)(K & 3);
     constexpr uint32_t sel = 0x7600u | (kk << 4) | (4u + (uint32_t)(K & 1));
@@ -257,38 +277,38 @@ __device__ __forceinline__ float ls_transpose_reduce(float (&v)[NV], int lane) {
 }
 
 // Code word of one lane and step.
-template <int G>
-using LsWord = typename std::conditional<G == 128, uint2, uint32_t>::type;
-template <int G>
-__device__ __forceinline__ LsWord<G> ls_load(const uint8_t* p) {
-    if constexpr (G == 128) return ldg_nc_u2(p);
+template <bool WIDE>
+using LsWord = typename std::conditional<WIDE, uint2, uint32_t>::type;
+template <bool WIDE>
+__device__ __forceinline__ LsWord<WIDE> ls_load(const uint8_t* p) {
+    if constexpr (WIDE) return ldg_nc_u2(p);
     else return ldg_nc_u32(p);
 }
 
 // The scaled sums of two steps' code words (wa, wb), side by side:
 // ((t0+t1)+(t2+t3)) + ((t4+t5)+(t6+t7)) per step, times the step's scale.
-template <int G>
-__device__ __forceinline__ float2 ls_two_steps(const LsWord<G>& wa, const LsWord<G>& wb, const LsLane& L,
+template <bool WIDE>
+__device__ __forceinline__ float2 ls_two_steps(const LsWord<WIDE>& wa, const LsWord<WIDE>& wb, const LsLane& L,
                                                float sca, float scb) {
-    if constexpr (G == 128) {
+    if constexpr (WIDE) {
         const uint32_t a0 = L.h ? wa.y : wa.x, a1 = L.h ? wa.x : wa.y;
         const uint32_t b0 = L.h ? wb.y : wb.x, b1 = L.h ? wb.x : wb.y;
-        const uint64_t p0 = f2_pack(ls_lookup<G, 0>(a0, L.lb[0]), ls_lookup<G, 0>(b0, L.lb[0]));
-        const uint64_t p1 = f2_pack(ls_lookup<G, 1>(a0, L.lb[0]), ls_lookup<G, 1>(b0, L.lb[0]));
-        const uint64_t p2 = f2_pack(ls_lookup<G, 2>(a0, L.lb[1]), ls_lookup<G, 2>(b0, L.lb[1]));
-        const uint64_t p3 = f2_pack(ls_lookup<G, 3>(a0, L.lb[1]), ls_lookup<G, 3>(b0, L.lb[1]));
-        const uint64_t p4 = f2_pack(ls_lookup<G, 4>(a1, L.lb[2]), ls_lookup<G, 4>(b1, L.lb[2]));
-        const uint64_t p5 = f2_pack(ls_lookup<G, 5>(a1, L.lb[2]), ls_lookup<G, 5>(b1, L.lb[2]));
-        const uint64_t p6 = f2_pack(ls_lookup<G, 6>(a1, L.lb[3]), ls_lookup<G, 6>(b1, L.lb[3]));
-        const uint64_t p7 = f2_pack(ls_lookup<G, 7>(a1, L.lb[3]), ls_lookup<G, 7>(b1, L.lb[3]));
+        const uint64_t p0 = f2_pack(ls_lookup<0>(a0, L.lb[0]), ls_lookup<0>(b0, L.lb[0]));
+        const uint64_t p1 = f2_pack(ls_lookup<1>(a0, L.lb[0]), ls_lookup<1>(b0, L.lb[0]));
+        const uint64_t p2 = f2_pack(ls_lookup<2>(a0, L.lb[1]), ls_lookup<2>(b0, L.lb[1]));
+        const uint64_t p3 = f2_pack(ls_lookup<3>(a0, L.lb[1]), ls_lookup<3>(b0, L.lb[1]));
+        const uint64_t p4 = f2_pack(ls_lookup<4>(a1, L.lb[2]), ls_lookup<4>(b1, L.lb[2]));
+        const uint64_t p5 = f2_pack(ls_lookup<5>(a1, L.lb[2]), ls_lookup<5>(b1, L.lb[2]));
+        const uint64_t p6 = f2_pack(ls_lookup<6>(a1, L.lb[3]), ls_lookup<6>(b1, L.lb[3]));
+        const uint64_t p7 = f2_pack(ls_lookup<7>(a1, L.lb[3]), ls_lookup<7>(b1, L.lb[3]));
         const uint64_t lo = f2_add(f2_add(p0, p1), f2_add(p2, p3));
         const uint64_t hi = f2_add(f2_add(p4, p5), f2_add(p6, p7));
         return f2_unpack(f2_mul(f2_add(lo, hi), f2_pack(sca, scb)));
     } else {
-        const uint64_t p0 = f2_pack(ls_lookup<G, 0>(wa, L.lb[0]), ls_lookup<G, 0>(wb, L.lb[0]));
-        const uint64_t p1 = f2_pack(ls_lookup<G, 1>(wa, L.lb[0]), ls_lookup<G, 1>(wb, L.lb[0]));
-        const uint64_t p2 = f2_pack(ls_lookup<G, 2>(wa, L.lb[1]), ls_lookup<G, 2>(wb, L.lb[1]));
-        const uint64_t p3 = f2_pack(ls_lookup<G, 3>(wa, L.lb[1]), ls_lookup<G, 3>(wb, L.lb[1]));
+        const uint64_t p0 = f2_pack(ls_lookup<0>(wa, L.lb[0]), ls_lookup<0>(wb, L.lb[0]));
+        const uint64_t p1 = f2_pack(ls_lookup<1>(wa, L.lb[0]), ls_lookup<1>(wb, L.lb[0]));
+        const uint64_t p2 = f2_pack(ls_lookup<2>(wa, L.lb[1]), ls_lookup<2>(wb, L.lb[1]));
+        const uint64_t p3 = f2_pack(ls_lookup<3>(wa, L.lb[1]), ls_lookup<3>(wb, L.lb[1]));
         return f2_unpack(f2_mul(f2_add(f2_add(p0, p1), f2_add(p2, p3)), f2_pack(sca, scb)));
     }
 }
@@ -299,12 +319,13 @@ __device__ __forceinline__ void st_cluster_f32(uint32_t local_addr, int rank, fl
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
-template <int G, int CS>
+template <int G, int FMT, int CS>
 __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const LsArgs a) {
-    using C = LsCfg<G>;
-    using Word = LsWord<G>;
+    using C = LsCfg<G, FMT>;
+    constexpr bool WIDE = ls_wide<G, FMT>();
+    using Word = LsWord<WIDE>;
     constexpr int SPC = C::SPC, U = C::U, RPS = C::RPS, GPS = C::GPS;
-    constexpr int64_t RB = (int64_t)CS * kLsSliceBytes;  // code bytes per row
+    constexpr int64_t RB = (int64_t)CS * C::SB;          // code bytes per row
     constexpr int NG = CS * GPS;                         // groups per row
     constexpr int64_t STEP = RPS * RB;                   // code bytes between a lane's consecutive steps
     constexpr int PS = (kLsRound + CS - 1) / CS;         // partial rows per rank slot
@@ -322,7 +343,7 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
     // [0x10000, 0x30000), the scales, partials and activations just below.
     const uint32_t dyn = (uint32_t)__cvta_generic_to_shared(smem);
     const uint32_t wbase = dyn & 0xFF000000u, doff = dyn - wbase;
-    const uint32_t misc = kLsTableAbs - ls_misc_bytes<G>();
+    const uint32_t misc = kLsTableAbs - ls_misc_bytes<G, FMT>();
     if (doff > misc) {  // the same offset in every CTA: all of them leave here, none waits on a peer
         if (threadIdx.x == 0 && a.d_err) atomicOr(a.d_err, TQ_DERR_TIMEOUT);
         return;
@@ -330,37 +351,51 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
     // peers store partial rows into this CTA only after the matching wait
     cluster_arrive_relaxed();
     float* ssc = reinterpret_cast<float*>(smem + (misc - doff)) + warp * GPS * kLsScaleStride;
-    float* part = reinterpret_cast<float*>(smem + (misc - doff) + ls_scale_bytes<G>());
+    float* part = reinterpret_cast<float*>(smem + (misc - doff) + ls_scale_bytes<G, FMT>());
     float* xs = part + 2 * kLsPartFloats;
     const uint32_t part_sa = (uint32_t)__cvta_generic_to_shared(part);
     const uint32_t tabs = wbase + kLsTableAbs;  // the tables, for the stores of the build
     const float nan = __uint_as_float(0x7FC00000u);
 
-    // constant parts of the tables: the masking columns (banks 26..31) and
-    // the invalid-byte rows 243..255 (NaN in the table columns)
-    for (int it = warp; it < 36; it += kLsWarps) {
-        if (lane >= kLsFreeBank) {
-            const int bs = it / 9, d34 = it - 9 * bs;
-            const uint32_t base = tabs + (bs >> 1) * kLsBlockBytes + 27u * d34 * 256u + 4u * (uint32_t)(lane + 32 * (bs & 1));
+    if constexpr (FMT == 3) {
+        // constant parts of the tables: the masking columns (banks 26..31) and
+        // the invalid-byte rows 243..255 (NaN in the table columns)
+        for (int it = warp; it < 36; it += kLsWarps) {
+            if (lane >= kLsFreeBank) {
+                const int bs = it / 9, d34 = it - 9 * bs;
+                const uint32_t base =
+                    tabs + (bs >> 1) * kLsBlockBytes + 27u * d34 * 256u + 4u * (uint32_t)(lane + 32 * (bs & 1));
 #pragma unroll
-            for (int e = 0; e < 27; ++e) sts_f32(base + 256u * e, 0.f);
+                for (int e = 0; e < 27; ++e) sts_f32(base + 256u * e, 0.f);
+            }
+        }
+        for (int it = warp; it < 4; it += kLsWarps) {
+            const uint32_t base = tabs + (it >> 1) * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * (it & 1));
+            const float v = lane < kLsFreeBank ? nan : 0.f;
+#pragma unroll
+            for (int b = 243; b < 256; ++b) sts_f32(base + 256u * b, v);
+        }
+    } else {
+        // constant parts of the tables: every byte with a code 3 is invalid (NaN);
+        // warp item (block, sub, c2, c3): entries b = c0 + 4 c1 + 16 c2 + 64 c3
+        for (int it = warp; it < 64; it += kLsWarps) {
+            const int bs = it >> 4, c2 = it & 3, c3 = (it >> 2) & 3;
+            const uint32_t base = tabs + (bs >> 1) * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * (bs & 1)) +
+                                  256u * (uint32_t)(16 * c2 + 64 * c3);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                if (c2 == 3 || c3 == 3 || (e & 3) == 3 || (e >> 2) == 3) sts_f32(base + 256u * e, nan);
         }
     }
-    for (int it = warp; it < 4; it += kLsWarps) {
-        const uint32_t base = tabs + (it >> 1) * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * (it & 1));
-        const float v = lane < kLsFreeBank ? nan : 0.f;
-#pragma unroll
-        for (int b = 243; b < 256; ++b) sts_f32(base + 256u * b, v);
-    }
 
-    const LsLane L = ls_lane<G>(lane, wbase);
+    const LsLane L = ls_lane<G, FMT>(lane, wbase);
     const int64_t crow0 = (int64_t)cid * a.rows_per_cluster;
     const int64_t crow1 = min(a.N, crow0 + a.rows_per_cluster);
-    const uint8_t* cbase = a.codes + (int64_t)crank * kLsSliceBytes + L.wofs;
+    const uint8_t* cbase = a.codes + (int64_t)crank * C::SB + L.wofs;
     const uint16_t* sbase = a.scales + (int64_t)crank * GPS;
     // this lane's scales in the warp's block: group L.grp, row L.h of each step, steps in order
     const float4* ssc_lane = reinterpret_cast<const float4*>(ssc + L.grp * kLsScaleStride + (RPS == 2 ? 16 * L.h : 0));
-    const int res_row = G == 128 ? 2 * (lane & 15) + (lane >> 4) : lane;  // row of the reduced value, in the chunk
+    const int res_row = WIDE ? 2 * (lane & 15) + (lane >> 4) : lane;  // row of the reduced value, in the chunk
     uint32_t err_acc = 0;
     bool tables_built = false;
     int round = 0;
@@ -381,7 +416,7 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
         auto load_clamped = [&](int t) -> Word {
             int r = RPS * t + L.h;
             r = r < nr ? r : nr - 1;
-            return ls_load<G>(cbase + (wr0 + r) * RB);
+            return ls_load<WIDE>(cbase + (wr0 + r) * RB);
         };
         using SRaw = typename std::conditional<G == 128, uint2, uint4>::type;
         auto load_scales = [&](int ch) -> SRaw {
@@ -408,39 +443,58 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
             asm volatile("griddepcontrol.wait;" ::: "memory");
             xs[threadIdx.x] = __uint_as_float((uint32_t)__ldcg(a.X + crank * kLsSliceCols + threadIdx.x) << 16);
             __syncthreads();
-            // warp item (block, sub, d3 + 3 d4): the 27 entries b = d0 + 3 d1 + 9 d2 + 27 (d3 + 3 d4)
-            // of one table row per lane (lane = bank)
-            for (int it = warp; it < 36; it += kLsWarps) {
-                if (lane < kLsFreeBank) {
-                    const int bs = it / 9, d34 = it - 9 * bs;
-                    const int block = bs >> 1, sub = bs & 1;
-                    const uint32_t base = tabs + block * kLsBlockBytes + 27u * d34 * 256u +
-                                          4u * (uint32_t)(lane + 32 * sub);
-                    const int p = ls_slot_position<G>(block, sub, lane);
-                    const int g = p / C::B, j = p - g * C::B;
-                    const int real = min(5, G - 5 * j);
-                    const float* xp = xs + g * G + 5 * j;
-                    float x[5];
-#pragma unroll
-                    for (int i = 0; i < 5; ++i) x[i] = i < real ? xp[i] : 0.f;
-                    const int d3 = d34 % 3, d4 = d34 / 3;
-                    const bool bad34 = (3 >= real && d3 != 1) || (4 >= real && d4 != 1);
-                    const float h34 = bad34 ? nan : (float)(d3 - 1) * x[3] + (float)(d4 - 1) * x[4];
-                    float P[9];
-#pragma unroll
-                    for (int d1 = 0; d1 < 3; ++d1)
-#pragma unroll
-                        for (int d0 = 0; d0 < 3; ++d0) {
-                            const bool bad = (1 >= real && d1 != 1) || (0 >= real && d0 != 1);
-                            P[d0 + 3 * d1] = bad ? nan : (float)(d0 - 1) * x[0] + (float)(d1 - 1) * x[1];
+            if constexpr (FMT == 3) {
+                // warp item (block, sub, d3 + 3 d4): the 27 entries b = d0 + 3 d1 + 9 d2 + 27 (d3 + 3 d4)
+                // of one table row per lane (lane = bank)
+                for (int it = warp; it < 36; it += kLsWarps) {
+                    if (lane < kLsFreeBank) {
+                        const int bs = it / 9, d34 = it - 9 * bs;
+                        const int block = bs >> 1, sub = bs & 1;
+                        const uint32_t base = tabs + block * kLsBlockBytes + 27u * d34 * 256u +
+                                              4u * (uint32_t)(lane + 32 * sub);
+                        const int p = ls_slot_position<G, FMT>(block, sub, lane);
+                        const int g = p / C::B, j = p - g * C::B;
+                        const int real = min(5, G - 5 * j);
+                        const float* xp = xs + g * G + 5 * j;
+                        float x[5];
+    #pragma unroll
+                        for (int i = 0; i < 5; ++i) x[i] = i < real ? xp[i] : 0.f;
+                        const int d3 = d34 % 3, d4 = d34 / 3;
+                        const bool bad34 = (3 >= real && d3 != 1) || (4 >= real && d4 != 1);
+                        const float h34 = bad34 ? nan : (float)(d3 - 1) * x[3] + (float)(d4 - 1) * x[4];
+                        float P[9];
+    #pragma unroll
+                        for (int d1 = 0; d1 < 3; ++d1)
+    #pragma unroll
+                            for (int d0 = 0; d0 < 3; ++d0) {
+                                const bool bad = (1 >= real && d1 != 1) || (0 >= real && d0 != 1);
+                                P[d0 + 3 * d1] = bad ? nan : (float)(d0 - 1) * x[0] + (float)(d1 - 1) * x[1];
+                            }
+    #pragma unroll
+                        for (int d2 = 0; d2 < 3; ++d2) {
+                            const bool bad2 = 2 >= real && d2 != 1;
+                            const float q2 = bad2 ? nan : h34 + (float)(d2 - 1) * x[2];
+    #pragma unroll
+                            for (int e = 0; e < 9; ++e) sts_f32(base + 256u * (9 * d2 + e), P[e] + q2);
                         }
-#pragma unroll
-                    for (int d2 = 0; d2 < 3; ++d2) {
-                        const bool bad2 = 2 >= real && d2 != 1;
-                        const float q2 = bad2 ? nan : h34 + (float)(d2 - 1) * x[2];
-#pragma unroll
-                        for (int e = 0; e < 9; ++e) sts_f32(base + 256u * (9 * d2 + e), P[e] + q2);
                     }
+                }
+            } else {
+                // warp item (block, sub, c2 + 3 c3), c2, c3 < 3: the 9 valid entries
+                // b = c0 + 4 c1 + 16 c2 + 64 c3 (c0, c1 < 3) of one table row per lane (lane = bank)
+                for (int it = warp; it < 36; it += kLsWarps) {
+                    const int bs = it / 9, c23 = it - 9 * bs, c2 = c23 % 3, c3 = c23 / 3;
+                    const int block = bs >> 1, sub = bs & 1;
+                    const uint32_t base = tabs + block * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * sub) +
+                                          256u * (uint32_t)(16 * c2 + 64 * c3);
+                    const float* xp = xs + 4 * ls_slot_position<G, FMT>(block, sub, lane);
+                    const float q = (float)(c2 - 1) * xp[2] + (float)(c3 - 1) * xp[3];
+#pragma unroll
+                    for (int c1 = 0; c1 < 3; ++c1)
+#pragma unroll
+                        for (int c0 = 0; c0 < 3; ++c0)
+                            sts_f32(base + 256u * (uint32_t)(c0 + 4 * c1),
+                                    ((float)(c0 - 1) * xp[0] + (float)(c1 - 1) * xp[1]) + q);
                 }
             }
             __syncthreads();
@@ -472,15 +526,15 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
             for (int s = 0; s < SPC; s += 2) {
                 const Word wa = cb[s % U], wb = cb[(s + 1) % U];
                 if constexpr (WALK) {
-                    cb[s % U] = ls_load<G>(lp + s * STEP);
-                    cb[(s + 1) % U] = ls_load<G>(lp + (s + 1) * STEP);
+                    cb[s % U] = ls_load<WIDE>(lp + s * STEP);
+                    cb[(s + 1) % U] = ls_load<WIDE>(lp + (s + 1) * STEP);
                 } else {
                     cb[s % U] = load_clamped(ch * SPC + s + U);
                     cb[(s + 1) % U] = load_clamped(ch * SPC + s + 1 + U);
                 }
                 if (s % 4 == 0) sc4 = ssc_lane[s / 4];
-                const float2 r = s % 4 == 0 ? ls_two_steps<G>(wa, wb, L, sc4.x, sc4.y)
-                                            : ls_two_steps<G>(wa, wb, L, sc4.z, sc4.w);
+                const float2 r = s % 4 == 0 ? ls_two_steps<WIDE>(wa, wb, L, sc4.x, sc4.y)
+                                            : ls_two_steps<WIDE>(wa, wb, L, sc4.z, sc4.w);
                 v[s] = r.x;
                 v[s + 1] = r.y;
             }
@@ -504,15 +558,17 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
         cluster_arrive();
         cluster_wait();
         const int own = (nround - crank + CS - 1) / CS;
-        const float* pb = reinterpret_cast<const float*>(smem + (misc - doff) + ls_scale_bytes<G>()) +
+        const float* pb = reinterpret_cast<const float*>(smem + (misc - doff) + ls_scale_bytes<G, FMT>()) +
                           (round & 1) * kLsPartFloats;
         for (int i = (int)threadIdx.x; i < own; i += kLsThreads) {
             float y = 0.f;
 #pragma unroll
             for (int q = 0; q < CS; ++q) y += pb[q * PS + i];
             const int64_t n = rr0 + crank + (int64_t)CS * i;
-            if (y != y)
-                err_acc |= scan_row_errors(a.codes + n * RB, a.scales + n * NG, NG, G, C::B);
+            if (y != y) {
+                if constexpr (FMT == 3) err_acc |= scan_row_errors(a.codes + n * RB, a.scales + n * NG, NG, G, C::B);
+                else err_acc |= scan_row_errors2(a.codes + n * RB, a.scales + n * NG, NG, G);
+            }
             if (a.y_bf16) reinterpret_cast<__nv_bfloat16*>(a.Y)[n] = __float2bfloat16_rn(y);
             else reinterpret_cast<float*>(a.Y)[n] = y;
         }
@@ -524,9 +580,9 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
     if (err_acc && a.d_err) atomicOr(a.d_err, err_acc);
 }
 
-template <int G, int CS>
+template <int G, int FMT, int CS>
 cudaError_t launch_ls(const LsArgs& a0, cudaStream_t stream, int sm_count) {
-    auto kern = gemv_lut_stream_kernel<G, CS>;
+    auto kern = gemv_lut_stream_kernel<G, FMT, CS>;
     static SmemAttr smem_attr;
     static int max_clusters = 0;
     static std::mutex mu;
@@ -563,37 +619,40 @@ cudaError_t launch_ls(const LsArgs& a0, cudaStream_t stream, int sm_count) {
     cfg.gridDim = dim3((unsigned)(ncl * CS));
     static const bool debug = getenv("TQ_DEBUG_PLAN") != nullptr;
     if (debug)
-        fprintf(stderr, "tq gemv_lut_stream N=%lld K=%d G=%d: CS=%d clusters=%d rows/cluster=%lld\n",
+        fprintf(stderr, "tq gemv_lut_stream fmt=%d N=%lld K=%d G=%d: CS=%d clusters=%d rows/cluster=%lld\n", FMT,
                 (long long)a.N, a.K, G, CS, ncl, (long long)a.rows_per_cluster);
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int G>
+template <int G, int FMT>
 cudaError_t launch_ls_cs(const LsArgs& a, cudaStream_t stream, int sm_count) {
     switch (a.CS) {
-        case 1: return launch_ls<G, 1>(a, stream, sm_count);
-        case 2: return launch_ls<G, 2>(a, stream, sm_count);
-        case 3: return launch_ls<G, 3>(a, stream, sm_count);
-        case 4: return launch_ls<G, 4>(a, stream, sm_count);
-        case 5: return launch_ls<G, 5>(a, stream, sm_count);
-        case 6: return launch_ls<G, 6>(a, stream, sm_count);
-        case 7: return launch_ls<G, 7>(a, stream, sm_count);
-        case 8: return launch_ls<G, 8>(a, stream, sm_count);
+        case 1: return launch_ls<G, FMT, 1>(a, stream, sm_count);
+        case 2: return launch_ls<G, FMT, 2>(a, stream, sm_count);
+        case 3: return launch_ls<G, FMT, 3>(a, stream, sm_count);
+        case 4: return launch_ls<G, FMT, 4>(a, stream, sm_count);
+        case 5: return launch_ls<G, FMT, 5>(a, stream, sm_count);
+        case 6: return launch_ls<G, FMT, 6>(a, stream, sm_count);
+        case 7: return launch_ls<G, FMT, 7>(a, stream, sm_count);
+        case 8: return launch_ls<G, FMT, 8>(a, stream, sm_count);
         default: return cudaErrorNotSupported;
     }
 }
 
 }  // namespace
 
-// Returns cudaErrorNotSupported when the shape is not covered: M != 1, G not
-// 64 or 128, K not a multiple of 512 or above 4096, or unaligned codes/scales.
+// fmt 3: base-3 codes, fmt 2: 2-bit codes.  Returns cudaErrorNotSupported
+// when the shape is not covered: M != 1, G not 64 or 128, K not a multiple
+// of 512 or above 4096, or unaligned codes/scales.
 cudaError_t launch_gemv_lut_stream(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                    int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                                   cudaStream_t stream, int sm_count) {
-    if (M != 1 || (G != 64 && G != 128) || K % kLsSliceCols != 0 || K > 8 * kLsSliceCols || N < 1)
+                                   cudaStream_t stream, int sm_count, int fmt) {
+    if (M != 1 || (G != 64 && G != 128) || (fmt != 2 && fmt != 3) || K % kLsSliceCols != 0 ||
+        K > 8 * kLsSliceCols || N < 1)
         return cudaErrorNotSupported;
+    const bool wide = G == 128 || fmt == 2;
     const uintptr_t ca = reinterpret_cast<uintptr_t>(codes), sa = reinterpret_cast<uintptr_t>(scales);
-    if ((ca & (G == 128 ? 7 : 3)) || (sa & (G == 128 ? 7 : 15))) return cudaErrorNotSupported;
+    if ((ca & (wide ? 7 : 3)) || (sa & (G == 128 ? 7 : 15))) return cudaErrorNotSupported;
     LsArgs a{};
     a.X = X;
     a.codes = codes;
@@ -604,7 +663,8 @@ cudaError_t launch_gemv_lut_stream(const uint16_t* X, int64_t M, const uint8_t* 
     a.Y = Y;
     a.y_bf16 = y_bf16;
     a.d_err = d_err;
-    return G == 128 ? launch_ls_cs<128>(a, stream, sm_count) : launch_ls_cs<64>(a, stream, sm_count);
+    if (fmt == 2) return G == 128 ? launch_ls_cs<128, 2>(a, stream, sm_count) : launch_ls_cs<64, 2>(a, stream, sm_count);
+    return G == 128 ? launch_ls_cs<128, 3>(a, stream, sm_count) : launch_ls_cs<64, 3>(a, stream, sm_count);
 }
 
 }  // namespace tq

@@ -23,7 +23,7 @@ cudaError_t launch_gemv_lut(const uint16_t* X, int64_t M, const uint8_t* codes, 
                             cudaStream_t stream, int sm_count, size_t smem_limit);
 cudaError_t launch_gemv_lut_stream(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                    int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                                   cudaStream_t stream, int sm_count);
+                                   cudaStream_t stream, int sm_count, int fmt);
 cudaError_t launch_gemv_w4(const uint16_t* X, int64_t M, const uint32_t* codes, const uint16_t* scales,
                            const uint16_t* biases, int64_t N, int64_t K, int G, void* Y, int y_bf16,
                            cudaStream_t stream, int sm_count);
@@ -217,7 +217,7 @@ tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* sc
     // per CTA, slices spread over a cluster, code words streamed per lane
     if (M == 1) {
         e = launch_gemv_lut_stream(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
-                                   N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count);
+                                   N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, 3);
         if (e != cudaErrorNotSupported) return from_cuda(e);
         cudaGetLastError();
     }
@@ -337,6 +337,20 @@ tq_status tq2_gemv(const void* X, int64_t M, const uint8_t* codes, const void* s
                                                 d_err, (cudaStream_t)stream, d->sm_count, &handled, 2);
         if (e != cudaSuccess) return from_cuda(e);
         if (handled) return TQ_OK;
+    }
+    // one token over a large matrix: lookup tables of one 512-column K slice
+    // per CTA, as tq_gemv (its fixed cost, the table build after the
+    // activations arrive, loses to the CUDA-core kernel below about 24 M
+    // weights at K <= 1536 and 8 M weights above: 14336 x 1024 takes 6.0 us
+    // against 7.7 us, 28672 x 1024 9.7 us against 7.9 us, 3584 x 3584 10.9
+    // us against 7.8 us)
+    const bool big = K >= 2048 ? N * K >= (int64_t)(8 << 20) : N * K >= (int64_t)(24 << 20);
+    if (M == 1 && big) {
+        const cudaError_t e = launch_gemv_lut_stream(static_cast<const uint16_t*>(X), M, codes,
+                                                     static_cast<const uint16_t*>(scales), N, K, G, Y,
+                                                     yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, 2);
+        if (e != cudaErrorNotSupported) return from_cuda(e);
+        cudaGetLastError();
     }
     const cudaError_t e = launch_gemv2(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
                                        N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count);

@@ -159,6 +159,75 @@ def test_gemv2_stack_full_size_sampled():
     assert int(err.item()) == 0
 
 
+# M = 1, G in {64, 128}, K a multiple of 512 up to 4096: the streaming
+# lookup-table kernel (cluster sizes 1..8, ragged row counts)
+STREAM2_SHAPES = [(16385, 512, 128), (16391, 1024, 64), (9001, 2048, 128), (3000, 1536, 64),
+                  (4501, 3584, 64), (4097, 4096, 128), (257, 2560, 128), (7000, 3072, 64)]
+
+
+@pytest.mark.parametrize("N,K,G", STREAM2_SHAPES)
+def test_gemv2_stream_shapes(N, K, G):
+    W = synthetic.weights(N, K, index=N % 997 + G, outlier_frac=1e-3)
+    codes, scales, _ = oracle.quantize_pack2(W, G)
+    X = synthetic.activations(1, K, offset=300)
+    ref = oracle.linear2(X, codes, scales, N, K, G)
+    Y, e = run_gemv2(X, codes, scales, N, K, G, torch.float32)
+    assert_rows_close_f32(Y, ref)
+    assert e == 0
+    Yb, _ = run_gemv2(X, codes, scales, N, K, G, torch.bfloat16)
+    assert_close_bf16(Yb, ref)
+    Y2, _ = run_gemv2(X, codes, scales, N, K, G, torch.float32)
+    assert np.array_equal(Y, Y2), "repeated launches differ"
+
+
+@pytest.mark.parametrize("G", [64, 128])
+def test_gemv2_stream_every_valid_byte(G):
+    """Every one of the 81 valid code bytes at every byte position of a
+    512-column slice (both K slices of a 2-CTA cluster), in rows that run
+    past a warp's share and a cluster's share."""
+    N, K = 9001, 1024
+    B = G // 4
+    valid = np.array([b for b in range(256) if all((b >> (2 * i)) & 3 != 3 for i in range(4))], dtype=np.uint8)
+    assert valid.size == 81
+    n = np.arange(N)[:, None, None]
+    g = np.arange(K // G)[None, :, None]
+    j = np.arange(B)[None, None, :]
+    codes = valid[(n * 7 + g * B + j * 11) % 81].astype(np.uint8)
+    scales = synthetic.weights(N, K // G, index=5).astype(np.uint16) & 0x3FFF  # positive finite binary16
+    X = synthetic.activations(1, K, offset=900)
+    ref = oracle.linear2(X, codes, scales, N, K, G)
+    Y, e = run_gemv2(X, codes, scales, N, K, G, torch.float32)
+    assert_rows_close_f32(Y, ref)
+    assert e == 0
+
+
+@pytest.mark.parametrize("G", [64, 128])
+def test_gemv2_stream_rejected_groups(G):
+    """Code 3 in each byte lane of a word, in both K slices and in the first
+    and last rows; Inf, NaN and -0 scales; zero groups stay finite."""
+    N, K = 20000, 1024
+    W = synthetic.weights(N, K, index=G + 3)
+    codes, scales, _ = oracle.quantize_pack2(W, G)
+    B = G // 4
+    bad_rows = []
+    for i, (n, byte) in enumerate([(0, 0), (1, 5), (777, 9), (4096, B - 1), (12345, 3), (N - 1, 7)]):
+        grp = i % (K // G)
+        codes[n, grp, byte % B] |= 0x03 << (2 * (i % 4))
+        bad_rows.append(n)
+    scales[130, 0] = 0x7C00
+    scales[9999, K // G - 1] = 0x7E00
+    scales[N - 2, 1] = 0x8000
+    scales[77, 3] = 0
+    bad_rows += [130, 9999, N - 2]
+    X = synthetic.activations(1, K)
+    ref = oracle.linear2(X, codes, scales, N, K, G)
+    _, e_ref = oracle.unpack2_bf16(codes, scales, N, K, G)
+    Y, e = run_gemv2(X, codes, scales, N, K, G, torch.float32)
+    assert_rows_close_f32(Y, ref)
+    assert np.all(np.isnan(Y[:, bad_rows])) and np.all(np.isfinite(Y[:, 77]))
+    assert e == e_ref == tq.DERR_BYTE | tq.DERR_SCALE
+
+
 def test_gemv2_unsupported_group_size():
     N, K, G = 64, 480, 48
     W = synthetic.weights(N, K, index=1)
