@@ -72,6 +72,35 @@ def test_rejected_groups_give_nan_rows():
         assert e == e_ref
 
 
+@pytest.mark.parametrize("G", [64, 128])
+def test_every_code_byte(G):
+    """All 243 valid bytes at every non-final byte position of a group, every
+    canonical final byte, and the 13 invalid bytes (NaN rows), through the
+    prefill kernel (M = 130) and the small-M kernel (M = 16)."""
+    N, K = 520, 1024
+    B = (G + 4) // 5
+    real = G - 5 * (B - 1)  # digits of the final byte that hold weights
+    finals = np.array([b for b in range(243)
+                       if all((b // 3 ** i) % 3 == 1 for i in range(real, 5))], dtype=np.uint8)
+    n = np.arange(N)[:, None, None]
+    g = np.arange(K // G)[None, :, None]
+    j = np.arange(B)[None, None, :]
+    codes = ((n * B + g * 7 + j * 31) % 243).astype(np.uint8)
+    codes[:, :, B - 1] = finals[(np.arange(N)[:, None] * 5 + np.arange(K // G)[None, :]) % finals.size]
+    bad = list(range(507, 520))
+    for i, r in enumerate(bad):
+        codes[r, i % (K // G), (3 * i) % (B - 1)] = 243 + i
+    scales = (synthetic.weights(N, K // G, index=9).astype(np.uint16) & 0x3FFF) | 0x0400
+    X = synthetic.activations(130, K, offset=40)
+    ref = oracle.linear(X, codes, scales, N, K, G)
+    assert np.all(np.isnan(ref[:, bad])) and np.all(np.isfinite(ref[:, :507]))
+    _, e_ref = oracle.unpack_bf16(codes, scales, N, K, G)
+    for M in (130, 16):
+        Y, e = run(X[:M], codes, scales, N, K, G, torch.float32)
+        assert_rows_close_f32(Y, ref[:M])
+        assert e == e_ref == tq.DERR_BYTE
+
+
 def test_unsupported_group_size():
     W = synthetic.weights(64, 500, index=3)
     codes, scales, _ = oracle.quantize_pack(W, 100)
