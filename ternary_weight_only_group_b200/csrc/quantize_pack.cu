@@ -146,46 +146,159 @@ __host__ __device__ constexpr uint32_t code_place(int j) {
            << (8 * ((j / (FMT == 3 ? 5 : 4)) % 4));
 }
 
+// |w| of the two bf16 weights of a word as a pair of fp32 values (exact).
+__device__ __forceinline__ uint64_t mag_pair_f32x2(uint32_t w) {
+    return f2_pack(__uint_as_float((w << 16) & 0x7FFF0000u), __uint_as_float(w & 0x7FFF0000u));
+}
+
+// Sum of the G magnitudes of a group in fp32, the words' pairs spread over
+// NA packed accumulators (2 NA chains; chain c adds the magnitudes of words
+// i = c / 2 mod NA in order).  Recursive summation of nonnegative terms errs
+// by at most (n - 1) u of the exact sum for a chain of n terms (u = 2^-24),
+// and adding the 2 NA chains pairwise adds at most log2(2 NA) u more.
+template <int NA, int NW>
+__device__ __forceinline__ float group_sum_f32(const uint32_t (&h)[NW]) {
+    uint64_t acc[NA];
+#pragma unroll
+    for (int a = 0; a < NA; ++a) acc[a] = 0;
+#pragma unroll
+    for (int i = 0; i < NW; ++i) acc[i % NA] = f2_add(acc[i % NA], mag_pair_f32x2(h[i]));
+#pragma unroll
+    for (int n = NA / 2; n >= 1; n >>= 1)
+#pragma unroll
+        for (int a = 0; a < n; ++a) acc[a] = f2_add(acc[a], acc[a + n]);
+    const float2 r = f2_unpack(acc[0]);
+    return r.x + r.y;
+}
+
+// RNE_fp16(mean |w|) from a computed sum S of the G magnitudes whose relative
+// error is at most rel: accepted when S is finite and both ends of
+// [S (1 - rel), S (1 + rel)] / G round to the same finite binary16 (the
+// exact mean lies between them and rounding is monotone; the endpoints are
+// formed in binary64, whose own rounding is far inside the slack in rel).
+// Otherwise the caller takes an exact path: a mean within rel of a rounding
+// tie, a rejected (Inf/NaN) weight, or an overflowing mean.
+template <int G>
+__device__ __forceinline__ bool scale_from_sum(double S, double rel, uint16_t* s) {
+    if (!(S <= 3.4028234663852886e38)) return false;  // Inf or NaN
+    const double m = S * (1.0 / G);
+    const uint16_t lo = __half_as_ushort(__double2half(m * (1.0 - rel)));
+    const uint16_t hi = __half_as_ushort(__double2half(m * (1.0 + rel)));
+    if (lo != hi || lo >= 0x7C00u) return false;
+    *s = lo;
+    return true;
+}
+
+// Codes d = t + 1 (0, 1, 2) of the two bf16 weights of a word, in the two
+// 16-bit halves: 2 where w > s/2, 0 where w < -s/2, else 1 (ties round to
+// the even trit 0).  thp holds th = floor_bf16(s / 2) in both halves, thn
+// -th; for s = 0 both are NaN patterns and every code is 1.  A bf16 weight
+// exceeds s/2 exactly when it exceeds th.
+__device__ __forceinline__ uint32_t codes_pair(uint32_t w, uint32_t thp, uint32_t thn) {
+    uint32_t g, l;
+    asm("set.gt.u32.bf16x2 %0, %1, %2;" : "=r"(g) : "r"(w), "r"(thp));
+    asm("set.lt.u32.bf16x2 %0, %1, %2;" : "=r"(l) : "r"(w), "r"(thn));
+    return 0x00010001u + (g & 0x00010001u) - (l & 0x00010001u);
+}
+
+// Packed code words of a group from its words' code pairs, in word order:
+// byte q is the sum over its weights j of code_j * place_j (3^(j mod 5)
+// base-3, 4^(j mod 4) 2-bit), and the 4 bytes of a packed word cover exactly
+// WPW = 2 PER words of weights.  a[r] collects byte 4k + r of the current
+// packed word k in bits 16..31: a pair d2 = lo + 2^16 hi times (Q + 2^16 P)
+// leaves lo P + hi Q there (P, Q the places of the pair's weights in that
+// byte, 0 for a weight of another byte), while the lo Q products below stay
+// under 2^16.  Padding positions (j >= G) add their code 1.  Only the four
+// accumulators of the word being built are live.
+template <int G, int FMT>
+struct CodeWords {
+    static constexpr int PER = FMT == 3 ? 5 : 4;
+    static constexpr int B = (G + PER - 1) / PER;
+    static constexpr int NCW = (B + 3) / 4;
+    static constexpr int NWD = G / 2;
+    static constexpr int WPW = 2 * PER;
+    uint32_t a[4];
+    static __host__ __device__ constexpr uint32_t place(int j) {
+        return FMT == 3 ? (j % 5 == 0 ? 1u : j % 5 == 1 ? 3u : j % 5 == 2 ? 9u : j % 5 == 3 ? 27u : 81u)
+                        : 1u << (2 * (j % 4));
+    }
+    static __host__ __device__ constexpr uint32_t padding(int q) {
+        uint32_t pad = 0;
+        for (int j = PER * q; j < PER * q + PER; ++j)
+            if (j >= G) pad += place(j);
+        return pad << 16;
+    }
+    // word i of the group (weights 2i, 2i + 1), i = 0 .. NWD - 1 in order
+    __device__ __forceinline__ void put(int i, uint32_t d2, uint32_t (&cw)[NCW]) {
+        const int k = i / WPW;
+        if (i % WPW == 0) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a[r] = padding(4 * k + r);
+        }
+        const int j0 = 2 * i, j1 = 2 * i + 1, r0 = j0 / PER - 4 * k, r1 = j1 / PER - 4 * k;
+        if (r0 == r1) {
+            a[r0] += d2 * (place(j1) + (place(j0) << 16));
+        } else {
+            a[r0] += d2 * (place(j0) << 16);
+            a[r1] += d2 * place(j1);
+        }
+        if (i % WPW == WPW - 1 || i == NWD - 1) {
+            const uint32_t b1 = 4 * k + 1 < B ? a[1] : 0u, b2 = 4 * k + 2 < B ? a[2] : 0u,
+                           b3 = 4 * k + 3 < B ? a[3] : 0u;
+            cw[k] = prmt32(prmt32(a[0], b1, 0x0062u), prmt32(b2, b3, 0x0062u), 0x5410u);
+        }
+    }
+};
+
 // One lane per group (G = 8, 16, 32, 64, 128): the group's weights sit in
-// the lane's registers (G = 128: one half at a time, read twice), so max and
-// sum need no shuffles; every weight's byte
-// and power of three are compile-time constants, so encoding is one
-// multiply-add per weight into packed code words; each warp's 32 groups of
-// code bytes are assembled in shared memory and written with 16-byte stores
-// when the destination allows it.  The scale arithmetic is the one above.
-// FMT selects the packing: 3 = base-3 (five digits per byte), 2 = the 2-bit
-// format (four codes per byte; these G are multiples of 4, no padding).
+// the lane's registers, so sum and codes need no shuffles.  The scale comes
+// from an fp32 sum of the magnitudes (packed pairs, several chains) checked
+// against its error bound (scale_from_sum); the rare group near a rounding
+// tie takes the exact binary64 window of the fast path above, or the
+// multi-word path.  Codes: two bf16 comparisons per pair of weights
+// (codes_pair) and one multiply-add per pair into the current packed word
+// (CodeWords), every place value a compile-time constant.  Each warp's 32
+// groups of code bytes are assembled in shared memory and written with
+// 16-byte stores when the destination allows it.  FMT selects the packing:
+// 3 = base-3 (five digits per byte), 2 = the 2-bit format (four codes per
+// byte; these G are multiples of 4, no padding).
+// Threads per block of the group kernel: G = 128 holds its whole group (64
+// words) in registers and its ring rows are 272 bytes, so it runs 128-thread
+// blocks, three per SM; the others 256.
+template <int G>
+constexpr int qg_threads() { return G == 128 ? 128 : 256; }
+
 template <int G, int FMT = 3>
-__global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kernel(
+__global__ void __launch_bounds__(qg_threads<G>(), G <= 32 || G == 128 ? 3 : 2) quantize_pack_group_kernel(
     const uint16_t* __restrict__ W, int64_t num_groups, uint8_t* __restrict__ codes,
     uint16_t* __restrict__ scales, uint32_t* __restrict__ d_err) {
     constexpr int NWD = G / 2;                 // 32-bit words of a group
     constexpr int PER = FMT == 3 ? 5 : 4;  // codes per byte
     constexpr int B = (G + PER - 1) / PER;
     constexpr int NCW = (B + 3) / 4;           // packed code words
-    __shared__ __align__(16) uint8_t stage[256 / 32][32 * B];
+    constexpr int NW = qg_threads<G>() / 32;  // warps per block
+    __shared__ __align__(16) uint8_t stage[NW][32 * B];
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const bool vec_out = (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
     uint32_t err_acc = 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    // The warp's next 32 groups (G <= 64) or next half-groups of 64 weights
-    // (G = 128) are copied into a double-buffered shared-memory ring by
-    // coalesced cp.async while the current ones are quantized (the loads cost
-    // no registers, which the group occupies).  Ring rows are padded to
-    // 16 bytes past the data so that the 16-byte reads of the lanes' own rows
-    // are free of bank conflicts.
-    constexpr int RS = (G <= 64 ? 2 * G : 128) + 16;
-    extern __shared__ __align__(16) uint8_t qring[];  // [2][8 warps][32 rows][RS]
-    auto issue = [&](int64_t gb, int half, int buf) {
-        constexpr int PIECES = (G <= 64 ? G : 64) / 8;  // 16-byte pieces of a ring row
-        uint8_t* base = qring + ((size_t)buf * 8 + wib) * 32 * RS;
+    // The warp's next 32 groups are copied into a double-buffered
+    // shared-memory ring by coalesced cp.async while the current ones are
+    // quantized (the loads cost no registers, which the group occupies).  Ring
+    // rows are padded to 16 bytes past the data so that the 16-byte reads of
+    // the lanes' own rows are free of bank conflicts.
+    constexpr int RS = 2 * G + 16;
+    extern __shared__ __align__(16) uint8_t qring[];  // [2][NW warps][32 rows][RS]
+    auto issue = [&](int64_t gb, int buf) {
+        constexpr int PIECES = G / 8;  // 16-byte pieces of a ring row
+        uint8_t* base = qring + ((size_t)buf * NW + wib) * 32 * RS;
 #pragma unroll
         for (int k = 0; k < PIECES; ++k) {
             const int c = lane + 32 * k, grp = c / PIECES, piece = c - grp * PIECES;
             if (gb + grp < num_groups)
                 asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
                                  (uint32_t)__cvta_generic_to_shared(base + grp * RS + piece * 16)),
-                             "l"(__cvta_generic_to_global(W + (gb + grp) * G + half * 64 + piece * 8))
+                             "l"(__cvta_generic_to_global(W + (gb + grp) * G + piece * 8))
                              : "memory");
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -194,7 +307,7 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
     auto take = [&](int buf, uint32_t* h) {
         asm volatile("cp.async.wait_group 1;" ::: "memory");
         __syncwarp();
-        const uint4* row = reinterpret_cast<const uint4*>(qring + (((size_t)buf * 8 + wib) * 32 + lane) * RS);
+        const uint4* row = reinterpret_cast<const uint4*>(qring + (((size_t)buf * NW + wib) * 32 + lane) * RS);
 #pragma unroll
         for (int k = 0; k < (RS - 16) / 16; ++k) {
             const uint4 v = row[k];
@@ -206,7 +319,7 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
         __syncwarp();  // every lane has read this buffer before it is refilled
     };
     const int64_t g_first = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-    if (g_first < num_groups) issue(g_first, 0, 0);
+    if (g_first < num_groups) issue(g_first, 0);
     int pass = 0;
     for (int64_t g0 = g_first; g0 < num_groups; g0 += stride, ++pass) {
         const int64_t gi = g0 + lane;  // the warp's groups g0 .. g0+31
@@ -214,110 +327,48 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
         uint16_t s = 0;
         uint32_t gerr = 0;
         uint32_t cw[NCW];
-        if constexpr (G <= 64) {
+        {
             uint32_t h[NWD];
-            issue(g0 + stride, 0, (pass + 1) & 1);  // that buffer was read last pass
+            issue(g0 + stride, (pass + 1) & 1);  // that buffer was read last pass
             take(pass & 1, h);
-            uint32_t amax = 0;
+            // fp32 sum in 8 chains of G / 16 terms (G = 8..64; 16 chains of 8 at
+            // G = 128); a group whose mean lies within the sum's error of a
+            // rounding tie, or that holds an Inf/NaN weight or overflows, takes
+            // the exact binary64 window below
+            constexpr int NA = G == 128 ? 8 : NWD >= 4 ? 4 : NWD;
+            constexpr int TPC = (NWD + NA - 1) / NA;  // terms per chain
+            if (!scale_from_sum<G>((double)group_sum_f32<NA>(h), (TPC + 4) * 0x1p-24, &s)) {
+                uint32_t amax = 0;
 #pragma unroll
-            for (int j = 0; j < G; ++j) amax = max(amax, (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu);
-            const uint32_t emax = amax >> 7;
-            const uint32_t thr = emax > 37 ? (emax - 37) << 7 : 0;  // smallest pattern in the exact window
-            double sum = 0.0;
-            uint32_t outside = 0;
+                for (int j = 0; j < G; ++j) amax = max(amax, (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu);
+                const uint32_t emax = amax >> 7;
+                const uint32_t thr = emax > 37 ? (emax - 37) << 7 : 0;  // smallest pattern in the exact window
+                double sum = 0.0;
+                uint32_t outside = 0;
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-                const uint32_t a = (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
-                if (a >= thr) sum += bf16_normal_mag_to_f64(a);
-                else outside |= a;
-            }
-            if (amax >= 0x7F80u) {
-                gerr = TQ_DERR_WEIGHT;
-            } else if (amax > kTinyMaxBits) {
-                if (outside) {
-                    gerr = exact_group_scale(W + (active ? gi : 0) * G, G, &s);
-                } else {
-                    const uint16_t bits = __half_as_ushort(__double2half(sum * (1.0 / G)));
-                    if (bits >= 0x7C00u) gerr = TQ_DERR_OVERFLOW;
-                    else s = bits;
-                }
-            }
-            if (gerr) s = 0;
-            const uint32_t th = trit_threshold(s);
-            // code words: byte q of the group in byte q % 4 of word q / 4; code
-            // d = t + 1 of weight j at code_place(j); positions j >= G hold the
-            // padding code 1
-#pragma unroll
-            for (int i = 0; i < NCW; ++i) cw[i] = 0;
-#pragma unroll
-            for (int j = 0; j < PER * B; ++j) {
-                const uint32_t pw = code_place<FMT>(j);
-                if (j < G) {
-                    const uint32_t hw = h[j >> 1] >> (16 * (j & 1));
-                    const uint32_t d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
-                    cw[j / PER / 4] += d * pw;
-                } else {
-                    cw[j / PER / 4] += pw;  // padding code 1
-                }
-            }
-        } else {
-            // G = 128: the group is read twice in halves of 64 weights, so only
-            // one half (32 words) is live at a time.  Pass 1 takes max, the
-            // smallest nonzero magnitude and the binary64 sum of every nonzero
-            // magnitude; the sum is exact when all of them lie within 2^37 of the
-            // maximum (the same window as above), else the group takes the exact
-            // multi-word path.  Pass 2 re-reads the halves (cache hits) to encode.
-            // Ring steps: half 0 and 1 of pass 1 in buffers 0 and 1, then of
-            // pass 2; each step issues the next (the last one the next 32
-            // groups' first half).
-            uint32_t amax = 0, amin1 = 0xFFFFFFFFu;  // amin1 = smallest nonzero magnitude - 1
-            double sum = 0.0;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t h[32];
-                issue(g0, 1 - half, 1 - half);
-                take(half, h);
-#pragma unroll
-                for (int j = 0; j < 64; ++j) {
+                for (int j = 0; j < G; ++j) {
                     const uint32_t a = (h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu;
-                    amax = max(amax, a);
-                    amin1 = min(amin1, a - 1u);  // a = 0 wraps to the largest value
-                    if (a) sum += bf16_normal_mag_to_f64(a);
+                    if (a >= thr) sum += bf16_normal_mag_to_f64(a);
+                    else outside |= a;
                 }
-            }
-            const uint32_t emax = amax >> 7;
-            const uint32_t thr = emax > 37 ? (emax - 37) << 7 : 0;
-            const bool outside = amin1 != 0xFFFFFFFFu && amin1 + 1u < thr;
-            if (amax >= 0x7F80u) {
-                gerr = TQ_DERR_WEIGHT;
-            } else if (amax > kTinyMaxBits) {
-                if (outside) {
-                    gerr = exact_group_scale(W + (active ? gi : 0) * G, G, &s);
-                } else {
-                    const uint16_t bits = __half_as_ushort(__double2half(sum * (1.0 / G)));
-                    if (bits >= 0x7C00u) gerr = TQ_DERR_OVERFLOW;
-                    else s = bits;
+                if (amax >= 0x7F80u) {
+                    gerr = TQ_DERR_WEIGHT;
+                } else if (amax > kTinyMaxBits) {
+                    if (outside) {
+                        gerr = exact_group_scale(W + (active ? gi : 0) * G, G, &s);
+                    } else {
+                        const uint16_t bits = __half_as_ushort(__double2half(sum * (1.0 / G)));
+                        if (bits >= 0x7C00u) gerr = TQ_DERR_OVERFLOW;
+                        else s = bits;
+                    }
                 }
             }
             if (gerr) s = 0;
             const uint32_t th = trit_threshold(s);
+            const uint32_t thp = th | (th << 16), thn = thp | 0x80008000u;
+            CodeWords<G, FMT> cwb;
 #pragma unroll
-            for (int i = 0; i < NCW; ++i) cw[i] = 0;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t h[32];
-                issue(half == 0 ? g0 : g0 + stride, 1 - half, 1 - half);
-                take(half, h);
-#pragma unroll
-                for (int jj = 0; jj < 64; ++jj) {
-                    const int j = 64 * half + jj;
-                    const uint32_t hw = h[jj >> 1] >> (16 * (jj & 1));
-                    const uint32_t d = ((hw & 0x7FFFu) > th) ? ((hw & 0x8000u) ? 0u : 2u) : 1u;
-                    cw[j / PER / 4] += d * code_place<FMT>(j);
-                }
-            }
-#pragma unroll
-            for (int j = G; j < PER * B; ++j) cw[j / PER / 4] += code_place<FMT>(j);  // padding codes 1
+            for (int i = 0; i < NWD; ++i) cwb.put(i, codes_pair(h[i], thp, thn), cw);
         }
         if (active) {
             scales[gi] = s;
@@ -346,17 +397,28 @@ __global__ void __launch_bounds__(256, G <= 32 ? 3 : 2) quantize_pack_group_kern
 }
 
 // Dynamic shared memory of quantize_pack_group_kernel: the load ring.
-static size_t quantize_ring_bytes(int G) { return (size_t)2 * 8 * 32 * ((G <= 64 ? 2 * G : 128) + 16); }
+static size_t quantize_ring_bytes(int G) { return (size_t)2 * (G == 128 ? 4 : 8) * 32 * (2 * G + 16); }
 
 template <int G, int FMT = 3>
 static cudaError_t launch_quantize_group(const uint16_t* W, int64_t num_groups, uint8_t* codes, uint16_t* scales,
-                                         uint32_t* d_err, cudaStream_t stream, int grid) {
+                                         uint32_t* d_err, cudaStream_t stream, int grid, int sm_count) {
     auto kern = quantize_pack_group_kernel<G, FMT>;
     const size_t smem = quantize_ring_bytes(G);
     static SmemAttr smem_attr;
     if ((int)smem > 48 * 1024)
         if (cudaError_t e = smem_attr.ensure(kern, (int)smem)) return e;
-    kern<<<grid, 256, smem, stream>>>(W, num_groups, codes, scales, d_err);
+    // one wave of resident blocks, each warp looping over many passes: the
+    // ring's fill is paid once per warp, and a warp that takes the slow exact
+    // path delays only itself, not the tail of a wave of short blocks
+    static std::atomic<int> per_sm{0};
+    int bps = per_sm.load();
+    if (bps == 0) {
+        if (cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kern, qg_threads<G>(), smem)) return e;
+        bps = bps < 1 ? 1 : bps;
+        per_sm.store(bps);
+    }
+    if (grid > bps * sm_count) grid = bps * sm_count;
+    kern<<<grid, qg_threads<G>(), smem, stream>>>(W, num_groups, codes, scales, d_err);
     return cudaGetLastError();
 }
 
@@ -419,7 +481,7 @@ cudaError_t launch_quantize_pack(const uint16_t* W, int64_t N, int64_t K, int G,
 #define TQ_QG_CASE(GG)                                                                              \
     case GG:                                                                                        \
         return launch_quantize_group<GG>(W, num_groups, codes, scales, d_err, stream,              \
-                                         grid_for((num_groups + 31) / 32 * 32, block, sm_count));
+                                         grid_for((num_groups + 31) / 32 * 32, block, sm_count), sm_count);
     switch (G) {
         TQ_QG_CASE(8)
         TQ_QG_CASE(16)
@@ -479,11 +541,11 @@ cudaError_t launch_quantize_pack2(const uint16_t* W, int64_t N, int64_t K, int G
     if (num_groups == 0) return cudaSuccess;
     const int grid = grid_for((num_groups + 31) / 32 * 32, 256, sm_count);
     switch (G) {
-        case 8: return launch_quantize_group<8, 2>(W, num_groups, codes, scales, d_err, stream, grid);
-        case 16: return launch_quantize_group<16, 2>(W, num_groups, codes, scales, d_err, stream, grid);
-        case 32: return launch_quantize_group<32, 2>(W, num_groups, codes, scales, d_err, stream, grid);
-        case 64: return launch_quantize_group<64, 2>(W, num_groups, codes, scales, d_err, stream, grid);
-        case 128: return launch_quantize_group<128, 2>(W, num_groups, codes, scales, d_err, stream, grid);
+        case 8: return launch_quantize_group<8, 2>(W, num_groups, codes, scales, d_err, stream, grid, sm_count);
+        case 16: return launch_quantize_group<16, 2>(W, num_groups, codes, scales, d_err, stream, grid, sm_count);
+        case 32: return launch_quantize_group<32, 2>(W, num_groups, codes, scales, d_err, stream, grid, sm_count);
+        case 64: return launch_quantize_group<64, 2>(W, num_groups, codes, scales, d_err, stream, grid, sm_count);
+        case 128: return launch_quantize_group<128, 2>(W, num_groups, codes, scales, d_err, stream, grid, sm_count);
         default: break;
     }
     quantize_pack2_generic_kernel<<<grid_for(num_groups, 128, sm_count), 128, 0, stream>>>(

@@ -45,6 +45,11 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -136,14 +141,13 @@ static __device__ __noinline__ uint32_t exact_group_scale(const uint16_t* __rest
                                                     uint16_t* s_out) {
     *s_out = 0;
     uint32_t amax = 0;
-    for (int j = 0; j < G; ++j) amax = max(amax, (uint32_t)(w[j] & 0x7FFF));
-    if (amax >= 0x7F80u) return TQ_DERR_WEIGHT;
-    if (amax >= kHugeBits) return TQ_DERR_OVERFLOW;
-    if (amax <= kTinyMaxBits) return 0;
-    // Every magnitude is below 2^32 = 2^165 units; G <= 2^12 of them fit in 6 words.
+    // Every magnitude below 2^32 (kHugeBits) is below 2^165 units; G <= 2^12
+    // of them fit in 6 words.  Larger ones (and Inf/NaN) only decide the error
+    // below, so they are not added.
     uint32_t L[6] = {0, 0, 0, 0, 0, 0};
-    for (int j = 0; j < G; ++j) {
-        uint32_t a = w[j] & 0x7FFF;
+    auto add = [&](uint32_t a) {
+        amax = max(amax, a);
+        if (a >= kHugeBits) return;
         uint32_t e = a >> 7;
         uint32_t m = (a & 0x7F) | (e ? 0x80u : 0u);
         uint32_t sh = e ? e - 1 : 0;
@@ -157,7 +161,27 @@ static __device__ __noinline__ uint32_t exact_group_scale(const uint16_t* __rest
             v >>= 32;
             if (v == 0 && carry == 0) break;
         }
+    };
+    if ((reinterpret_cast<uintptr_t>(w) & 15) == 0 && G % 8 == 0) {
+        // 16-byte loads, four in flight: the group costs a few load latencies, not G
+        for (int j = 0; j < G; j += 32) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                v[u] = j + 8 * u < G ? __ldg(reinterpret_cast<const uint4*>(w + j + 8 * u)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t h[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int k = 0; k < 8; ++k) add((h[k >> 1] >> (16 * (k & 1))) & 0x7FFFu);
+            }
+        }
+    } else {
+        for (int j = 0; j < G; ++j) add(w[j] & 0x7FFFu);
     }
+    if (amax >= 0x7F80u) return TQ_DERR_WEIGHT;
+    if (amax >= kHugeBits) return TQ_DERR_OVERFLOW;
+    if (amax <= kTinyMaxBits) return 0;
     uint32_t Q[6];
     uint64_t r = 0;
     for (int i = 5; i >= 0; --i) {
