@@ -516,6 +516,24 @@ def bench_gemv_stream(tq, args, world, peaks):
     return res
 
 
+def decode_shapes_once(tq, args, world, peaks):
+    """One tq_gemv launch (M=1) for each decode shape of the headline, gate
+    3584x1024 and down 1024x3584 at both G, in that order: the run that the
+    DRAM-traffic capture behind PREDECODE_DRAM_BYTES profiles (ncu flushes
+    the caches before each profiled launch)."""
+    import torch
+    res = {}
+    for G in GROUPS:
+        for name in ("gate", "down"):
+            N, K = FFN[name]
+            c, s = tq.quantize_pack(device_weights(N, K, seed=7000), G)
+            X = device_acts(1, K, seed=7100)
+            tq.gemv(X, c, s, N, K, G)
+            torch.cuda.synchronize()
+            res[f"{name}{N}x{K}_G{G}"] = {"bytes": packed_bytes(N, K, G) + 2 * K + 2 * N}
+    return res
+
+
 def bench_gemv_shapes(tq, args, world, peaks):
     """Each decode projection alone (M=1, both G), and gate and up stacked as
     one [7168 x 1024] matrix (one launch for both): per-launch time over 160
@@ -972,7 +990,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
-    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv", "msweep", "ternary2", "w4"], default=None,
+    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv", "msweep", "ternary2", "w4", "traffic"],
+                    default=None,
                     help="run one sub-benchmark alone and print its result (profiling aid)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -988,7 +1007,8 @@ def main():
             torch.cuda.set_device(local)
             peaks = load_peaks()
             fn = {"stream": bench_gemv_stream, "codec": bench_bulk_codec, "prefill": bench_prefill,
-                  "gemv": bench_gemv_shapes, "msweep": bench_msweep, "ternary2": bench_ternary2, "w4": bench_w4}
+                  "gemv": bench_gemv_shapes, "msweep": bench_msweep, "ternary2": bench_ternary2, "w4": bench_w4,
+                  "traffic": decode_shapes_once}
             res = fn[args.only](tq, args, world, peaks)
             if rank == 0:
                 print(json.dumps({"only": args.only, "result": res}), flush=True)
