@@ -37,13 +37,14 @@ sys.path.insert(0, ROOT)
 METRIC = "ternary x bf16 GEMV HBM GB/s (% of peak); prefill GEMM TFLOP/s; pack GB/s"
 # DRAM bytes (read + write) of one gemv_predecode_kernel launch per decode
 # shape (N, K, G), M=1, from an ncu capture of dram__bytes_read.sum +
-# dram__bytes_write.sum on `bench.py --only gemv` (one launch per shape).
+# dram__bytes_write.sum on `bench.py --only traffic` (one launch per shape,
+# caches flushed by ncu before each; the bf16 Y stays in L2, 0 bytes written).
 # Valid only for the kernel source they were captured on: the SHA-256 of
 # gemv_predecode.cu at capture time is recorded beside them, and the figures
 # are reported only while the current source still has that hash.
-PREDECODE_DRAM_BYTES = {(3584, 1024, 64): 906496, (1024, 3584, 64): 911104,
-                        (3584, 1024, 128): 848896, (1024, 3584, 128): 854528}
-PREDECODE_DRAM_SRC_SHA256 = None
+PREDECODE_DRAM_BYTES = {(3584, 1024, 64): 905984, (1024, 3584, 64): 910336,
+                        (3584, 1024, 128): 848896, (1024, 3584, 128): 853760}
+PREDECODE_DRAM_SRC_SHA256 = "8ccc418b8745d4e8bc48b571c4b42920da749cfa994ea2ac577c81627928bab4"
 FFN = {"gate": (3584, 1024), "up": (3584, 1024), "down": (1024, 3584)}
 MSWEEP = {"q": (1536, 1536), "o": (1536, 1536), "gate": (4096, 1536), "up": (4096, 1536), "down": (1536, 4096)}
 MSWEEP_LAYERS = 28
