@@ -510,6 +510,17 @@ def bench_gemv_stream(tq, args, world, peaks):
                      f"({ncopy * byts / 1e6:.0f} MB > L2)"}
         if layers == 24 and G == 128:
             res.update(r)
+            # 2 and 4 tokens on the same matrix (one streaming launch per token)
+            for M in (2, 4):
+                XM = device_acts(M, K, seed=79)
+                YM = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+                lm = [lambda c=c, s=s: tq.gemv(XM, c, s, N, K, G, out=YM) for c, s in packs]
+                usm = graph_launch_us(lm, 16 // ncopy, args, world)
+                bm = packed_bytes(N, K, G) + 2 * M * K + 2 * M * N
+                res[f"tokens{M}"] = {"us": round(usm, 2), "GB/s": round(bm / (usm * 1e-6) / 1e9, 1),
+                                     "launches": max(3, args.steps) * 16 * M,
+                                     "note": "one streaming launch per token; GB/s on the weights read once"}
+                del lm, XM, YM
         else:
             res[f"stack{layers}_G{G}"] = r
         del packs, launches

@@ -123,9 +123,11 @@ TQ_API tq_status tq_unpack_bf16(const uint8_t *codes, const void *scales_f16, in
  * Matvec" stage): Y[m][n] = sum_g RNE_bf16(s[n][g]) * sum_{j in g} t[n][j] X[m][j],
  * accumulated in fp32, written as fp32 or RNE bf16.  Any M >= 1: CUDA-core
  * kernels up to 8 tokens (weights decoded on chip ahead of the activations
- * when a matrix's rows fit, lookup tables otherwise), tensor-core small-M
- * kernels up to 64 tokens, a row kernel beyond and for the shapes those do
- * not cover.  X: [M][K] bf16, 16-byte aligned; Y: [M][N]
+ * when a matrix's rows fit; otherwise lookup tables: one streaming launch
+ * per token for 1 token, and for 2..4 tokens on matrices of at least 48 M
+ * weights, with G in {64, 128} and K a multiple of 512 up to 4096),
+ * tensor-core small-M kernels up to 64 tokens, a row kernel beyond and for
+ * the shapes those do not cover.  X: [M][K] bf16, 16-byte aligned; Y: [M][N]
  * (fp32: 4-byte aligned, bf16: 2-byte aligned), must not overlap the inputs.
  * K == 0 is allowed: every output is an empty sum and Y is set to +0.
  * workspace: at least tq_workspace_bytes(M, N, K, G) bytes of device scratch
@@ -177,10 +179,14 @@ TQ_API tq_status tq2_unpack_bf16(const uint8_t *codes, const void *scales_f16, i
  * definition, arguments, alignment and ordering rule as tq_gemv (X is read
  * after the preceding work has completed; codes and scales may be read
  * before, so the kernel launched immediately before on the same stream must
- * not write them).  3..64 tokens with K % 64 == 0 and G % 64 == 0 take the
- * tensor-core small-M kernels (2-bit codes decoded on chip); otherwise the
- * CUDA-core kernel, eight tokens per launch, which covers G in {16, 32, 64,
- * 128, 256} and K <= 49152; other shapes return TQ_ERR_UNSUPPORTED. */
+ * not write them).  1 token on matrices of at least 24 M weights (8 M at
+ * K >= 2048), and 2..4 tokens from 48 M weights, with G in {64, 128}, K a
+ * multiple of 512 up to 4096 and 8-byte-aligned codes, take the streaming
+ * lookup-table kernel, one launch per token; 3..64 tokens with K % 64 == 0
+ * and G % 64 == 0 the tensor-core small-M kernels (2-bit codes decoded on
+ * chip); otherwise the CUDA-core kernel, eight tokens per launch, which
+ * covers G in {16, 32, 64, 128, 256} and K <= 49152; other shapes return
+ * TQ_ERR_UNSUPPORTED. */
 TQ_API tq_status tq2_gemv(const void *X_bf16, int64_t M, const uint8_t *codes, const void *scales_f16,
                    int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype, void *workspace,
                    size_t ws_bytes, uint32_t *d_err, tq_stream_t stream);

@@ -124,8 +124,13 @@ __host__ __device__ constexpr uint32_t ls_scale_bytes() {
 }
 template <int G, int FMT>
 __host__ __device__ constexpr uint32_t ls_misc_bytes() {
-    return ls_scale_bytes<G, FMT>() + 2u * kLsPartFloats * 4 + (uint32_t)kLsSliceCols * 4;
+    return ls_scale_bytes<G, FMT>() + 2u * kLsPartFloats * 4 + (uint32_t)(kLsSliceCols + kLsSliceCols / 32) * 4;
 }
+
+// Index of activation c of the slice in the staged copy: one padding float
+// after every 32, so that the build's lanes, which read columns 20 or 32
+// apart, spread over the banks.
+__device__ __forceinline__ int xs_at(int c) { return c + (c >> 5); }
 
 struct LsArgs {
     const uint16_t* X;
@@ -441,7 +446,7 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
             // activations (every CTA of the grid reads the same 1 KB, so the
             // per-entry reads of the build go to shared memory).
             asm volatile("griddepcontrol.wait;" ::: "memory");
-            xs[threadIdx.x] = __uint_as_float((uint32_t)__ldcg(a.X + crank * kLsSliceCols + threadIdx.x) << 16);
+            xs[xs_at(threadIdx.x)] = __uint_as_float((uint32_t)__ldcg(a.X + crank * kLsSliceCols + threadIdx.x) << 16);
             __syncthreads();
             if constexpr (FMT == 3) {
                 // warp item (block, sub, d3 + 3 d4): the 27 entries b = d0 + 3 d1 + 9 d2 + 27 (d3 + 3 d4)
@@ -455,26 +460,26 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
                         const int p = ls_slot_position<G, FMT>(block, sub, lane);
                         const int g = p / C::B, j = p - g * C::B;
                         const int real = min(5, G - 5 * j);
-                        const float* xp = xs + g * G + 5 * j;
+                        const int c0 = g * G + 5 * j;
                         float x[5];
-    #pragma unroll
-                        for (int i = 0; i < 5; ++i) x[i] = i < real ? xp[i] : 0.f;
+#pragma unroll
+                        for (int i = 0; i < 5; ++i) x[i] = i < real ? xs[xs_at(c0 + i)] : 0.f;
                         const int d3 = d34 % 3, d4 = d34 / 3;
                         const bool bad34 = (3 >= real && d3 != 1) || (4 >= real && d4 != 1);
                         const float h34 = bad34 ? nan : (float)(d3 - 1) * x[3] + (float)(d4 - 1) * x[4];
                         float P[9];
-    #pragma unroll
+#pragma unroll
                         for (int d1 = 0; d1 < 3; ++d1)
-    #pragma unroll
+#pragma unroll
                             for (int d0 = 0; d0 < 3; ++d0) {
                                 const bool bad = (1 >= real && d1 != 1) || (0 >= real && d0 != 1);
                                 P[d0 + 3 * d1] = bad ? nan : (float)(d0 - 1) * x[0] + (float)(d1 - 1) * x[1];
                             }
-    #pragma unroll
+#pragma unroll
                         for (int d2 = 0; d2 < 3; ++d2) {
                             const bool bad2 = 2 >= real && d2 != 1;
                             const float q2 = bad2 ? nan : h34 + (float)(d2 - 1) * x[2];
-    #pragma unroll
+#pragma unroll
                             for (int e = 0; e < 9; ++e) sts_f32(base + 256u * (9 * d2 + e), P[e] + q2);
                         }
                     }
@@ -487,7 +492,10 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
                     const int block = bs >> 1, sub = bs & 1;
                     const uint32_t base = tabs + block * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * sub) +
                                           256u * (uint32_t)(16 * c2 + 64 * c3);
-                    const float* xp = xs + 4 * ls_slot_position<G, FMT>(block, sub, lane);
+                    const int c0 = 4 * ls_slot_position<G, FMT>(block, sub, lane);
+                    float xp[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) xp[i] = xs[xs_at(c0 + i)];
                     const float q = (float)(c2 - 1) * xp[2] + (float)(c3 - 1) * xp[3];
 #pragma unroll
                     for (int c1 = 0; c1 < 3; ++c1)

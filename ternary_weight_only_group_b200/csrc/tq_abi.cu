@@ -196,6 +196,29 @@ tq_status tq_unpack_bf16(const uint8_t* codes, const void* scales, int64_t N, in
                                    d->sm_count));
 }
 
+// The streaming one-token kernel once per token row (X row m -> Y row m), for
+// M <= kStreamMaxTokens.  One token always; 2..4 tokens only from
+// kStreamMinWeightsMulti weights, where M passes over the weights still beat
+// the multi-token kernels (172032 x 1024: 14.3 us per pass).  Returns
+// cudaErrorNotSupported, having launched nothing, when the kernel does not
+// cover the shape.
+constexpr int64_t kStreamMaxTokens = 4;
+constexpr int64_t kStreamMinWeightsMulti = (int64_t)48 << 20;
+static cudaError_t stream_per_token(const void* X, int64_t M, const uint8_t* codes, const void* scales, int64_t N,
+                                    int64_t K, int G, void* Y, tq_out_dtype yt, uint32_t* d_err, cudaStream_t stream,
+                                    int sm_count, int fmt) {
+    if (M > kStreamMaxTokens || (M > 1 && N * K < kStreamMinWeightsMulti)) return cudaErrorNotSupported;
+    const size_t ysz = yt == TQ_OUT_BF16 ? 2 : 4;
+    for (int64_t m = 0; m < M; ++m) {
+        const cudaError_t e = launch_gemv_lut_stream(static_cast<const uint16_t*>(X) + m * K, 1, codes,
+                                                     static_cast<const uint16_t*>(scales), N, K, G,
+                                                     static_cast<char*>(Y) + (size_t)m * N * ysz, yt == TQ_OUT_BF16,
+                                                     d_err, stream, sm_count, fmt);
+        if (e != cudaSuccess) return e;  // NotSupported can only come from the first (same shape every time)
+    }
+    return cudaSuccess;
+}
+
 tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* scales, int64_t N,
                   int64_t K, int G, void* Y, tq_out_dtype yt, void* workspace, size_t ws_bytes,
                   uint32_t* d_err, tq_stream_t stream) {
@@ -213,11 +236,13 @@ tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* sc
                                           d_err, (cudaStream_t)stream, d->sm_count);
     if (e != cudaErrorNotSupported) return from_cuda(e);
     cudaGetLastError();
-    // one token over a larger matrix: lookup tables of one 512-column K slice
-    // per CTA, slices spread over a cluster, code words streamed per lane
-    if (M == 1) {
-        e = launch_gemv_lut_stream(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
-                                   N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, 3);
+    // 1..4 tokens over a larger matrix: lookup tables of one 512-column K
+    // slice per CTA, slices spread over a cluster, code words streamed per
+    // lane; one launch per token (172032 x 1024: 14.3 us per token, against
+    // 49 us for two tokens on the lookup-table kernel below and 88 us for the
+    // tensor-core path at 3..16 tokens)
+    if (M <= kStreamMaxTokens) {
+        e = stream_per_token(X, M, codes, scales, N, K, G, Y, yt, d_err, (cudaStream_t)stream, d->sm_count, 3);
         if (e != cudaErrorNotSupported) return from_cuda(e);
         cudaGetLastError();
     }
@@ -329,6 +354,19 @@ tq_status tq2_gemv(const void* X, int64_t M, const uint8_t* codes, const void* s
     if (K == 0) return zero_output(a, (cudaStream_t)stream);  // empty sums
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
+    // 1..4 tokens over a large matrix: the streaming lookup-table kernel once
+    // per token, as tq_gemv (its fixed cost, the table build after the
+    // activations arrive, loses to the CUDA-core kernel below about 24 M
+    // weights at K <= 1536 and 8 M weights above: 14336 x 1024 takes 6.0 us
+    // against 7.7 us, 28672 x 1024 9.7 us against 7.9 us, 3584 x 3584 10.9
+    // us against 7.8 us)
+    const bool big = K >= 2048 ? N * K >= (int64_t)(8 << 20) : N * K >= (int64_t)(24 << 20);
+    if (M <= kStreamMaxTokens && big) {
+        const cudaError_t e = stream_per_token(X, M, codes, scales, N, K, G, Y, yt, d_err, (cudaStream_t)stream,
+                                               d->sm_count, 2);
+        if (e != cudaErrorNotSupported) return from_cuda(e);
+        cudaGetLastError();
+    }
     // 3..64 tokens: the tensor-core small-M kernels on the 2-bit codes
     if (M >= 3) {
         bool handled = false;
@@ -337,20 +375,6 @@ tq_status tq2_gemv(const void* X, int64_t M, const uint8_t* codes, const void* s
                                                 d_err, (cudaStream_t)stream, d->sm_count, &handled, 2);
         if (e != cudaSuccess) return from_cuda(e);
         if (handled) return TQ_OK;
-    }
-    // one token over a large matrix: lookup tables of one 512-column K slice
-    // per CTA, as tq_gemv (its fixed cost, the table build after the
-    // activations arrive, loses to the CUDA-core kernel below about 24 M
-    // weights at K <= 1536 and 8 M weights above: 14336 x 1024 takes 6.0 us
-    // against 7.7 us, 28672 x 1024 9.7 us against 7.9 us, 3584 x 3584 10.9
-    // us against 7.8 us)
-    const bool big = K >= 2048 ? N * K >= (int64_t)(8 << 20) : N * K >= (int64_t)(24 << 20);
-    if (M == 1 && big) {
-        const cudaError_t e = launch_gemv_lut_stream(static_cast<const uint16_t*>(X), M, codes,
-                                                     static_cast<const uint16_t*>(scales), N, K, G, Y,
-                                                     yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, 2);
-        if (e != cudaErrorNotSupported) return from_cuda(e);
-        cudaGetLastError();
     }
     const cudaError_t e = launch_gemv2(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
                                        N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count);

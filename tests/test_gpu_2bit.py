@@ -228,6 +228,21 @@ def test_gemv2_stream_rejected_groups(G):
     assert e == e_ref == tq.DERR_BYTE | tq.DERR_SCALE
 
 
+@pytest.mark.parametrize("M", [2, 4])
+@pytest.mark.parametrize("G", [64, 128])
+def test_gemv2_stream_per_token(M, G):
+    """2..4 tokens over a matrix of at least 48 M weights: one streaming
+    launch per token row."""
+    N, K = 24593, 2048
+    W = synthetic.weights(N, K, index=M * G)
+    codes, scales, _ = oracle.quantize_pack2(W, G)
+    X = synthetic.activations(M, K, offset=5)
+    ref = oracle.linear2(X, codes, scales, N, K, G)
+    Y, e = run_gemv2(X, codes, scales, N, K, G, torch.float32)
+    assert_rows_close_f32(Y, ref)
+    assert e == 0
+
+
 def test_gemv2_unsupported_group_size():
     N, K, G = 64, 480, 48
     W = synthetic.weights(N, K, index=1)

@@ -150,3 +150,22 @@ def test_stream_gemv_every_byte_value():
     Y, e = run(X, to_dev_u8(codes), to_dev_f16(scales), N, K, G)
     assert_rows_close_f32(Y, ref)
     assert e == e_ref
+
+
+@pytest.mark.parametrize("M", [2, 3, 4])
+@pytest.mark.parametrize("G", [64, 128])
+def test_stream_gemv_per_token(M, G):
+    """2..4 tokens over a matrix of at least 48 M weights: one streaming
+    launch per token row; every output compared."""
+    N, K = 49159, 1024
+    W = synthetic.weights(N, K, index=M + G, outlier_frac=1e-3)
+    codes, scales, _ = oracle.quantize_pack(W, G)
+    X = synthetic.activations(M, K, offset=11)
+    ref = oracle.linear(X, codes, scales, N, K, G)
+    dc, ds = to_dev_u8(codes), to_dev_f16(scales)
+    Y, e = run(X, dc, ds, N, K, G)
+    assert_rows_close_f32(Y, ref)
+    assert e == 0
+    Yb, _ = run(X, dc, ds, N, K, G, torch.bfloat16)
+    assert_close_bf16(Yb, ref)
+
