@@ -143,14 +143,19 @@ __global__ void __launch_bounds__(kUnpackThreads, kUnpackCtasPerSm) unpack16_ker
             s = __ldg(scales + gi);
         }
     };
-    uint32_t bv_next[4], s_next;
+    // code bytes and scale of the next two passes in flight
+    uint32_t bv_next[4], s_next, bv_next2[4], s_next2;
     load(warp * GPW, bv_next, s_next);
+    load(warp * GPW + stride, bv_next2, s_next2);
     for (int64_t base = warp * GPW; base < num_groups; base += stride) {
         const int64_t gi = base + lane / LPG;
         const bool active = gi < num_groups;
         const uint32_t bv[4] = {bv_next[0], bv_next[1], bv_next[2], bv_next[3]};
         const uint32_t s = s_next;
-        load(base + stride, bv_next, s_next);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) bv_next[t] = bv_next2[t];
+        s_next = s_next2;
+        load(base + 2 * stride, bv_next2, s_next2);
         uint32_t bad = scale_is_bad(s) ? TQ_DERR_SCALE : 0u;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
