@@ -57,14 +57,31 @@ __global__ void __launch_bounds__(256) unpack2_words_kernel(const uint32_t* __re
     const int lane = threadIdx.x & 31;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     uint32_t err_acc = 0;
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < nwords; base += stride) {
-        const int64_t w = base + lane;
-        const bool active = w < nwords;
-        uint32_t c = 0x55555555u, s = 0;  // past the end: zero trits, never stored
-        if (active) {
+    // the code words and scales of the next kPre passes are in flight (one
+    // 4-byte word per lane and pass is too little to cover the load latency)
+    constexpr int kPre = 4;
+    auto load = [&](int64_t w, uint32_t& c, uint32_t& s) {
+        c = 0x55555555u;  // past the end: zero trits, never stored
+        s = 0;
+        if (w < nwords) {
             c = __ldcs(codes + w);
             s = __ldg(scales + w / WPG);
         }
+    };
+    const int64_t first = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+    uint32_t cq[kPre], sq[kPre];
+#pragma unroll
+    for (int i = 0; i < kPre; ++i) load(first + i * stride + lane, cq[i], sq[i]);
+    for (int64_t base = first; base < nwords; base += stride) {
+        const int64_t w = base + lane;
+        const bool active = w < nwords;
+        const uint32_t c = cq[0], s = sq[0];
+#pragma unroll
+        for (int i = 0; i + 1 < kPre; ++i) {
+            cq[i] = cq[i + 1];
+            sq[i] = sq[i + 1];
+        }
+        load(base + kPre * stride + lane, cq[kPre - 1], sq[kPre - 1]);
         uint32_t bad = (scale_is_bad(s) ? TQ_DERR_SCALE : 0u) | (has_code3(c) ? TQ_DERR_BYTE : 0u);
         bad = seg_or_u32(bad, WPG);
         uint32_t V, Z;
