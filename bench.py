@@ -790,28 +790,27 @@ def w4_bytes(N, K, G):
 
 def bench_w4(tq, args, world, peaks):
     """The W4A16 affine format (the second weight format): the streaming
-    decode GEMV over the [172032 x 1024] gate/up-shaped stack at G=128 (two
-    copies, 182 MB > L2) and the tensor-core prefill GEMM at M=4096,
-    4096 -> 14336 (L2 flushed before every launch)."""
+    decode GEMV over the [172032 x 1024] gate/up-shaped stack at G=128 (four
+    copies, 374 MB > L2, used in turn from one CUDA graph) and the
+    tensor-core prefill GEMM at M=4096, 4096 -> 14336 (L2 flushed before
+    every launch)."""
     import torch
     res = {}
     N, K, G = 48 * 3584, 1024, 128
-    packs = [device_w4_params(N, K, G, seed=300 + c) for c in range(2)]
+    ncopy = 4
+    packs = [device_w4_params(N, K, G, seed=300 + c) for c in range(ncopy)]
     X = device_acts(1, K, seed=301)
     Y = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
-    reps = 4 * max(2, args.steps // 4)
-    state = {"i": 0}
-
-    def one():
-        c, s_, b = packs[state["i"] % 2]
-        state["i"] += 1
-        tq.w4_gemv(X, c, s_, b, N, K, G, out=Y)
-    ms = timed(one, reps, max(4, args.warmup), world)
-    gbs = (w4_bytes(N, K, G) + 2 * K + 2 * N) * reps / (ms * 1e-3) / 1e9
-    res["gemv_stream"] = {"shape": [N, K], "G": G, "us": round(ms * 1e3 / reps, 2), "GB/s": round(gbs, 1),
-                          "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": reps,
-                          "kernel": "gemv_w4_kernel<1, 1>"}
-    del packs
+    launches = [lambda p=p: tq.w4_gemv(X, p[0], p[1], p[2], N, K, G, out=Y) for p in packs]
+    us = graph_launch_us(launches, 16 // ncopy, args, world)
+    byts = w4_bytes(N, K, G) + 2 * K + 2 * N
+    gbs = byts / (us * 1e-6) / 1e9
+    res["gemv_stream"] = {"shape": [N, K], "G": G, "us": round(us, 2), "GB/s": round(gbs, 1),
+                          "frac": round(gbs / peaks["hbm_gbs"], 4), "launches": max(3, args.steps) * 16,
+                          "kernel": "gemv_lut_stream_kernel<128, 4, 4> (lookup tables of one 256-column slice "
+                                    "per CTA, 4-CTA clusters)",
+                          "note": f"{ncopy} copies of {byts / 1e6:.1f} MB used in turn from one CUDA graph"}
+    del packs, launches
     torch.cuda.empty_cache()
     M, N, K = 4096, 14336, 4096
     c, s_, b = device_w4_params(N, K, G, seed=302)

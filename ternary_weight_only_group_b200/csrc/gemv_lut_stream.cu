@@ -50,6 +50,15 @@
 // (st.shared::cluster), and after one cluster barrier per round the owner
 // adds the CS partials in rank order and writes Y.
 //
+// Other formats.  The same kernel reads 2-bit codes (a byte is four codes,
+// 81 valid entries, NaN for any code 3) and the affine 4-bit codes of the
+// W4A16 format (tiny-llm "Week 2 Day 3: Quantize the Model", "Group-Wise
+// Affine Quantization"): a byte is two codes q0 (low nibble) and q1, its
+// entry q0 x_0 + q1 x_1 over all 256 values, so a CTA's 128 table slots cover
+// 256 columns; a lane's step is s S + b Xw, S its table sum, s and b the
+// group's bf16 scale and bias and Xw the sum of the lane's 16 activations, so
+// the lanes of a group add up to s sum q x + b sum x.
+//
 // Ordering.  Codes and scales do not depend on earlier kernels: the first
 // steps' loads and the constant parts of the tables (the masking columns,
 // the invalid-byte rows) are issued before griddepcontrol.wait; the
@@ -79,11 +88,12 @@ constexpr int kLsRound = 4096;               // rows per cluster round (partials
 constexpr int kLsFreeBank = 26;              // banks 26..31: all-zero columns for masked lookups
 constexpr int kLsChunkRows = 32;             // rows per warp chunk
 constexpr int kLsScaleStride = 36;           // floats per group in a warp's scale block
-static_assert(kLsThreads == kLsSliceCols, "one thread per activation of the slice");
+static_assert(kLsThreads == kLsSliceCols, "at most one activation of the slice per thread");
 
 // FMT 3: base-3 codes (five digits per byte, 104 bytes per 512 columns);
 // FMT 2: 2-bit codes (four per byte, 128 bytes per 512 columns, groups of
-// 64 or 128 columns are whole 8-byte words).
+// 64 or 128 columns are whole 8-byte words); FMT 4: the affine 4-bit codes
+// (two per byte, 128 bytes per 256 columns, groups whole 8-byte words).
 template <int G, int FMT>
 struct LsCfg;
 template <>
@@ -107,6 +117,17 @@ template <>
 struct LsCfg<64, 2> {
     static constexpr int B = 16, SB = 128, GPS = 8, RPS = 2, SPC = 16, U = 8;
 };
+template <>
+struct LsCfg<128, 4> {
+    static constexpr int B = 64, SB = 128, GPS = 2, RPS = 2, SPC = 16, U = 8;
+};
+template <>
+struct LsCfg<64, 4> {
+    static constexpr int B = 32, SB = 128, GPS = 4, RPS = 2, SPC = 16, U = 8;
+};
+// K columns of one CTA's tables: 128 table slots, one per code byte
+template <int FMT>
+__host__ __device__ constexpr int ls_slice_cols() { return FMT == 4 ? 256 : kLsSliceCols; }
 // 8-byte code words, two rows per step
 template <int G, int FMT>
 constexpr bool ls_wide() { return LsCfg<G, FMT>::RPS == 2; }
@@ -114,13 +135,14 @@ constexpr bool ls_wide() { return LsCfg<G, FMT>::RPS == 2; }
 // Shared memory below the tables: per-warp decoded scales of a chunk (stored
 // group-major, and within a group in step order for each row of the step,
 // kLsScaleStride floats per group so that the float4 reads of lanes of
-// different groups and rows land in different banks), then two buffers of
+// different groups and rows land in different banks; FMT 4 adds the biases
+// in a second such block), then two buffers of
 // partial rows (CS slots of kLsRound / CS rows each, alternating by round),
 // then the slice's activations in fp32.
 constexpr int kLsPartFloats = kLsRound + 8;
 template <int G, int FMT>
 __host__ __device__ constexpr uint32_t ls_scale_bytes() {
-    return (uint32_t)kLsWarps * LsCfg<G, FMT>::GPS * kLsScaleStride * 4;
+    return (uint32_t)kLsWarps * LsCfg<G, FMT>::GPS * kLsScaleStride * 4 * (FMT == 4 ? 2 : 1);
 }
 template <int G, int FMT>
 __host__ __device__ constexpr uint32_t ls_misc_bytes() {
@@ -136,6 +158,7 @@ struct LsArgs {
     const uint16_t* X;
     const uint8_t* codes;
     const uint16_t* scales;
+    const uint16_t* biases;  // FMT 4 only
     int64_t N;
     int K, CS;
     int64_t rows_per_cluster;
@@ -173,7 +196,7 @@ __device__ __forceinline__ LsLane ls_lane(int lane, uint32_t win_base) {
         const uint32_t block = ls_wide<G, FMT>() ? (uint32_t)(i & 1) : (uint32_t)i;  // lookups 2i, 2i + 1
         L.lb[i] = (win_base & 0xFF000000u) | (((kLsTableAbs + block * kLsBlockBytes) >> 16) << 16) | 0x8000u;
     }
-    if constexpr (FMT == 2) {
+    if constexpr (FMT == 2 || FMT == 4) {
         // 16 words per row, no group straddles a word: every lookup is live
         const int h = lane >> 4, w = lane & 15;
         for (int k = 0; k < 8; ++k) {
@@ -290,11 +313,10 @@ __device__ __forceinline__ LsWord<WIDE> ls_load(const uint8_t* p) {
     else return ldg_nc_u32(p);
 }
 
-// The scaled sums of two steps' code words (wa, wb), side by side:
-// ((t0+t1)+(t2+t3)) + ((t4+t5)+(t6+t7)) per step, times the step's scale.
+// The table sums of two steps' code words (wa, wb), side by side (packed):
+// ((t0+t1)+(t2+t3)) + ((t4+t5)+(t6+t7)) per step.
 template <bool WIDE>
-__device__ __forceinline__ float2 ls_two_steps(const LsWord<WIDE>& wa, const LsWord<WIDE>& wb, const LsLane& L,
-                                               float sca, float scb) {
+__device__ __forceinline__ uint64_t ls_two_sums(const LsWord<WIDE>& wa, const LsWord<WIDE>& wb, const LsLane& L) {
     if constexpr (WIDE) {
         const uint32_t a0 = L.h ? wa.y : wa.x, a1 = L.h ? wa.x : wa.y;
         const uint32_t b0 = L.h ? wb.y : wb.x, b1 = L.h ? wb.x : wb.y;
@@ -308,15 +330,20 @@ __device__ __forceinline__ float2 ls_two_steps(const LsWord<WIDE>& wa, const LsW
         const uint64_t p7 = f2_pack(ls_lookup<7>(a1, L.lb[3]), ls_lookup<7>(b1, L.lb[3]));
         const uint64_t lo = f2_add(f2_add(p0, p1), f2_add(p2, p3));
         const uint64_t hi = f2_add(f2_add(p4, p5), f2_add(p6, p7));
-        return f2_unpack(f2_mul(f2_add(lo, hi), f2_pack(sca, scb)));
+        return f2_add(lo, hi);
     } else {
         const uint64_t p0 = f2_pack(ls_lookup<0>(wa, L.lb[0]), ls_lookup<0>(wb, L.lb[0]));
         const uint64_t p1 = f2_pack(ls_lookup<1>(wa, L.lb[0]), ls_lookup<1>(wb, L.lb[0]));
         const uint64_t p2 = f2_pack(ls_lookup<2>(wa, L.lb[1]), ls_lookup<2>(wb, L.lb[1]));
         const uint64_t p3 = f2_pack(ls_lookup<3>(wa, L.lb[1]), ls_lookup<3>(wb, L.lb[1]));
-        return f2_unpack(f2_mul(f2_add(f2_add(p0, p1), f2_add(p2, p3)), f2_pack(sca, scb)));
+        return f2_add(f2_add(p0, p1), f2_add(p2, p3));
     }
 }
+
+// Packed raw scales of one row's groups in a slice (2 bytes per group).
+template <int BYTES>
+using LsRaw = typename std::conditional<BYTES == 4, uint32_t,
+                                        typename std::conditional<BYTES == 8, uint2, uint4>::type>::type;
 
 __device__ __forceinline__ void st_cluster_f32(uint32_t local_addr, int rank, float v) {
     uint32_t ra;
@@ -355,7 +382,7 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
     }
     // peers store partial rows into this CTA only after the matching wait
     cluster_arrive_relaxed();
-    float* ssc = reinterpret_cast<float*>(smem + (misc - doff)) + warp * GPS * kLsScaleStride;
+    float* ssc = reinterpret_cast<float*>(smem + (misc - doff)) + warp * GPS * kLsScaleStride * (FMT == 4 ? 2 : 1);
     float* part = reinterpret_cast<float*>(smem + (misc - doff) + ls_scale_bytes<G, FMT>());
     float* xs = part + 2 * kLsPartFloats;
     const uint32_t part_sa = (uint32_t)__cvta_generic_to_shared(part);
@@ -380,7 +407,7 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
 #pragma unroll
             for (int b = 243; b < 256; ++b) sts_f32(base + 256u * b, v);
         }
-    } else {
+    } else if constexpr (FMT == 2) {
         // constant parts of the tables: every byte with a code 3 is invalid (NaN);
         // warp item (block, sub, c2, c3): entries b = c0 + 4 c1 + 16 c2 + 64 c3
         for (int it = warp; it < 64; it += kLsWarps) {
@@ -398,8 +425,11 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
     const int64_t crow1 = min(a.N, crow0 + a.rows_per_cluster);
     const uint8_t* cbase = a.codes + (int64_t)crank * C::SB + L.wofs;
     const uint16_t* sbase = a.scales + (int64_t)crank * GPS;
+    const uint16_t* bbase = a.biases + (int64_t)crank * GPS;  // FMT 4
     // this lane's scales in the warp's block: group L.grp, row L.h of each step, steps in order
     const float4* ssc_lane = reinterpret_cast<const float4*>(ssc + L.grp * kLsScaleStride + (RPS == 2 ? 16 * L.h : 0));
+    constexpr int kBiasF4 = GPS * kLsScaleStride / 4;  // FMT 4: the biases' block, in float4 past the scales'
+    float xw = 0.f;  // FMT 4: sum of the activations of the lane's 16 columns
     const int res_row = WIDE ? 2 * (lane & 15) + (lane >> 4) : lane;  // row of the reduced value, in the chunk
     uint32_t err_acc = 0;
     bool tables_built = false;
@@ -423,21 +453,20 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
             r = r < nr ? r : nr - 1;
             return ls_load<WIDE>(cbase + (wr0 + r) * RB);
         };
-        using SRaw = typename std::conditional<G == 128, uint2, uint4>::type;
-        auto load_scales = [&](int ch) -> SRaw {
+        using SRaw = LsRaw<2 * GPS>;
+        auto load_scales = [&](const uint16_t* base, int ch) -> SRaw {
             int r = ch * kLsChunkRows + lane;
             r = r < nr ? r : nr - 1;
-            const uint16_t* p = sbase + (wr0 + r) * NG;
-            if constexpr (G == 128) return __ldg(reinterpret_cast<const uint2*>(p));
-            else return __ldg(reinterpret_cast<const uint4*>(p));
+            return __ldg(reinterpret_cast<const SRaw*>(base + (wr0 + r) * NG));
         };
 
         Word cb[U];
-        SRaw sraw{};
+        SRaw sraw{}, braw{};
         if (nr > 0) {
 #pragma unroll
             for (int u = 0; u < U; ++u) cb[u] = load_clamped(u);
-            sraw = load_scales(0);
+            sraw = load_scales(sbase, 0);
+            if constexpr (FMT == 4) braw = load_scales(bbase, 0);
         }
 
         if (!tables_built) {
@@ -446,7 +475,9 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
             // activations (every CTA of the grid reads the same 1 KB, so the
             // per-entry reads of the build go to shared memory).
             asm volatile("griddepcontrol.wait;" ::: "memory");
-            xs[xs_at(threadIdx.x)] = __uint_as_float((uint32_t)__ldcg(a.X + crank * kLsSliceCols + threadIdx.x) << 16);
+            constexpr int SC = ls_slice_cols<FMT>();
+            if (threadIdx.x < SC)
+                xs[xs_at(threadIdx.x)] = __uint_as_float((uint32_t)__ldcg(a.X + crank * SC + threadIdx.x) << 16);
             __syncthreads();
             if constexpr (FMT == 3) {
                 // warp item (block, sub, d3 + 3 d4): the 27 entries b = d0 + 3 d1 + 9 d2 + 27 (d3 + 3 d4)
@@ -484,6 +515,22 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
                         }
                     }
                 }
+            } else if constexpr (FMT == 4) {
+                // warp item (block, sub, q1): the 16 entries b = q0 + 16 q1 of one
+                // table row per lane (lane = bank), q0 x[2p] + q1 x[2p + 1]
+                for (int it = warp; it < 64; it += kLsWarps) {
+                    const int bs = it >> 4, q1 = it & 15;
+                    const int block = bs >> 1, sub = bs & 1;
+                    const uint32_t base = tabs + block * kLsBlockBytes + 4u * (uint32_t)(lane + 32 * sub) +
+                                          256u * (uint32_t)(16 * q1);
+                    const int c0 = 2 * ls_slot_position<G, FMT>(block, sub, lane);
+                    const float hi = (float)q1 * xs[xs_at(c0 + 1)], x0 = xs[xs_at(c0)];
+#pragma unroll
+                    for (int q0 = 0; q0 < 16; ++q0) sts_f32(base + 256u * (uint32_t)q0, __fmaf_rn((float)q0, x0, hi));
+                }
+                // the lane's columns 16 w .. 16 w + 15 of the slice
+#pragma unroll
+                for (int i = 0; i < 16; ++i) xw += xs[xs_at(2 * (int)L.wofs + i)];
             } else {
                 // warp item (block, sub, c2 + 3 c3), c2, c3 < 3: the 9 valid entries
                 // b = c0 + 4 c1 + 16 c2 + 64 c3 (c0, c1 < 3) of one table row per lane (lane = bank)
@@ -523,13 +570,27 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
                 const uint32_t* sw = reinterpret_cast<const uint32_t*>(&sraw);
                 const int col = RPS == 2 ? 16 * (lane & 1) + (lane >> 1) : lane;
 #pragma unroll
-                for (int g = 0; g < GPS; ++g)
-                    ssc[g * kLsScaleStride + col] = ls_scale(g & 1 ? sw[g >> 1] >> 16 : sw[g >> 1] & 0xFFFFu);
-                if (ch + 1 < nch) sraw = load_scales(ch + 1);
+                for (int g = 0; g < GPS; ++g) {
+                    const uint32_t raw = g & 1 ? sw[g >> 1] >> 16 : sw[g >> 1] & 0xFFFFu;
+                    // FMT 4: bf16 scale and bias, taken as they are
+                    ssc[g * kLsScaleStride + col] = FMT == 4 ? __uint_as_float(raw << 16) : ls_scale(raw);
+                }
+                if constexpr (FMT == 4) {
+                    const uint32_t* bw = reinterpret_cast<const uint32_t*>(&braw);
+#pragma unroll
+                    for (int g = 0; g < GPS; ++g)
+                        ssc[(GPS + g) * kLsScaleStride + col] =
+                            __uint_as_float((g & 1 ? bw[g >> 1] >> 16 : bw[g >> 1] & 0xFFFFu) << 16);
+                }
+                if (ch + 1 < nch) {
+                    sraw = load_scales(sbase, ch + 1);
+                    if constexpr (FMT == 4) braw = load_scales(bbase, ch + 1);
+                }
                 __syncwarp();
             }
             float v[SPC];
             float4 sc4;
+            [[maybe_unused]] float4 bi4;
 #pragma unroll
             for (int s = 0; s < SPC; s += 2) {
                 const Word wa = cb[s % U], wb = cb[(s + 1) % U];
@@ -540,9 +601,20 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
                     cb[s % U] = load_clamped(ch * SPC + s + U);
                     cb[(s + 1) % U] = load_clamped(ch * SPC + s + 1 + U);
                 }
-                if (s % 4 == 0) sc4 = ssc_lane[s / 4];
-                const float2 r = s % 4 == 0 ? ls_two_steps<WIDE>(wa, wb, L, sc4.x, sc4.y)
-                                            : ls_two_steps<WIDE>(wa, wb, L, sc4.z, sc4.w);
+                if (s % 4 == 0) {
+                    sc4 = ssc_lane[s / 4];
+                    if constexpr (FMT == 4) bi4 = ssc_lane[kBiasF4 + s / 4];
+                }
+                const uint64_t sum = ls_two_sums<WIDE>(wa, wb, L);
+                const uint64_t sc = s % 4 == 0 ? f2_pack(sc4.x, sc4.y) : f2_pack(sc4.z, sc4.w);
+                float2 r;
+                if constexpr (FMT == 4) {
+                    // s S + b Xw: the lane's share of the group's bias term
+                    const uint64_t bi = s % 4 == 0 ? f2_pack(bi4.x, bi4.y) : f2_pack(bi4.z, bi4.w);
+                    r = f2_unpack(f2_fma(sum, sc, f2_mul(bi, f2_pack(xw, xw))));
+                } else {
+                    r = f2_unpack(f2_mul(sum, sc));
+                }
                 v[s] = r.x;
                 v[s + 1] = r.y;
             }
@@ -575,7 +647,7 @@ __global__ void __launch_bounds__(kLsThreads, 1) gemv_lut_stream_kernel(const Ls
             const int64_t n = rr0 + crank + (int64_t)CS * i;
             if (y != y) {
                 if constexpr (FMT == 3) err_acc |= scan_row_errors(a.codes + n * RB, a.scales + n * NG, NG, G, C::B);
-                else err_acc |= scan_row_errors2(a.codes + n * RB, a.scales + n * NG, NG, G);
+                else if constexpr (FMT == 2) err_acc |= scan_row_errors2(a.codes + n * RB, a.scales + n * NG, NG, G);
             }
             if (a.y_bf16) reinterpret_cast<__nv_bfloat16*>(a.Y)[n] = __float2bfloat16_rn(y);
             else reinterpret_cast<float*>(a.Y)[n] = y;
@@ -673,6 +745,33 @@ cudaError_t launch_gemv_lut_stream(const uint16_t* X, int64_t M, const uint8_t* 
     a.d_err = d_err;
     if (fmt == 2) return G == 128 ? launch_ls_cs<128, 2>(a, stream, sm_count) : launch_ls_cs<64, 2>(a, stream, sm_count);
     return G == 128 ? launch_ls_cs<128, 3>(a, stream, sm_count) : launch_ls_cs<64, 3>(a, stream, sm_count);
+}
+
+// The affine 4-bit codes (uint32 [N][K/8], low nibble first) with bf16 scales
+// and biases [N][K/G].  Returns cudaErrorNotSupported when the shape is not
+// covered: M != 1, G not 64 or 128, K not a multiple of 256 or above 2048,
+// codes not 8-byte aligned, scales or biases not aligned to G = 128 ? 4 : 8.
+cudaError_t launch_gemv_lut_stream_w4(const uint16_t* X, int64_t M, const uint32_t* codes, const uint16_t* scales,
+                                      const uint16_t* biases, int64_t N, int64_t K, int G, void* Y, int y_bf16,
+                                      cudaStream_t stream, int sm_count) {
+    constexpr int SC = ls_slice_cols<4>();
+    if (M != 1 || (G != 64 && G != 128) || K % SC != 0 || K > 8 * SC || N < 1) return cudaErrorNotSupported;
+    const uintptr_t ca = reinterpret_cast<uintptr_t>(codes), sa = reinterpret_cast<uintptr_t>(scales),
+                    ba = reinterpret_cast<uintptr_t>(biases);
+    const uintptr_t sm = G == 128 ? 3 : 7;
+    if ((ca & 7) || (sa & sm) || (ba & sm)) return cudaErrorNotSupported;
+    LsArgs a{};
+    a.X = X;
+    a.codes = reinterpret_cast<const uint8_t*>(codes);
+    a.scales = scales;
+    a.biases = biases;
+    a.N = N;
+    a.K = (int)K;
+    a.CS = (int)(K / SC);
+    a.Y = Y;
+    a.y_bf16 = y_bf16;
+    a.d_err = nullptr;
+    return G == 128 ? launch_ls_cs<128, 4>(a, stream, sm_count) : launch_ls_cs<64, 4>(a, stream, sm_count);
 }
 
 }  // namespace tq

@@ -27,6 +27,9 @@ cudaError_t launch_gemv_lut_stream(const uint16_t* X, int64_t M, const uint8_t* 
 cudaError_t launch_gemv_w4(const uint16_t* X, int64_t M, const uint32_t* codes, const uint16_t* scales,
                            const uint16_t* biases, int64_t N, int64_t K, int G, void* Y, int y_bf16,
                            cudaStream_t stream, int sm_count);
+cudaError_t launch_gemv_lut_stream_w4(const uint16_t* X, int64_t M, const uint32_t* codes, const uint16_t* scales,
+                                      const uint16_t* biases, int64_t N, int64_t K, int G, void* Y, int y_bf16,
+                                      cudaStream_t stream, int sm_count);
 cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                   int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                                   cudaStream_t stream, int sm_count);
@@ -203,6 +206,9 @@ tq_status tq_unpack_bf16(const uint8_t* codes, const void* scales, int64_t N, in
 // cudaErrorNotSupported, having launched nothing, when the kernel does not
 // cover the shape.
 constexpr int64_t kStreamMaxTokens = 4;
+// tq_w4_gemv: tokens and weights from which the streaming kernel runs
+constexpr int64_t kW4StreamMaxTokens = 1;
+constexpr int64_t kW4StreamMinWeights = (int64_t)16 << 20;
 constexpr int64_t kStreamMinWeightsMulti = (int64_t)48 << 20;
 static cudaError_t stream_per_token(const void* X, int64_t M, const uint8_t* codes, const void* scales, int64_t N,
                                     int64_t K, int G, void* Y, tq_out_dtype yt, uint32_t* d_err, cudaStream_t stream,
@@ -431,6 +437,19 @@ tq_status tq_w4_gemv(const void* X, int64_t M, const uint32_t* codes, const void
     if (K == 0) return from_cuda(cudaMemsetAsync(Y, 0, yb, (cudaStream_t)stream));  // empty sums
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
+    // 1..kW4StreamMaxTokens tokens over a large matrix: the streaming
+    // lookup-table kernel once per token (tables of 256 columns per CTA)
+    if (M <= kW4StreamMaxTokens && N * K >= kW4StreamMinWeights) {
+        const size_t ysz = yt == TQ_OUT_BF16 ? 2 : 4;
+        cudaError_t e = cudaSuccess;
+        for (int64_t m = 0; m < M && e == cudaSuccess; ++m)
+            e = launch_gemv_lut_stream_w4(static_cast<const uint16_t*>(X) + m * K, 1, codes,
+                                          static_cast<const uint16_t*>(scales), static_cast<const uint16_t*>(biases),
+                                          N, K, G, static_cast<char*>(Y) + (size_t)m * N * ysz, yt == TQ_OUT_BF16,
+                                          (cudaStream_t)stream, d->sm_count);
+        if (e != cudaErrorNotSupported) return from_cuda(e);  // NotSupported only from the first launch
+        cudaGetLastError();
+    }
     const cudaError_t e = launch_gemv_w4(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
                                          static_cast<const uint16_t*>(biases), N, K, G, Y, yt == TQ_OUT_BF16,
                                          (cudaStream_t)stream, d->sm_count);

@@ -70,6 +70,52 @@ def test_w4_gemv_every_code_value():
     assert_rows_close_f32(to_f64(Y), ref)
 
 
+@pytest.mark.parametrize("G", [64, 128])
+@pytest.mark.parametrize("K", [256, 512, 768, 1024, 1280, 1536, 1792, 2048])
+def test_w4_gemv_stream(K, G):
+    """One token over 16 M weights and more: the streaming lookup-table kernel
+    (tables of 256 columns per CTA, K / 256 CTAs per cluster, one to eight),
+    the last cluster's rows ragged."""
+    N = (16 << 20) // K + 37
+    check(N, K, G, 1, index=K + 3 * G)
+
+
+def test_w4_gemv_stream_every_byte():
+    """Every code byte (two nibbles) in every byte position of the tables:
+    row n, word w, byte i holds (n + 8 w + i) mod 256."""
+    N, K, G = 16411, 1024, 128
+    codes, scales, biases = synthetic.w4_params(N, K, G, index=5)
+    n = np.arange(N, dtype=np.uint32)[:, None, None]
+    w = np.arange(K // 8, dtype=np.uint32)[None, :, None]
+    i = np.arange(4, dtype=np.uint32)[None, None, :]
+    byte = (n + 8 * w + i) % 256
+    codes = (byte << (8 * i)).sum(axis=2).astype(np.uint32)
+    X = synthetic.activations(1, K, offset=802)
+    ref = oracle.linear_w4(X, codes, scales, biases, N, K, G)
+    dc, ds, db = dev_params(codes, scales, biases)
+    Y = tq.w4_gemv(to_dev_bf16(X), dc, ds, db, N, K, G, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert_rows_close_f32(to_f64(Y), ref)
+
+
+def test_w4_gemv_stream_unaligned_operands():
+    """Scales and biases views that start 2 bytes in (not 4-byte aligned): the
+    streaming kernel declines and the row kernel answers."""
+    N, K, G = 16411, 1024, 128
+    codes, scales, biases = synthetic.w4_params(N, K, G, index=6)
+    X = synthetic.activations(1, K, offset=803)
+    ref = oracle.linear_w4(X, codes, scales, biases, N, K, G)
+    dc, ds, db = dev_params(codes, scales, biases)
+    flat_s = torch.empty(ds.numel() + 1, dtype=torch.bfloat16, device="cuda")
+    flat_s[1:] = ds.reshape(-1)
+    flat_b = torch.empty(db.numel() + 1, dtype=torch.bfloat16, device="cuda")
+    flat_b[1:] = db.reshape(-1)
+    Y = tq.w4_gemv(to_dev_bf16(X), dc, flat_s[1:].view(N, K // G), flat_b[1:].view(N, K // G), N, K, G,
+                   out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert_rows_close_f32(to_f64(Y), ref)
+
+
 @pytest.mark.parametrize("M", [1, 16, 256, 300])
 @pytest.mark.parametrize("N,K,G", [(512, 1024, 128), (1000, 4096, 64), (4096, 1024, 128), (130, 2048, 256)])
 def test_w4_gemm_tensor_cores(N, K, G, M):
