@@ -217,11 +217,13 @@ TQ_API size_t tq_w4_codes_bytes(int64_t N, int64_t K, int G);
  * launch): Y[m][n] = sum_g (s[n][g] * sum_{j in g} q[n][j] X[m][j] + b[n][g] *
  * sum_{j in g} X[m][j]) with fp32 accumulation ("Stage 2: SIMD Matvec" factors
  * the bias out of the group's dot product), written as fp32 or RNE bf16.
- * Ordering rule as tq_gemv.  One token over 16 Mi weights and more, with
- * G in {64, 128}, K a multiple of 256 up to 2048, 8-byte-aligned codes and
- * scales and biases aligned to 4 bytes (G = 128) or 8 (G = 64), takes the
- * streaming lookup-table kernel (one 256-column slice of tables per CTA,
- * the slices of a row over a thread-block cluster); other shapes with
+ * Ordering rule as tq_gemv.  G in {64, 128}, K a multiple of 256 up to
+ * 2048, 8-byte-aligned codes and scales and biases aligned to 4 bytes
+ * (G = 128) or 8 (G = 64) take the streaming lookup-table kernel (one
+ * 256-column slice of tables per CTA, the slices of a row over a
+ * thread-block cluster), one launch per token, for one token from 12 Mi
+ * weights (6 Mi at K >= 2048) and for 2..4 tokens from 12 Mi weights at
+ * K <= 512 or from 96 Mi weights at any K; other shapes with
  * G % 32 == 0, K % 32 == 0 and K <= 4096 the CUDA-core streaming kernel,
  * eight tokens per launch, and the rest a plain one-warp-per-row kernel.
  * Errors: TQ_ERR_INVALID_ARG (shapes, G % 8, nulls, Y overlapping an input),

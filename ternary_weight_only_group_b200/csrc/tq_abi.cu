@@ -206,9 +206,19 @@ tq_status tq_unpack_bf16(const uint8_t* codes, const void* scales, int64_t N, in
 // cudaErrorNotSupported, having launched nothing, when the kernel does not
 // cover the shape.
 constexpr int64_t kStreamMaxTokens = 4;
-// tq_w4_gemv: tokens and weights from which the streaming kernel runs
-constexpr int64_t kW4StreamMaxTokens = 1;
-constexpr int64_t kW4StreamMinWeights = (int64_t)16 << 20;
+// tq_w4_gemv: whether the streaming lookup-table kernel, once per token,
+// beats the CUDA-core kernel (all tokens in one pass).  Measured on B200:
+// one token from about 12 Mi weights (6 Mi at K >= 2048): 14336 x 1024 5.8
+// us against 6.1, 8192 x 1024 5.5 against 4.3, 4096 x 2048 5.7 against 9.2;
+// 2..4 tokens where the CUDA-core kernel has few 32-column chunks per row
+// (K <= 512: 65536 x 512 at 4 tokens 32 us against 50) or from 96 Mi weights
+// (172032 x 1024 at 4 tokens 112 us against 132; 57344 x 1024 49 against 48).
+constexpr int64_t kW4StreamMaxTokens = 4;
+static bool w4_stream_wins(int64_t M, int64_t N, int64_t K) {
+    const int64_t nk = N * K;
+    if (M < 1 || M > kW4StreamMaxTokens || nk < (K >= 2048 ? (int64_t)6 << 20 : (int64_t)12 << 20)) return false;
+    return M == 1 || K <= 512 || nk >= (int64_t)96 << 20;
+}
 constexpr int64_t kStreamMinWeightsMulti = (int64_t)48 << 20;
 static cudaError_t stream_per_token(const void* X, int64_t M, const uint8_t* codes, const void* scales, int64_t N,
                                     int64_t K, int G, void* Y, tq_out_dtype yt, uint32_t* d_err, cudaStream_t stream,
@@ -437,9 +447,9 @@ tq_status tq_w4_gemv(const void* X, int64_t M, const uint32_t* codes, const void
     if (K == 0) return from_cuda(cudaMemsetAsync(Y, 0, yb, (cudaStream_t)stream));  // empty sums
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
-    // 1..kW4StreamMaxTokens tokens over a large matrix: the streaming
-    // lookup-table kernel once per token (tables of 256 columns per CTA)
-    if (M <= kW4StreamMaxTokens && N * K >= kW4StreamMinWeights) {
+    // 1..4 tokens over a large matrix: the streaming lookup-table kernel once
+    // per token (tables of 256 columns per CTA)
+    if (w4_stream_wins(M, N, K)) {
         const size_t ysz = yt == TQ_OUT_BF16 ? 2 : 4;
         cudaError_t e = cudaSuccess;
         for (int64_t m = 0; m < M && e == cudaSuccess; ++m)

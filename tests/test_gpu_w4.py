@@ -80,6 +80,20 @@ def test_w4_gemv_stream(K, G):
     check(N, K, G, 1, index=K + 3 * G)
 
 
+@pytest.mark.parametrize("M", [2, 3, 4])
+@pytest.mark.parametrize("N,K,G", [(24593, 512, 128), (49157, 256, 64)])
+def test_w4_gemv_stream_tokens(N, K, G, M):
+    """2..4 tokens at K <= 512 over 12 Mi weights and more: one streaming
+    launch per token."""
+    check(N, K, G, M, index=M + K)
+
+
+def test_w4_gemv_stream_tokens_large():
+    """Two tokens over 96 Mi weights and more (K = 1024): one streaming launch
+    per token."""
+    check(98317, 1024, 128, 2, index=17, dtypes=(torch.bfloat16,))
+
+
 def test_w4_gemv_stream_every_byte():
     """Every code byte (two nibbles) in every byte position of the tables:
     row n, word w, byte i holds (n + 8 w + i) mod 256."""
