@@ -33,10 +33,15 @@ using namespace tc;
 
 constexpr int WM = 128;  // W rows per CTA (UMMA M)
 constexpr int BK = 64;
-// Pipeline depth: 4 stages for 16-token tiles (97 KB of shared memory) and 3
-// for 32-token tiles (89 KB), so two CTAs fit per SM; 6 for 64-token tiles.
+// Pipeline depth of the decoded W tiles: 4 stages for 16-token tiles and 3
+// for 32-token tiles, so two CTAs fit per SM (106 and 103 KB of shared
+// memory); 6 for 64-token tiles.  The X tiles have a ring of their own, as
+// deep as a CTA's K slice usually is, so every X load is issued as soon as
+// the activations are ready instead of one W stage at a time.
 template <int NT>
 constexpr int kStages = NT == 16 ? 4 : (NT == 32 ? 3 : 6);
+template <int NT>
+constexpr int kXStages = NT == 32 ? 6 : 8;
 constexpr int kThreads = 256;
 constexpr int kDecodeWarp0 = 4, kDecodeWarps = 4;
 constexpr uint32_t W_STAGE = WM * BK * 2;  // 16 KB
@@ -46,13 +51,16 @@ constexpr int kMaxCS = 8;
 
 template <int NT>
 struct Smem {
-    static constexpr int STAGES = kStages<NT>;
+    static constexpr int STAGES = kStages<NT>, XS = kXStages<NT>;
     uint8_t w[STAGES][W_STAGE];   // decoded W tiles (UMMA A), 1024-byte aligned
-    uint8_t x[STAGES][NT * 128];  // X tiles (UMMA B): NT rows of 128 bytes
+    uint8_t x[XS][NT * 128];      // X tiles (UMMA B): NT rows of 128 bytes
     uint8_t c[STAGES][C_STAGE];   // code-byte windows
-    float red[WM * NT];           // partials pushed by the cluster: [rank][row of owner][token]
+    // partials pushed by the cluster: [rank][row of owner][token], rows NT + 4
+    // floats apart, so that eight lanes storing or loading 16 bytes of eight
+    // consecutive rows cover all 32 banks
+    float red[WM * (NT + 4)];
     uint32_t lut[256];                // byte -> PRMT selectors of its digits 0..3
-    uint64_t full_x[STAGES], full_c[STAGES], full_w[STAGES], empty[STAGES], done;
+    uint64_t full_x[XS], xempty[XS], full_c[STAGES], full_w[STAGES], empty[STAGES], done;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -77,7 +85,7 @@ template <int NT, bool CODES_TMA, int FMT>
 __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                  const __grid_constant__ CUtensorMap tmap_c,
                                                                  const Params p) {
-    constexpr int STAGES = kStages<NT>;
+    constexpr int STAGES = kStages<NT>, XS = kXStages<NT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem<NT>& sm = *reinterpret_cast<Smem<NT>*>(smem_raw + ((1024 - (s32(smem_raw) & 1023)) & 1023));
     cg::cluster_group cluster = cg::this_cluster();
@@ -99,10 +107,13 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
     if (FMT == 3) fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES; ++st) {
-            mbar_init(&sm.full_x[st], 1);
             mbar_init(&sm.full_c[st], 1);
             mbar_init(&sm.full_w[st], kDecodeWarps);
             mbar_init(&sm.empty[st], 1);
+        }
+        for (int xs = 0; xs < XS; ++xs) {
+            mbar_init(&sm.full_x[xs], 1);
+            mbar_init(&sm.xempty[xs], 1);
         }
         mbar_init(&sm.done, 1);
         sm.abort_flag = 0;
@@ -130,47 +141,61 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
 
     if (warp == 0) {
         if (lane == 0) {
-            asm volatile("griddepcontrol.wait;" ::: "memory");  // X comes from the preceding kernel
-            int issued = 0;
-            for (int i = 0; i < nkl; ++i) {
-                const int kb = kb_lo + i, st = i % STAGES, use = i / STAGES;
-                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
+            // Code windows (weights: independent of the preceding kernel) of the
+            // first stages go out before the grid-dependency wait, every X tile
+            // the X ring holds right after it, the rest as stages free up.
+            auto load_c = [&](int i) {
                 int g, c0, q_lo;
-                stage_geom(kb, g, c0, q_lo);
-                if (!(p.wc.withhold_x && i == 0)) {  // test hook: the first load left out
-                    mbar_arrive_expect_tx(&sm.full_x[st], NT * 128);
-                    tma_load_2d(sm.x[st], &tmap_x, kb * BK, 0, &sm.full_x[st]);
+                stage_geom(kb_lo + i, g, c0, q_lo);
+                mbar_arrive_expect_tx(&sm.full_c[i % STAGES], C_STAGE);
+                tma_load_2d(sm.c[i % STAGES], &tmap_c, (g * p.B + q_lo) & ~15, (int)n0, &sm.full_c[i % STAGES]);
+            };
+            auto load_x = [&](int i) {
+                if (p.wc.withhold_x && i == 0) return;  // test hook: the first load left out
+                mbar_arrive_expect_tx(&sm.full_x[i % XS], NT * 128);
+                tma_load_2d(sm.x[i % XS], &tmap_x, (kb_lo + i) * BK, 0, &sm.full_x[i % XS]);
+            };
+            int ci = 0, xi = 0;  // code windows and X tiles issued
+            if (CODES_TMA)
+                for (; ci < nkl && ci < STAGES; ++ci) load_c(ci);
+            asm volatile("griddepcontrol.wait;" ::: "memory");  // X comes from the preceding kernel
+            for (; xi < nkl && xi < XS; ++xi) load_x(xi);
+            for (int i = 0; i < nkl; ++i) {
+                if (CODES_TMA && i >= STAGES) {
+                    if (!mbar_wait(&sm.empty[i % STAGES], (i / STAGES - 1) & 1, abort_flag, lim)) break;
+                    load_c(i);
+                    ci = i + 1;
                 }
-                if (CODES_TMA) {
-                    mbar_arrive_expect_tx(&sm.full_c[st], C_STAGE);
-                    tma_load_2d(sm.c[st], &tmap_c, (g * p.B + q_lo) & ~15, (int)n0, &sm.full_c[st]);
+                if (i >= XS) {
+                    if (!mbar_wait(&sm.xempty[i % XS], (i / XS - 1) & 1, abort_flag, lim)) break;
+                    load_x(i);
+                    xi = i + 1;
                 }
-                ++issued;
             }
-            for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
-                const int st = i % STAGES, use = i / STAGES;
-                const uint64_t t0 = globaltimer();
-                while (!mbar_try_wait(&sm.full_x[st], use & 1) && globaltimer() - t0 < lim) {
+            // let every copy in flight land before the CTA can exit
+            const uint64_t t0 = globaltimer();
+            for (int i = (xi > XS ? xi - XS : 0); i < xi; ++i)
+                while (!mbar_try_wait(&sm.full_x[i % XS], (i / XS) & 1) && globaltimer() - t0 < lim) {
                 }
-                if (CODES_TMA)
-                    while (!mbar_try_wait(&sm.full_c[st], use & 1) && globaltimer() - t0 < lim) {
-                    }
-            }
+            for (int i = (ci > STAGES ? ci - STAGES : 0); i < ci; ++i)
+                while (!mbar_try_wait(&sm.full_c[i % STAGES], (i / STAGES) & 1) && globaltimer() - t0 < lim) {
+                }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = instr_desc(WM, NT);
             for (int i = 0; i < nkl; ++i) {
                 const int st = i % STAGES, use = i / STAGES;
-                if (!mbar_wait(&sm.full_x[st], use & 1, abort_flag, lim)) break;
+                if (!mbar_wait(&sm.full_x[i % XS], (i / XS) & 1, abort_flag, lim)) break;
                 if (!mbar_wait(&sm.full_w[st], use & 1, abort_flag, lim)) break;
                 tc_fence_after();
-                const uint32_t a0 = s32(sm.w[st]), b0 = s32(sm.x[st]);
+                const uint32_t a0 = s32(sm.w[st]), b0 = s32(sm.x[i % XS]);
 #pragma unroll
                 for (int k = 0; k < BK / 16; ++k)
                     mma_bf16(tmem, smem_desc_sw128(a0 + 32 * k), smem_desc_sw128(b0 + 32 * k), idesc,
                              (i > 0 || k > 0) ? 1u : 0u);
                 mma_commit(&sm.empty[st]);
+                mma_commit(&sm.xempty[i % XS]);
             }
             mma_commit(&sm.done);
         }
@@ -261,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
             for (int j = 0; j < NT; ++j) v[j] = 0x7FC00000u;
         }
         const int owner = r / RPQ;
-        float* dst = cluster.map_shared_rank(sm.red, owner) + ((crank * RPQ) + (r - owner * RPQ)) * NT;
+        float* dst = cluster.map_shared_rank(sm.red, owner) + ((crank * RPQ) + (r - owner * RPQ)) * (NT + 4);
 #pragma unroll
         for (int j = 0; j < NT; j += 4)
             *reinterpret_cast<float4*>(dst + j) = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
@@ -270,21 +295,37 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
     tc_fence_before();
     cluster.sync();
     tc_fence_after();
-    // owner: rows [crank*RPQ, (crank+1)*RPQ) of the tile, all tokens
+    // owner: rows [crank*RPQ, (crank+1)*RPQ) of the tile, all tokens; a thread
+    // adds four tokens of one row (16-byte loads), consecutive lanes take
+    // consecutive rows, so each token's stores cover consecutive outputs
     const int64_t Mv = p.M < NT ? p.M : NT;
+    const int MQ = (int)((Mv + 3) / 4);
     uint32_t err_acc = 0;
-    for (int i = threadIdx.x; i < RPQ * Mv; i += kThreads) {
-        const int m = i / RPQ, rr = i - m * RPQ;
-        float acc = 0.f;
-        for (int qr = 0; qr < p.CS; ++qr) acc += sm.red[(qr * RPQ + rr) * NT + m];
+    for (int i = threadIdx.x; i < RPQ * MQ; i += kThreads) {
+        const int mq = i / RPQ, rr = i - mq * RPQ;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int qr = 0; qr < p.CS; ++qr) {
+            const float4 v4 = *reinterpret_cast<const float4*>(&sm.red[(qr * RPQ + rr) * (NT + 4) + 4 * mq]);
+            acc.x += v4.x;
+            acc.y += v4.y;
+            acc.z += v4.z;
+            acc.w += v4.w;
+        }
         const int64_t n = n0 + crank * RPQ + rr;
         if (n < p.N) {
-            if (m == 0 && acc != acc)  // NaN output of the first token: rescan that W row
+            const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+            if (mq == 0 && acc.x != acc.x)  // NaN output of the first token: rescan that W row
                 err_acc |= FMT == 3 ? scan_row_errors(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G, p.B)
                                     : scan_row_errors2(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G);
-            const int64_t o = (int64_t)m * p.N + n;
-            if (p.y_bf16) reinterpret_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(acc);
-            else reinterpret_cast<float*>(p.Y)[o] = acc;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int64_t m = 4 * mq + t;
+                if (m < Mv) {
+                    const int64_t o = m * p.N + n;
+                    if (p.y_bf16) reinterpret_cast<__nv_bfloat16*>(p.Y)[o] = __float2bfloat16_rn(a4[t]);
+                    else reinterpret_cast<float*>(p.Y)[o] = a4[t];
+                }
+            }
         }
     }
 
@@ -363,7 +404,9 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     if (tiles * kMaxCS > 0x7FFFFFFF) return cudaSuccess;
     // split K so the grid covers the SMs, keeping at least two stages per CTA
     int CS = 1;
-    const int64_t slots = (M <= 32 ? 2 : 1) * (int64_t)sm_count;  // resident CTAs (16/32-token tiles: two per SM)
+    // at most one CTA per SM: the next dependent launch finds a free slot on
+    // every SM (16/32-token tiles fit twice) and decodes before its wait
+    const int64_t slots = (int64_t)sm_count;
     while (CS < kMaxCS && tiles * CS * 2 <= slots && nk / (CS * 2) >= 2) CS *= 2;
     if (CS == 1)  // no K split: the persistent kernel walks the tiles
         return launch_gemm_stream(X, M, codes, scales, N, K, G, Y, y_bf16, d_err, stream, sm_count, handled, fmt);
