@@ -6,14 +6,18 @@
 // the decode and matrix schedules are chosen by M), for 5 <= M <= 64 tokens.
 // The roles of the operands are swapped so the tensor core's 128-row side is
 // filled by weights:  D^T[128 W rows x NT tokens] += What[128 x 16] . X[NT x 16]^T
-// with What decoded on chip into the 128-byte-swizzled K-major layout (as in
-// the prefill GEMM) and X tiles (NT = 16, 32 or 64 rows, zero-filled past M)
-// loaded by TMA.  K is split across the CTAs of a thread-block cluster; each
-// CTA pushes its fp32 partial tile into the shared memory of the rank that
-// owns those rows (distributed shared memory), one cluster barrier, and the
-// owner adds the partials in rank order (deterministic) and writes Y.
-//   warp 0  TMA producer (X tile and the stage's code-byte window)
-//   warp 1  MMA issuer (tcgen05.mma kind::f16, M=128, N=NT, fp32 in TMEM)
+// with What decoded on chip straight into tensor memory (each decoder thread
+// owns one W row = one tensor-memory lane and stores its 64 bf16 of a stage
+// with tcgen05.st), where the MMA reads it as the A operand, and X tiles
+// (NT = 16, 32 or 64 rows, zero-filled past M) loaded by TMA.  K is split
+// across the CTAs of a thread-block cluster; each CTA pushes its fp32 partial
+// tile into the shared memory of the rank that owns those rows (distributed
+// shared memory), one cluster barrier, and the owner adds the partials in
+// rank order (deterministic) and writes Y.  In a chain of launches a CTA
+// decodes (up to seven stages) while the preceding kernel still runs: only
+// the X loads wait for it.
+//   warp 0  TMA producer (code-byte windows, then X tiles)
+//   warp 1  MMA issuer (tcgen05.mma kind::f16, M=128, N=NT, A in tensor memory)
 //   warp 2  tensor-memory allocation
 //   warps 4-7  decoders (one W row per thread), then the epilogue
 // All mbarrier waits are bounded (globaltimer deadline -> TQ_DERR_TIMEOUT).
@@ -33,34 +37,41 @@ using namespace tc;
 
 constexpr int WM = 128;  // W rows per CTA (UMMA M)
 constexpr int BK = 64;
-// Pipeline depth of the decoded W tiles: 4 stages for 16-token tiles and 3
-// for 32-token tiles, so two CTAs fit per SM (106 and 103 KB of shared
-// memory); 6 for 64-token tiles.  The X tiles have a ring of their own, as
-// deep as a CTA's K slice usually is, so every X load is issued as soon as
-// the activations are ready instead of one W stage at a time.
+// Tensor memory: 256 columns per CTA (two CTAs per SM use all 512): the
+// accumulator D in columns [0, ACC) and WSL slots of decoded W, 32 columns
+// (one 128 x 64 bf16 stage) each, as the MMA's A operand.  Shared memory
+// holds no decoded weights: X tiles in a ring of XS, code windows in a ring
+// of CST (deep enough for a CTA's whole K slice at the shapes that take this
+// kernel), so every code window is requested before the grid-dependency wait
+// and every X tile right after it.
+constexpr uint32_t kCols = 256;
 template <int NT>
-constexpr int kStages = NT == 16 ? 4 : (NT == 32 ? 3 : 6);
+constexpr int kAcc = NT < 32 ? 32 : NT;
 template <int NT>
-constexpr int kXStages = NT == 32 ? 6 : 8;
+constexpr int kWSlots = (int)(kCols - kAcc<NT>) / 32;  // 7, 7, 6
+template <int NT>
+constexpr int kXStages = NT == 64 ? 4 : 8;
+constexpr int kCStages = 8;
 constexpr int kThreads = 256;
 constexpr int kDecodeWarp0 = 4, kDecodeWarps = 4;
-constexpr uint32_t W_STAGE = WM * BK * 2;  // 16 KB
 constexpr uint32_t C_ROW = 32;
 constexpr uint32_t C_STAGE = WM * C_ROW;   // 4 KB
 constexpr int kMaxCS = 8;
+// At least this much dynamic shared memory per CTA, so that no more than two
+// CTAs (2 x 256 tensor-memory columns) ever share an SM.
+constexpr size_t kMinSmem = 80 * 1024;
 
 template <int NT>
 struct Smem {
-    static constexpr int STAGES = kStages<NT>, XS = kXStages<NT>;
-    uint8_t w[STAGES][W_STAGE];   // decoded W tiles (UMMA A), 1024-byte aligned
-    uint8_t x[XS][NT * 128];      // X tiles (UMMA B): NT rows of 128 bytes
-    uint8_t c[STAGES][C_STAGE];   // code-byte windows
+    static constexpr int XS = kXStages<NT>, CST = kCStages, WSL = kWSlots<NT>;
+    uint8_t x[XS][NT * 128];      // X tiles (UMMA B): NT rows of 128 bytes, 1024-byte aligned
+    uint8_t c[CST][C_STAGE];      // code-byte windows
     // partials pushed by the cluster: [rank][row of owner][token], rows NT + 4
     // floats apart, so that eight lanes storing or loading 16 bytes of eight
     // consecutive rows cover all 32 banks
     float red[WM * (NT + 4)];
     uint32_t lut[256];                // byte -> PRMT selectors of its digits 0..3
-    uint64_t full_x[XS], xempty[XS], full_c[STAGES], full_w[STAGES], empty[STAGES], done;
+    uint64_t full_x[XS], xempty[XS], full_c[CST], cempty[CST], full_w[WSL], wempty[WSL], done;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -82,10 +93,11 @@ struct Params {
 // FMT 3: base-3 codes (five digits per byte); FMT 2: the 2-bit format (four
 // codes per byte, G a multiple of 64: a stage's 64 codes are 16 whole bytes).
 template <int NT, bool CODES_TMA, int FMT>
-__global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
+__global__ void __launch_bounds__(kThreads, 2) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                  const __grid_constant__ CUtensorMap tmap_c,
                                                                  const Params p) {
-    constexpr int STAGES = kStages<NT>, XS = kXStages<NT>;
+    constexpr int XS = kXStages<NT>, CST = kCStages, WSL = kWSlots<NT>;
+    constexpr uint32_t ACC = kAcc<NT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem<NT>& sm = *reinterpret_cast<Smem<NT>*>(smem_raw + ((1024 - (s32(smem_raw) & 1023)) & 1023));
     cg::cluster_group cluster = cg::this_cluster();
@@ -95,7 +107,6 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
     const int nk = p.K / BK;
     const int kb_lo = (int)((int64_t)nk * crank / p.CS), kb_hi = (int)((int64_t)nk * (crank + 1) / p.CS);
     const int nkl = kb_hi - kb_lo;  // stages of this CTA (>= 1)
-    constexpr uint32_t kCols = NT < 32 ? 32 : NT;
     volatile int* abort_flag = &sm.abort_flag;
     const uint64_t lim = p.wc.limit_ns;
 
@@ -106,14 +117,17 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
     cluster_arrive_relaxed();  // waited on before the first store into a peer's shared memory
     if (FMT == 3) fill_digit_selector_lut4(sm.lut, threadIdx.x, kThreads);
     if (threadIdx.x == 0) {
-        for (int st = 0; st < STAGES; ++st) {
-            mbar_init(&sm.full_c[st], 1);
-            mbar_init(&sm.full_w[st], kDecodeWarps);
-            mbar_init(&sm.empty[st], 1);
+        for (int i = 0; i < XS; ++i) {
+            mbar_init(&sm.full_x[i], 1);
+            mbar_init(&sm.xempty[i], 1);
         }
-        for (int xs = 0; xs < XS; ++xs) {
-            mbar_init(&sm.full_x[xs], 1);
-            mbar_init(&sm.xempty[xs], 1);
+        for (int i = 0; i < CST; ++i) {
+            mbar_init(&sm.full_c[i], 1);
+            mbar_init(&sm.cempty[i], kDecodeWarps);
+        }
+        for (int i = 0; i < WSL; ++i) {
+            mbar_init(&sm.full_w[i], kDecodeWarps);
+            mbar_init(&sm.wempty[i], 1);
         }
         mbar_init(&sm.done, 1);
         sm.abort_flag = 0;
@@ -141,14 +155,11 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
 
     if (warp == 0) {
         if (lane == 0) {
-            // Code windows (weights: independent of the preceding kernel) of the
-            // first stages go out before the grid-dependency wait, every X tile
-            // the X ring holds right after it, the rest as stages free up.
             auto load_c = [&](int i) {
                 int g, c0, q_lo;
                 stage_geom(kb_lo + i, g, c0, q_lo);
-                mbar_arrive_expect_tx(&sm.full_c[i % STAGES], C_STAGE);
-                tma_load_2d(sm.c[i % STAGES], &tmap_c, (g * p.B + q_lo) & ~15, (int)n0, &sm.full_c[i % STAGES]);
+                mbar_arrive_expect_tx(&sm.full_c[i % CST], C_STAGE);
+                tma_load_2d(sm.c[i % CST], &tmap_c, (g * p.B + q_lo) & ~15, (int)n0, &sm.full_c[i % CST]);
             };
             auto load_x = [&](int i) {
                 if (p.wc.withhold_x && i == 0) return;  // test hook: the first load left out
@@ -157,12 +168,12 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
             };
             int ci = 0, xi = 0;  // code windows and X tiles issued
             if (CODES_TMA)
-                for (; ci < nkl && ci < STAGES; ++ci) load_c(ci);
+                for (; ci < nkl && ci < CST; ++ci) load_c(ci);
             asm volatile("griddepcontrol.wait;" ::: "memory");  // X comes from the preceding kernel
             for (; xi < nkl && xi < XS; ++xi) load_x(xi);
             for (int i = 0; i < nkl; ++i) {
-                if (CODES_TMA && i >= STAGES) {
-                    if (!mbar_wait(&sm.empty[i % STAGES], (i / STAGES - 1) & 1, abort_flag, lim)) break;
+                if (CODES_TMA && i >= CST) {
+                    if (!mbar_wait(&sm.cempty[i % CST], (i / CST - 1) & 1, abort_flag, lim)) break;
                     load_c(i);
                     ci = i + 1;
                 }
@@ -177,30 +188,30 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
             for (int i = (xi > XS ? xi - XS : 0); i < xi; ++i)
                 while (!mbar_try_wait(&sm.full_x[i % XS], (i / XS) & 1) && globaltimer() - t0 < lim) {
                 }
-            for (int i = (ci > STAGES ? ci - STAGES : 0); i < ci; ++i)
-                while (!mbar_try_wait(&sm.full_c[i % STAGES], (i / STAGES) & 1) && globaltimer() - t0 < lim) {
+            for (int i = (ci > CST ? ci - CST : 0); i < ci; ++i)
+                while (!mbar_try_wait(&sm.full_c[i % CST], (i / CST) & 1) && globaltimer() - t0 < lim) {
                 }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = instr_desc(WM, NT);
             for (int i = 0; i < nkl; ++i) {
-                const int st = i % STAGES, use = i / STAGES;
+                const int st = i % WSL;
                 if (!mbar_wait(&sm.full_x[i % XS], (i / XS) & 1, abort_flag, lim)) break;
-                if (!mbar_wait(&sm.full_w[st], use & 1, abort_flag, lim)) break;
+                if (!mbar_wait(&sm.full_w[st], (i / WSL) & 1, abort_flag, lim)) break;
                 tc_fence_after();
-                const uint32_t a0 = s32(sm.w[st]), b0 = s32(sm.x[i % XS]);
+                const uint32_t a0 = tmem + ACC + 32u * (uint32_t)st, b0 = s32(sm.x[i % XS]);
 #pragma unroll
                 for (int k = 0; k < BK / 16; ++k)
-                    mma_bf16(tmem, smem_desc_sw128(a0 + 32 * k), smem_desc_sw128(b0 + 32 * k), idesc,
-                             (i > 0 || k > 0) ? 1u : 0u);
-                mma_commit(&sm.empty[st]);
+                    mma_bf16_ts(tmem, a0 + 8u * k, smem_desc_sw128(b0 + 32 * k), idesc, (i > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&sm.wempty[st]);
                 mma_commit(&sm.xempty[i % XS]);
             }
             mma_commit(&sm.done);
         }
     } else if (warp >= kDecodeWarp0) {
-        const int t = threadIdx.x - kDecodeWarp0 * 32;  // W row of the tile
+        const int t = threadIdx.x - kDecodeWarp0 * 32;  // W row of the tile = tensor-memory lane
+        const uint32_t trow = tmem + ((uint32_t)(32 * (warp - kDecodeWarp0)) << 16) + ACC;
         const int64_t n = n0 + t;
         const uint16_t* srow = p.scales + (n < p.N ? n : 0) * p.ng;
         const uint8_t* crow = p.codes + (n < p.N ? n : 0) * p.row_bytes;
@@ -215,51 +226,65 @@ __global__ void __launch_bounds__(kThreads, NT <= 32 ? 2 : 1) gemm_small_kernel(
         if (!CODES_TMA && FMT == 3 && nkl > 0) load_global(kb_lo, cur);
         uint32_t sc_nxt = nkl > 0 ? __ldg(srow + (kb_lo * BK) / p.G) : 0u;
         for (int i = 0; i < nkl; ++i) {
-            const int kb = kb_lo + i, st = i % STAGES, use = i / STAGES;
+            const int kb = kb_lo + i, st = i % WSL, use = i / WSL;
             int g, c0, q_lo;
             stage_geom(kb, g, c0, q_lo);
             const uint32_t sc = sc_nxt;
             if (i + 1 < nkl) sc_nxt = __ldg(srow + ((kb + 1) * BK) / p.G);  // next stage's scale in flight
+            uint32_t wv[32];
+            auto put = [&](int k, uint4 v) {
+                wv[4 * k] = v.x;
+                wv[4 * k + 1] = v.y;
+                wv[4 * k + 2] = v.z;
+                wv[4 * k + 3] = v.w;
+            };
+            // the window's bytes are in registers: the window may be refilled
+            auto release_window = [&]() {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.cempty[i % CST]);
+            };
             if constexpr (FMT == 2) {
                 // the stage's 16 code bytes start on a 16-byte boundary of the row
                 uint32_t wd[4];
                 if (CODES_TMA) {
-                    if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag, lim)) break;
-                    const uint4 v = *reinterpret_cast<const uint4*>(sm.c[st] + t * C_ROW);
+                    if (!mbar_wait(&sm.full_c[i % CST], (i / CST) & 1, abort_flag, lim)) break;
+                    const uint4 v = *reinterpret_cast<const uint4*>(sm.c[i % CST] + t * C_ROW);
                     wd[0] = v.x, wd[1] = v.y, wd[2] = v.z, wd[3] = v.w;
+                    release_window();
                 } else {
-                    if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
                     const uint32_t* cw = reinterpret_cast<const uint32_t*>(crow + (int64_t)g * p.B + q_lo);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) wd[j] = __ldg(cw + j);
                 }
-                decode_stage64_2bit(wd, sc, sm.w[st] + t * 128, t & 7);
+                if (use > 0 && !mbar_wait(&sm.wempty[st], (use - 1) & 1, abort_flag, lim)) break;
+                decode_stage64_2bit_to(wd, sc, put);
             } else {
-            const int ql = p.B - 1 - q_lo;  // the group's last byte relative to q_lo
-            uint32_t bytes[14], lastb = 0;
-            if (CODES_TMA) {
-                if (!mbar_wait(&sm.full_c[st], use & 1, abort_flag, lim)) break;
-                const int off = (g * p.B + q_lo) & 15;
-                const uint8_t* win = sm.c[st] + t * C_ROW;
-                window_bytes(win, off, bytes);
-                if (ql < 14) lastb = win[off + ql];
-            } else {
-                if (i + 1 < nkl) load_global(kb + 1, nxt);  // next stage's bytes in flight
-                if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
+                const int ql = p.B - 1 - q_lo;  // the group's last byte relative to q_lo
+                uint32_t bytes[14], lastb = 0;
+                if (CODES_TMA) {
+                    if (!mbar_wait(&sm.full_c[i % CST], (i / CST) & 1, abort_flag, lim)) break;
+                    const int off = (g * p.B + q_lo) & 15;
+                    const uint8_t* win = sm.c[i % CST] + t * C_ROW;
+                    window_bytes(win, off, bytes);
+                    if (ql < 14) lastb = win[off + ql];
+                    release_window();
+                } else {
+                    if (i + 1 < nkl) load_global(kb + 1, nxt);  // next stage's bytes in flight
 #pragma unroll
-                for (int j = 0; j < 14; ++j) bytes[j] = cur[j];
-                if (ql < 14) lastb = __ldg(crow + (int64_t)g * p.B + p.B - 1);
+                    for (int j = 0; j < 14; ++j) bytes[j] = cur[j];
+                    if (ql < 14) lastb = __ldg(crow + (int64_t)g * p.B + p.B - 1);
+                }
+                if (use > 0 && !mbar_wait(&sm.wempty[st], (use - 1) & 1, abort_flag, lim)) break;
+                decode_stage64_to<1>(sm.lut, bytes, c0 - 5 * q_lo, ql < 14, lastb, p.pad_base, p.pad_span, sc, put);
+                if (!CODES_TMA) {
+#pragma unroll
+                    for (int j = 0; j < 14; ++j) cur[j] = nxt[j];
+                }
             }
-            decode_stage64(sm.lut, bytes, c0 - 5 * q_lo, ql < 14, lastb, p.pad_base, p.pad_span, sc,
-                           sm.w[st] + t * 128, t & 7);
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tmem_st32(trow + 32u * (uint32_t)st, wv);
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_w[st]);
-            if (!CODES_TMA && FMT == 3) {
-#pragma unroll
-                for (int j = 0; j < 14; ++j) cur[j] = nxt[j];
-            }
         }
     }
 
@@ -350,7 +375,7 @@ template <int NT, bool CT, int FMT>
 static cudaError_t launch_nt(const CUtensorMap& tx, const CUtensorMap& tc_, const Params& p, int tiles,
                              cudaStream_t stream) {
     auto kern = gemm_small_kernel<NT, CT, FMT>;
-    const size_t smem = sizeof(Smem<NT>) + 1024;
+    const size_t smem = sizeof(Smem<NT>) + 1024 > kMinSmem ? sizeof(Smem<NT>) + 1024 : kMinSmem;
     static SmemAttr smem_attr;
     if (cudaError_t e = smem_attr.ensure(kern, (int)smem)) return e;
     cudaLaunchConfig_t cfg = {};

@@ -110,6 +110,16 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
         "l"(a), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
+// The same MMA with A read from tensor memory (rows in lanes 0..127, two bf16
+// of a row per 32-bit column, K order), B from shared memory.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                            uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+            d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(s32(bar))
                  : "memory");
@@ -127,6 +137,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 32 consecutive columns of this thread's lane (warp quadrant's 32 lanes),
+// followed by the wait for the stores to land.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -189,11 +213,11 @@ __device__ __forceinline__ void window_bytes(const uint8_t* row32, int off, uint
 // bytes is packed into words by PRMT and funnel-shifted by r0 bytes, so every
 // stage takes the same code.  A rejected scale or padding digit makes the
 // row's stage NaN.  Writes the 128-byte swizzled K-major tile row.
-template <int LUT_STRIDE = 1>
-__device__ __forceinline__ void decode_stage64(const uint32_t* lut4, const uint32_t (&bytes)[14], int r0,
-                                               bool check_pad, uint32_t lastb, uint32_t pad_base,
-                                               uint32_t pad_span, uint32_t scale_bits, uint8_t* tile_row,
-                                               int row_in_atom) {
+// `put(k, v)` receives the decoded columns 8k .. 8k+7 as four bf16 pairs.
+template <int LUT_STRIDE, class Put>
+__device__ __forceinline__ void decode_stage64_to(const uint32_t* lut4, const uint32_t (&bytes)[14], int r0,
+                                                  bool check_pad, uint32_t lastb, uint32_t pad_base,
+                                                  uint32_t pad_span, uint32_t scale_bits, Put&& put) {
     uint2 e[14];
 #pragma unroll
     for (int i = 0; i < 14; ++i) {
@@ -228,9 +252,16 @@ __device__ __forceinline__ void decode_stage64(const uint32_t* lut4, const uint3
     for (int k = 0; k < 8; ++k) {
         const uint32_t o0 = __funnelshift_rc(W[2 * k], W[2 * k + 1], sh);
         const uint32_t o1 = __funnelshift_rc(W[2 * k + 1], W[2 * k + 2], sh);
-        *reinterpret_cast<uint4*>(tile_row + ((k ^ row_in_atom) << 4)) =
-            make_uint4(prmt(V, Z, o0), prmt(V, Z, o0 >> 16), prmt(V, Z, o1), prmt(V, Z, o1 >> 16));
+        put(k, make_uint4(prmt(V, Z, o0), prmt(V, Z, o0 >> 16), prmt(V, Z, o1), prmt(V, Z, o1 >> 16)));
     }
+}
+template <int LUT_STRIDE = 1>
+__device__ __forceinline__ void decode_stage64(const uint32_t* lut4, const uint32_t (&bytes)[14], int r0,
+                                               bool check_pad, uint32_t lastb, uint32_t pad_base,
+                                               uint32_t pad_span, uint32_t scale_bits, uint8_t* tile_row,
+                                               int row_in_atom) {
+    decode_stage64_to<LUT_STRIDE>(lut4, bytes, r0, check_pad, lastb, pad_base, pad_span, scale_bits,
+                                  [&](int k, uint4 v) { *reinterpret_cast<uint4*>(tile_row + ((k ^ row_in_atom) << 4)) = v; });
 }
 
 // Decoder of one row's 64 weights for a stage in the 2-bit format (code c =
@@ -242,8 +273,8 @@ __device__ __forceinline__ void decode_stage64(const uint32_t* lut4, const uint3
 // NaN} and interleaved by PRMT into the selector pairs of adjacent columns,
 // one PRMT per column pair picks the bf16 values.  Code 3 and a rejected
 // scale give NaN.  Writes the 128-byte swizzled K-major tile row.
-__device__ __forceinline__ void decode_stage64_2bit(const uint32_t (&w)[4], uint32_t scale_bits, uint8_t* tile_row,
-                                                    int row_in_atom) {
+template <class Put>
+__device__ __forceinline__ void decode_stage64_2bit_to(const uint32_t (&w)[4], uint32_t scale_bits, Put&& put) {
     uint32_t V, Z;
     if (scale_is_bad(scale_bits)) {
         V = Z = 0x7FC07FC0u;
@@ -261,11 +292,15 @@ __device__ __forceinline__ void decode_stage64_2bit(const uint32_t (&w)[4], uint
         const uint32_t p23a = prmt(s[2], s[3], 0x5140u);  // (2,3), (6,7)
         const uint32_t p01b = prmt(s[0], s[1], 0x7362u);  // (8,9), (12,13)
         const uint32_t p23b = prmt(s[2], s[3], 0x7362u);  // (10,11), (14,15)
-        *reinterpret_cast<uint4*>(tile_row + (((2 * q) ^ row_in_atom) << 4)) =
-            make_uint4(prmt(V, Z, p01a), prmt(V, Z, p23a), prmt(V, Z, p01a >> 16), prmt(V, Z, p23a >> 16));
-        *reinterpret_cast<uint4*>(tile_row + (((2 * q + 1) ^ row_in_atom) << 4)) =
-            make_uint4(prmt(V, Z, p01b), prmt(V, Z, p23b), prmt(V, Z, p01b >> 16), prmt(V, Z, p23b >> 16));
+        put(2 * q, make_uint4(prmt(V, Z, p01a), prmt(V, Z, p23a), prmt(V, Z, p01a >> 16), prmt(V, Z, p23a >> 16)));
+        put(2 * q + 1,
+            make_uint4(prmt(V, Z, p01b), prmt(V, Z, p23b), prmt(V, Z, p01b >> 16), prmt(V, Z, p23b >> 16)));
     }
+}
+__device__ __forceinline__ void decode_stage64_2bit(const uint32_t (&w)[4], uint32_t scale_bits, uint8_t* tile_row,
+                                                    int row_in_atom) {
+    decode_stage64_2bit_to(w, scale_bits,
+                           [&](int k, uint4 v) { *reinterpret_cast<uint4*>(tile_row + ((k ^ row_in_atom) << 4)) = v; });
 }
 
 // Canonical range of a group's last code byte: digits REAL..4 equal to 1,
