@@ -122,12 +122,13 @@ TQ_API tq_status tq_unpack_bf16(const uint8_t *codes, const void *scales_f16, in
  * "Computation Flow"; the scale is applied once per group as in its "SIMD
  * Matvec" stage): Y[m][n] = sum_g RNE_bf16(s[n][g]) * sum_{j in g} t[n][j] X[m][j],
  * accumulated in fp32, written as fp32 or RNE bf16.  Any M >= 1: CUDA-core
- * kernels up to 8 tokens (weights decoded on chip ahead of the activations
- * when a matrix's rows fit; otherwise lookup tables: one streaming launch
- * per token for 1 token, and for 2..4 tokens on matrices of at least 48 M
- * weights, with G in {64, 128} and K a multiple of 512 up to 4096),
- * tensor-core small-M kernels up to 64 tokens, a row kernel beyond and for
- * the shapes those do not cover.  X: [M][K] bf16, 16-byte aligned; Y: [M][N]
+ * kernels up to 4 tokens, and up to 8 where the tensor path does not take
+ * the shape (weights decoded on chip ahead of the activations when a
+ * matrix's rows fit; otherwise lookup tables: one streaming launch per token
+ * for 1 token, and for 2..4 tokens on matrices of at least 48 M weights,
+ * with G in {64, 128} and K a multiple of 512 up to 4096), tensor-core
+ * small-M kernels up to 64 tokens (K % 64 == 0, G % 64 == 0), a row kernel
+ * beyond and for the shapes those do not cover.  X: [M][K] bf16, 16-byte aligned; Y: [M][N]
  * (fp32: 4-byte aligned, bf16: 2-byte aligned), must not overlap the inputs.
  * K == 0 is allowed: every output is an empty sum and Y is set to +0.
  * workspace: at least tq_workspace_bytes(M, N, K, G) bytes of device scratch

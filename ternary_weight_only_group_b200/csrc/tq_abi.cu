@@ -245,13 +245,18 @@ tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* sc
     if (K == 0) return zero_output(a, (cudaStream_t)stream);  // empty sums
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
-    // 1..8 tokens, matrix small enough for one or two CTAs per SM to hold its
-    // decoded rows: weights decoded before the activations are awaited
-    cudaError_t e = launch_gemv_predecode(static_cast<const uint16_t*>(X), M, codes,
-                                          static_cast<const uint16_t*>(scales), N, K, G, Y, yt == TQ_OUT_BF16,
-                                          d_err, (cudaStream_t)stream, d->sm_count);
-    if (e != cudaErrorNotSupported) return from_cuda(e);
-    cudaGetLastError();
+    // 1..4 tokens (1..8 where the tensor path below does not take the
+    // shape), matrix small enough for one or two CTAs per SM to hold its
+    // decoded rows: weights decoded before the activations are awaited.  At
+    // 5..8 tokens the tensor path is faster (M-sweep, 28 layers of 1536-4096
+    // wide projections at 8 tokens: 5.7 us per launch against 6.9)
+    cudaError_t e = cudaErrorNotSupported;
+    if (M <= 4 || G % 64 != 0 || K % 64 != 0) {
+        e = launch_gemv_predecode(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
+                                  N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count);
+        if (e != cudaErrorNotSupported) return from_cuda(e);
+        cudaGetLastError();
+    }
     // 1..4 tokens over a larger matrix: lookup tables of one 512-column K
     // slice per CTA, slices spread over a cluster, code words streamed per
     // lane; one launch per token (172032 x 1024: 14.3 us per token, against

@@ -118,7 +118,8 @@ def test_predecode_row_batches(N, K, G, M):
     """One to eight tokens over matrices whose per-CTA rows fit in shared
     memory: more than eight row batches per CTA (8 rows, 4 rows from 5
     tokens), chunks split over two to eight warps, ragged last CTA, one or
-    two CTAs per SM, tokens padded with zeros up to the kernel's 4 or 8."""
+    two CTAs per SM, tokens padded with zeros up to the kernel's 4 or 8
+    (5..8 tokens with G a multiple of 64 take the tensor path instead)."""
     W = synthetic.weights(N, K, index=N + K)
     X = synthetic.activations(M, K)
     check(X, W, G)
