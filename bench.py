@@ -43,8 +43,8 @@ METRIC = "ternary x bf16 GEMV HBM GB/s (% of peak); prefill GEMM TFLOP/s; pack G
 # gemv_predecode.cu at capture time is recorded beside them, and the figures
 # are reported only while the current source still has that hash.
 PREDECODE_DRAM_BYTES = {(3584, 1024, 64): 902912, (1024, 3584, 64): 907008,
-                        (3584, 1024, 128): 845312, (1024, 3584, 128): 850432}
-PREDECODE_DRAM_SRC_SHA256 = "6c8b9831ac920cf1f2316b43239e500c5e96782d966acc923919c9cda723f255"
+                        (3584, 1024, 128): 845312, (1024, 3584, 128): 850176}
+PREDECODE_DRAM_SRC_SHA256 = "23cc404f71359f660e2b572e039476d724c2f30550d7fb53e89881631436f091"
 FFN = {"gate": (3584, 1024), "up": (3584, 1024), "down": (1024, 3584)}
 MSWEEP = {"q": (1536, 1536), "o": (1536, 1536), "gate": (4096, 1536), "up": (4096, 1536), "down": (1536, 4096)}
 MSWEEP_LAYERS = 28

@@ -183,7 +183,10 @@ TQ_API tq_status tq2_unpack_bf16(const uint8_t *codes, const void *scales_f16, i
  * not write them).  1 token on matrices of at least 24 M weights (8 M at
  * K >= 2048), and 2..4 tokens from 48 M weights, with G in {64, 128}, K a
  * multiple of 512 up to 4096 and 8-byte-aligned codes, take the streaming
- * lookup-table kernel, one launch per token; 3..64 tokens with K % 64 == 0
+ * lookup-table kernel, one launch per token; 1..4 tokens (1..8 at G < 64)
+ * with K % 512 == 0, G % 16 == 0, 4-byte-aligned codes and rows that fit
+ * in shared memory the pre-decode kernel (weights decoded before the
+ * activations are awaited); 3..64 tokens with K % 64 == 0
  * and G % 64 == 0 the tensor-core small-M kernels (2-bit codes decoded on
  * chip); otherwise the CUDA-core kernel, eight tokens per launch, which
  * covers G in {16, 32, 64, 128, 256} and K <= 49152; other shapes return

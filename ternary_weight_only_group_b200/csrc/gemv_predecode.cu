@@ -31,6 +31,7 @@
 // per-CTA rows fit in about 100 KB of bf16; the lookup-table GEMV takes the
 // rest.
 #include <atomic>
+#include <type_traits>
 
 #include "tq_internal.cuh"
 
@@ -145,11 +146,42 @@ __device__ __forceinline__ float fma_bf16(uint16_t a, uint16_t b, float c) {
 // chunks; both are free of bank conflicts this way.
 __device__ __forceinline__ int pd_swizzle(int c) { return c ^ ((c >> 3) & 7); }
 
-template <int G, int MT>
+// Code bytes per group: base-3 (FMT 3) ceil(G/5) + 2 ... as the codec
+// defines; 2-bit (FMT 2, G a multiple of 16) G/4.
+template <int G, int FMT>
+__host__ __device__ constexpr int pd_group_bytes() { return FMT == 3 ? bytes_per_group(G) : G / 4; }
+
+// The 2-bit format's decode of one lane's 16 * NWD weights: word q of the
+// lane's codes holds columns 16 q .. 16 q + 15 (code c = t + 1 of column j
+// in bits 2 (j mod 4) of byte j / 4); (w >> 2k) & 0x03030303 holds the codes
+// of columns k, k+4, k+8, k+12, mapped to the selector bytes 0x10 + 0x22 c
+// of {V, Z} and interleaved by PRMT into the selector pairs of adjacent
+// columns (code 3 selects NaN).  `put(k, v)` gets chunk k (columns 8k ..
+// 8k+7) as four bf16 pairs.
+template <int NWD, class Put>
+__device__ __forceinline__ void pd_decode_2bit(const uint32_t (&wd)[NWD], uint32_t V, uint32_t Z, Put&& put) {
+#pragma unroll
+    for (int q = 0; q < NWD; ++q) {
+        uint32_t sel[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sel[k] = 0x10101010u + 0x22u * ((wd[q] >> (2 * k)) & 0x03030303u);
+        const uint32_t p01a = prmt32(sel[0], sel[1], 0x5140u);  // columns (0,1) low half, (4,5) high half
+        const uint32_t p23a = prmt32(sel[2], sel[3], 0x5140u);  // (2,3), (6,7)
+        const uint32_t p01b = prmt32(sel[0], sel[1], 0x7362u);  // (8,9), (12,13)
+        const uint32_t p23b = prmt32(sel[2], sel[3], 0x7362u);  // (10,11), (14,15)
+        put(2 * q, make_uint4(prmt32(V, Z, p01a), prmt32(V, Z, p23a), prmt32(V, Z, p01a >> 16),
+                              prmt32(V, Z, p23a >> 16)));
+        put(2 * q + 1, make_uint4(prmt32(V, Z, p01b), prmt32(V, Z, p23b), prmt32(V, Z, p01b >> 16),
+                                  prmt32(V, Z, p23b >> 16)));
+    }
+}
+
+template <int G, int MT, int FMT>
 __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_kernel(
     const uint16_t* __restrict__ X, int M, const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
     int64_t N, int K, int R, void* __restrict__ Y, int y_bf16, uint32_t* __restrict__ d_err) {
-    constexpr int B = bytes_per_group(G);
+    static_assert(FMT == 3 || G % 16 == 0, "2-bit lanes decode whole 32-bit code words");
+    constexpr int B = pd_group_bytes<G, FMT>();
     constexpr int REAL = G - 5 * (B - 1);   // real digits in a group's last byte
     constexpr int SW = G < 64 ? G : 64;     // weights a decode lane writes
     constexpr int LPG = G / SW;             // lanes per group
@@ -176,8 +208,9 @@ __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_ke
     // are contiguous) in one round of copies
     const int ngroups = nrows * ng;
     unsigned char* raw = smem + pd_head_bytes(K, MT) + (size_t)R * K * 2;
-    for (int i = threadIdx.x; i < kPdTableBytes / 16; i += kPdThreads)
-        cp_async16(smem + 16 * i, reinterpret_cast<const unsigned char*>(&kPdSelectors) + 16 * i);
+    if (FMT == 3)
+        for (int i = threadIdx.x; i < kPdTableBytes / 16; i += kPdThreads)
+            cp_async16(smem + 16 * i, reinterpret_cast<const unsigned char*>(&kPdSelectors) + 16 * i);
     const unsigned char* craw = stage_bytes(raw, codes + row0 * ng * B, ngroups * B, threadIdx.x, kPdThreads);
     const uint16_t* sraw = reinterpret_cast<const uint16_t*>(
         stage_bytes(raw + pd_codes_area(R * ng * B), reinterpret_cast<const unsigned char*>(scales + row0 * ng),
@@ -187,6 +220,30 @@ __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_ke
     __syncthreads();
 
     // ---- decode (weights only: no dependence on earlier kernels)
+    if constexpr (FMT == 2) {
+        constexpr int NWD = SW / 16;  // code words of a lane
+        for (int u = threadIdx.x; u < ngroups * LPG; u += kPdThreads) {
+            const int gl = u / LPG, sub = u - gl * LPG;
+            const uint32_t s = sraw[gl];
+            // the staged copy keeps the source's offset within 16 bytes, and
+            // codes, rows and groups are 4-byte aligned: whole words
+            const uint32_t* in = reinterpret_cast<const uint32_t*>(craw + (size_t)gl * B + (size_t)sub * (SW / 4));
+            uint32_t wd[NWD];
+#pragma unroll
+            for (int i = 0; i < NWD; ++i) wd[i] = in[i];
+            uint32_t V, Z;  // {-s, 0} and {+s, NaN}
+            if (scale_is_bad(s)) {
+                V = Z = 0x7FC07FC0u;
+            } else {
+                const uint32_t mag = (s == 0) ? 0u : scale_to_bf16_bits((uint16_t)s);
+                V = mag ? (mag | 0x8000u) : 0u;
+                Z = mag | 0x7FC00000u;
+            }
+            const int cg0 = u * NCH;
+            pd_decode_2bit<NWD>(wd, V, Z,
+                                [&](int k, uint4 v) { *reinterpret_cast<uint4*>(w + 8 * pd_swizzle(cg0 + k)) = v; });
+        }
+    } else
     for (int u = threadIdx.x; u < ngroups * LPG; u += kPdThreads) {
         const int gl = u / LPG, sub = u - gl * LPG;  // group inside the CTA, lane's part of it
         const int p0 = SW * sub;                     // first weight of the part
@@ -309,7 +366,8 @@ __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_ke
             if (ks == 1) {
                 if (rr < nrows) {
                     if (tot[0] != tot[0])
-                        err_acc |= scan_row_errors(codes + (row0 + rr) * ng * B, scales + (row0 + rr) * ng, ng, G, B);
+                        err_acc |= FMT == 3 ? scan_row_errors(codes + (row0 + rr) * ng * B, scales + (row0 + rr) * ng, ng, G, B)
+                                            : scan_row_errors2(codes + (row0 + rr) * ng * B, scales + (row0 + rr) * ng, ng, G);
 #pragma unroll
                     for (int m = 0; m < MT; ++m)
                         if (m < M) store_y(Y, y_bf16, (int64_t)m * N + row0 + rr, tot[m]);
@@ -331,7 +389,8 @@ __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_ke
 #pragma unroll
                 for (int m = 0; m < MT; ++m) tot[m] += red[(sl * (RB * nb) + rr) * MT + m];
             if (tot[0] != tot[0])
-                err_acc |= scan_row_errors(codes + (row0 + rr) * ng * B, scales + (row0 + rr) * ng, ng, G, B);
+                err_acc |= FMT == 3 ? scan_row_errors(codes + (row0 + rr) * ng * B, scales + (row0 + rr) * ng, ng, G, B)
+                                    : scan_row_errors2(codes + (row0 + rr) * ng * B, scales + (row0 + rr) * ng, ng, G);
 #pragma unroll
             for (int m = 0; m < MT; ++m)
                 if (m < M) store_y(Y, y_bf16, (int64_t)m * N + row0 + rr, tot[m]);
@@ -340,11 +399,11 @@ __global__ void __launch_bounds__(kPdThreads, MT == 1 ? 3 : 2) gemv_predecode_ke
     if (err_acc && d_err) atomicOr(d_err, err_acc);
 }
 
-template <int G, int MT>
+template <int G, int MT, int FMT>
 static cudaError_t launch_pd(const uint16_t* X, int M, const uint8_t* codes, const uint16_t* scales, int64_t N,
                              int K, int R, int grid, size_t smem, void* Y, int y_bf16, uint32_t* d_err,
                              cudaStream_t stream) {
-    auto kern = gemv_predecode_kernel<G, MT>;
+    auto kern = gemv_predecode_kernel<G, MT, FMT>;
     static SmemAttr smem_attr;
     if (cudaError_t e = smem_attr.ensure(kern, (int)smem)) return e;
     cudaLaunchConfig_t cfg = {};
@@ -360,28 +419,31 @@ static cudaError_t launch_pd(const uint16_t* X, int M, const uint8_t* codes, con
     return cudaLaunchKernelEx(&cfg, kern, X, M, codes, scales, N, K, R, Y, y_bf16, d_err);
 }
 
-template <int MT>
+template <int MT, int FMT>
 static cudaError_t launch_pd_g(int G, const uint16_t* X, int M, const uint8_t* codes, const uint16_t* scales,
                                int64_t N, int K, int R, int grid, size_t smem, void* Y, int y_bf16, uint32_t* d_err,
                                cudaStream_t stream) {
     switch (G) {
-        case 8: return launch_pd<8, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
-        case 16: return launch_pd<16, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
-        case 32: return launch_pd<32, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
-        case 64: return launch_pd<64, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
-        case 128: return launch_pd<128, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
-        default: return launch_pd<256, MT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+        case 8:
+            if constexpr (FMT == 3) return launch_pd<8, MT, 3>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+            else return cudaErrorNotSupported;
+        case 16: return launch_pd<16, MT, FMT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+        case 32: return launch_pd<32, MT, FMT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+        case 64: return launch_pd<64, MT, FMT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+        case 128: return launch_pd<128, MT, FMT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
+        default: return launch_pd<256, MT, FMT>(X, M, codes, scales, N, K, R, grid, smem, Y, y_bf16, d_err, stream);
     }
 }
 
 // Returns cudaErrorNotSupported when the shape is not covered.
 cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                   int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                                  cudaStream_t stream, int sm_count) {
+                                  cudaStream_t stream, int sm_count, int fmt) {
     if (M < 1 || M > 8 || K % 512 != 0 || N < 1 || K > 65536) return cudaErrorNotSupported;
     if (G != 8 && G != 16 && G != 32 && G != 64 && G != 128 && G != 256) return cudaErrorNotSupported;
+    if (fmt != 3 && (fmt != 2 || G % 16 != 0 || (reinterpret_cast<uintptr_t>(codes) & 3))) return cudaErrorNotSupported;
     const int MT = M == 1 ? 1 : (M == 2 ? 2 : (M <= 4 ? 4 : 8));
-    const int64_t ng = K / G, B = bytes_per_group(G);
+    const int64_t ng = K / G, B = fmt == 3 ? bytes_per_group(G) : G / 4;
     // one CTA per SM if it fits (later launches then decode beside it), else two
     for (int per_sm = 1; per_sm <= 2; ++per_sm) {
         const int64_t R = (N + (int64_t)sm_count * per_sm - 1) / ((int64_t)sm_count * per_sm);
@@ -390,10 +452,14 @@ cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* c
                             (size_t)pd_codes_area((int)(R * ng * B)) + (size_t)pd_codes_area((int)(R * ng * 2));
         if (smem > kPdMaxSmem) continue;
         const int grid = (int)((N + R - 1) / R);
-        if (MT == 1) return launch_pd_g<1>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
-        if (MT == 2) return launch_pd_g<2>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
-        if (MT == 4) return launch_pd_g<4>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
-        return launch_pd_g<8>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
+        auto go = [&](auto fmt_tag) {
+            constexpr int F = decltype(fmt_tag)::value;
+            if (MT == 1) return launch_pd_g<1, F>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
+            if (MT == 2) return launch_pd_g<2, F>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
+            if (MT == 4) return launch_pd_g<4, F>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
+            return launch_pd_g<8, F>(G, X, (int)M, codes, scales, N, (int)K, (int)R, grid, smem, Y, y_bf16, d_err, stream);
+        };
+        return fmt == 3 ? go(std::integral_constant<int, 3>{}) : go(std::integral_constant<int, 2>{});
     }
     return cudaErrorNotSupported;
 }

@@ -32,7 +32,7 @@ cudaError_t launch_gemv_lut_stream_w4(const uint16_t* X, int64_t M, const uint32
                                       cudaStream_t stream, int sm_count);
 cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                   int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                                  cudaStream_t stream, int sm_count);
+                                  cudaStream_t stream, int sm_count, int fmt);
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                               int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                               cudaStream_t stream, int sm_count, bool* handled, int fmt);
@@ -253,7 +253,7 @@ tq_status tq_gemv(const void* X, int64_t M, const uint8_t* codes, const void* sc
     cudaError_t e = cudaErrorNotSupported;
     if (M <= 4 || G % 64 != 0 || K % 64 != 0) {
         e = launch_gemv_predecode(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
-                                  N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count);
+                                  N, K, G, Y, yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, 3);
         if (e != cudaErrorNotSupported) return from_cuda(e);
         cudaGetLastError();
     }
@@ -385,6 +385,18 @@ tq_status tq2_gemv(const void* X, int64_t M, const uint8_t* codes, const void* s
     if (M <= kStreamMaxTokens && big) {
         const cudaError_t e = stream_per_token(X, M, codes, scales, N, K, G, Y, yt, d_err, (cudaStream_t)stream,
                                                d->sm_count, 2);
+        if (e != cudaErrorNotSupported) return from_cuda(e);
+        cudaGetLastError();
+    }
+    // 1..4 tokens (1..8 where the tensor path does not take the shape), matrix
+    // small enough for one or two CTAs per SM to hold its decoded rows: the
+    // pre-decode kernel, weights decoded before the activations are awaited
+    // (the headline's FFN projections: 4.8 us per launch on the CUDA-core
+    // kernel below in a chain of dependent launches)
+    if (M <= 4 || G % 64 != 0 || K % 64 != 0) {
+        const cudaError_t e = launch_gemv_predecode(static_cast<const uint16_t*>(X), M, codes,
+                                                    static_cast<const uint16_t*>(scales), N, K, G, Y,
+                                                    yt == TQ_OUT_BF16, d_err, (cudaStream_t)stream, d->sm_count, 2);
         if (e != cudaErrorNotSupported) return from_cuda(e);
         cudaGetLastError();
     }

@@ -106,10 +106,13 @@ def run_gemv2(X, codes, scales, N, K, G, out_dtype):
 
 @pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 11])
 @pytest.mark.parametrize("N,K,G", [(3584, 1024, 64), (1024, 3584, 128), (1037, 1152, 128), (301, 1040, 16),
-                                   (130, 4096, 256), (77, 2048, 32)])
+                                   (130, 4096, 256), (77, 2048, 32), (300, 1024, 16)])
 def test_gemv2(N, K, G, M):
     """Token counts 1..11 (two launches past 8), ragged row batches and code
-    words per row that are not multiples of 32 lanes; fp32 and bf16 outputs."""
+    words per row that are not multiples of 32 lanes; fp32 and bf16 outputs.
+    K a multiple of 512 takes the pre-decode kernel up to 4 tokens (8 at
+    G < 64: one, two and four code words per decode lane), other K the
+    CUDA-core kernel, 5+ tokens at G % 64 == 0 the tensor path."""
     W = synthetic.weights(N, K, index=N + G)
     codes, scales, _ = oracle.quantize_pack2(W, G)
     X = synthetic.activations(M, K)
