@@ -7,9 +7,11 @@
 // 128-row tiles as half the SMs, where splitting K over a cluster buys
 // nothing.  One CTA per SM walks its tiles; each tile is
 //   D^T[128 W rows x NT tokens] += What[128 x 16] . X[NT x 16]^T
-// over K in 64-column stages, with What decoded on chip into the
-// 128-byte-swizzled K-major layout and X stages loaded by TMA (NT = 16, 32
-// or 64 rows, zero-filled past M).
+// over K in 64-column stages, with What decoded on chip straight into tensor
+// memory (a decoder thread owns one W row = one tensor-memory lane and
+// stores a stage's 64 bf16 with tcgen05.st), where the MMA reads it as the A
+// operand, and X stages loaded by TMA (NT = 16, 32 or 64 rows, zero-filled
+// past M).
 //   warp 0       TMA producer of the X stages
 //   warp 1       MMA issuer (kind::f16, M=128, N=NT, fp32 accumulators in TMEM)
 //   warp 2       tensor-memory allocation
@@ -38,13 +40,18 @@ constexpr int CR = 4;      // code windows in flight per decoder thread
 constexpr int kThreads = 512;
 constexpr int kDecWarp0 = 4, kEpiWarp0 = 12;
 constexpr int kGroupWarps = 4;
-constexpr uint32_t W_STAGE = WM * BK * 2;  // 16 KB
 constexpr uint32_t WIN = 48;               // per row: 32 code bytes, the 4-byte word holding the scale, pad
+
+// Tensor memory: two accumulators of NT columns, then one 32-column slot of
+// decoded W (128 x 64 bf16) per stage.
+template <int NT>
+constexpr uint32_t kAccCols = 2 * NT;
+template <int NT>
+constexpr uint32_t kTmemCols = kAccCols<NT> + 32 * STAGES <= 256 ? 256 : 512;
 
 template <int NT>
 struct Smem {
-    uint8_t w[STAGES][W_STAGE];     // decoded W stages (UMMA A), 1024-byte aligned
-    uint8_t x[STAGES][NT * 128];    // X stages (UMMA B): NT rows of 128 bytes
+    uint8_t x[STAGES][NT * 128];    // X stages (UMMA B): NT rows of 128 bytes, 1024-byte aligned
     uint8_t win[2][CR][WM * WIN];   // code windows + scales, per decoder group
     uint32_t lut[256 * 32];           // byte -> PRMT selectors of its digits 0..3, one copy per lane
     uint64_t full_x[STAGES], full_w[STAGES], empty[STAGES];
@@ -117,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     const int nk = p.K / BK;
     const int my_tiles = (p.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const int total = my_tiles * nk;  // stages of this CTA
-    constexpr uint32_t kCols = 2 * NT < 32 ? 32 : 2 * NT;
+    constexpr uint32_t kCols = kTmemCols<NT>, ACC = kAccCols<NT>;
     volatile int* abort_flag = &sm.abort_flag;
     const uint64_t lim = p.wc.limit_ns;
 
@@ -191,11 +198,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = s32(sm.w[st]), b0 = s32(sm.x[st]);
+                    const uint32_t a0 = tmem + ACC + 32u * (uint32_t)st, b0 = s32(sm.x[st]);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k)
-                        mma_bf16(d, smem_desc_sw128(a0 + 32 * k), smem_desc_sw128(b0 + 32 * k), idesc,
-                                 (kb > 0 || k > 0) ? 1u : 0u);
+                        mma_bf16_ts(d, a0 + 8u * k, smem_desc_sw128(b0 + 32 * k), idesc, (kb > 0 || k > 0) ? 1u : 0u);
                     mma_commit(&sm.empty[st]);
                 }
                 if (ok) mma_commit(&sm.tfull[buf]);
@@ -204,7 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
         }
     } else if (warp >= kDecWarp0 && warp < kEpiWarp0) {
         const int grp = (warp - kDecWarp0) >> 2;              // stages grp, grp + 2, ...
-        const int t = ((warp - kDecWarp0) & 3) * 32 + lane;  // W row of the tile
+        const int t = ((warp - kDecWarp0) & 3) * 32 + lane;  // W row of the tile = tensor-memory lane
+        const uint32_t trow = tmem + ((uint32_t)(t & ~31) << 16) + ACC;
         const int SPG = p.G / BK;                             // stages per group
         // stage position (tile iteration j, group g, part sub of the group),
         // advanced by two stages at a time without divisions
@@ -256,19 +263,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
             const uint8_t* slot = sm.win[grp][s % CR] + t * WIN;
             const uint8_t* cb = slot + (A & 15);
             const uint32_t sc = *reinterpret_cast<const uint16_t*>(slot + 32 + (S & 2));
+            uint32_t wv[32];
+            auto put = [&](int k, uint4 v) {
+                wv[4 * k] = v.x;
+                wv[4 * k + 1] = v.y;
+                wv[4 * k + 2] = v.z;
+                wv[4 * k + 3] = v.w;
+            };
             if constexpr (FMT == 2) {  // codes 4-byte aligned: cb is a word boundary of the window
                 const uint32_t* cw = reinterpret_cast<const uint32_t*>(cb);
                 const uint32_t wd[4] = {cw[0], cw[1], cw[2], cw[3]};
-                decode_stage64_2bit(wd, sc, sm.w[st] + t * 128, t & 7);
+                decode_stage64_2bit_to(wd, sc, put);
             } else {
-            uint32_t bytes[14];
+                uint32_t bytes[14];
 #pragma unroll
-            for (int b = 0; b < 14; ++b) bytes[b] = cb[b];
-            const int ql = p.B - 1 - q_lo;  // the group's last byte, relative to cb
-            decode_stage64<32>(sm.lut + (t & 31), bytes, c0 - 5 * q_lo, ql < 14, ql < 14 ? cb[ql] : 0u, p.pad_base, p.pad_span,
-                           sc, sm.w[st] + t * 128, t & 7);
+                for (int b = 0; b < 14; ++b) bytes[b] = cb[b];
+                const int ql = p.B - 1 - q_lo;  // the group's last byte, relative to cb
+                decode_stage64_to<32>(sm.lut + (t & 31), bytes, c0 - 5 * q_lo, ql < 14, ql < 14 ? cb[ql] : 0u,
+                                      p.pad_base, p.pad_span, sc, put);
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tmem_st32(trow + 32u * (uint32_t)st, wv);
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_w[st]);
             advance(pd);
