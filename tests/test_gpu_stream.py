@@ -1,8 +1,9 @@
 """GPU parity of the persistent small-M tensor-core path against the oracle.
 
 Matrices with more 128-row tiles than half the SMs take it, from tq_gemm
-for any M <= 64 and from tq_gemv for M >= 3 when the pre-decode kernel does
-not fit.  Sampled token rows (first,
+for any M <= 64 and from tq_gemv for M >= 5 (3..4 when the pre-decode kernel
+does not fit).  The decoded weights go to tensor memory as the MMA's A
+operand.  Sampled token rows (first,
 middle, last) are compared over every output column.  Tolerances as for the
 other matmul paths: fp32 max_n |gpu - oracle| <= 1e-3 * max_n |oracle| per
 row; bf16 |gpu - oracle| <= 2e-2 + 2e-2 |oracle|; NaN rows must coincide.
@@ -93,3 +94,30 @@ def test_stream_rejected_groups():
     assert_rows_close_f32(Y[rows], ref)
     assert np.all(np.isnan(Y[:, [5, 4000, 9599, 130]])) and np.all(np.isfinite(Y[:, 7777]))
     assert e == e_ref
+
+
+@pytest.mark.parametrize("M", [8, 16])
+def test_stream_path_ffn_stack_full_size(M):
+    """The 48 gate/up projections of the 24-layer stack as one [172032 x 1024]
+    matrix, G=128, through tq_gemv (each CTA walks about nine 128-row tiles):
+    four oracle-packed 3584-row projections repeated 12 times; sampled token
+    rows compared over every output column."""
+    K, G = 1024, 128
+    codes, scales = [], []
+    for l in range(4):
+        c, s_, _ = oracle.quantize_pack(synthetic.ffn_matrix("up", layer=l), G)
+        codes.append(c)
+        scales.append(s_)
+    codes, scales = np.concatenate(codes), np.concatenate(scales)
+    Nb = codes.shape[0]
+    N = 12 * Nb
+    X = synthetic.activations(M, K, offset=703)
+    rows = sample_rows(M)
+    ref = np.tile(oracle.linear(X, codes, scales, Nb, K, G, rows=rows), (1, 12))
+    dc = to_dev_u8(codes).repeat(12, 1, 1)
+    ds = to_dev_f16(scales).repeat(12, 1)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Y = tq.gemv(to_dev_bf16(X), dc, ds, N, K, G, out_dtype=torch.float32, d_err=err)
+    torch.cuda.synchronize()
+    assert_rows_close_f32(to_f64(Y)[rows], ref)
+    assert int(err.item()) == 0

@@ -94,6 +94,23 @@ def test_w4_gemv_stream_tokens_large():
     check(98317, 1024, 128, 2, index=17, dtypes=(torch.bfloat16,))
 
 
+@pytest.mark.parametrize("M", [1, 2])
+def test_w4_gemv_stream_full_size_sampled(M):
+    """The benchmark's workload: the 24-layer gate/up-shaped stack as one
+    [172032 x 1024] W4A16 matrix, G=128 (4-CTA clusters), one and two tokens
+    (one streaming launch per token); 512 sampled output columns against the
+    oracle on the same rows."""
+    N, K, G = 48 * 3584, 1024, 128
+    codes, scales, biases = synthetic.w4_params(N, K, G, index=41)
+    X = synthetic.activations(M, K, offset=805)
+    dc, ds, db = dev_params(codes, scales, biases)
+    Y = tq.w4_gemv(to_dev_bf16(X), dc, ds, db, N, K, G, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    cols = np.random.default_rng(1).choice(N, size=512, replace=False)
+    ref = oracle.linear_w4(X, codes[cols], scales[cols], biases[cols], len(cols), K, G)
+    assert_rows_close_f32(to_f64(Y)[:, cols], ref)
+
+
 def test_w4_gemv_stream_every_byte():
     """Every code byte (two nibbles) in every byte position of the tables:
     row n, word w, byte i holds (n + 8 w + i) mod 256."""
