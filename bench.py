@@ -345,6 +345,7 @@ def run_ours(args, rank, world, local):
         results["pack"], results["unpack"] = bench_bulk_codec(tq, args, world, peaks)
         results["prefill"] = bench_prefill(tq, args, world, peaks)
         results["msweep"] = bench_msweep(tq, args, world, peaks)
+        results["small_m_stack"] = bench_small_m_stack(tq, args, world, peaks)
         results["ternary2"] = bench_ternary2(tq, args, world, peaks)
         results["w4"] = bench_w4(tq, args, world, peaks)
     clk = clocks.summary()
@@ -402,6 +403,7 @@ def run_ours(args, rank, world, local):
         "unpack": results["unpack"],
         "prefill_gemm": results["prefill"],
         "msweep": results["msweep"],
+        "small_m_stack": results["small_m_stack"],
         "ternary2": results["ternary2"],
         "w4": results["w4"],
     }
@@ -577,6 +579,38 @@ def bench_gemv_shapes(tq, args, world, peaks):
             res[f"{name}{N}x{K}_G{G}"] = {"us": round(us, 2), "GB/s": round(byts / us / 1e3, 1),
                                            "launches": max(3, args.steps) * len(packs)}
             del packs
+    return res
+
+
+def bench_small_m_stack(tq, args, world, peaks):
+    """5..64 tokens over the 24-layer gate/up stack as one [172032 x 1024]
+    matrix, G=128 (the persistent small-M tensor kernel: more 128-row tiles
+    than SMs): four packed copies (38.9 MB of codes and scales each, 156 MB
+    in all, more than L2) used in turn from one CUDA graph.  GB/s on the
+    algorithmic bytes (codes, scales, X, Y)."""
+    import torch
+    N, K, G = 48 * 3584, 1024, 128
+    packs = []
+    for c in range(4):
+        W = device_weights(N, K, seed=77 + c)
+        packs.append(tq.quantize_pack(W, G))
+        del W
+    torch.cuda.empty_cache()
+    res = {}
+    for M in (5, 16, 64):
+        X = device_acts(M, K, seed=78)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        launches = [lambda c=c, s=s: tq.gemv(X, c, s, N, K, G, out=Y) for c, s in packs]
+        us = graph_launch_us(launches, 4, args, world)
+        byts = packed_bytes(N, K, G) + 2 * M * K + 2 * M * N
+        res[f"M{M}"] = {"us": round(us, 2), "GB/s": round(byts / us / 1e3, 1),
+                        "frac": round(byts / us / 1e3 / peaks["hbm_gbs"], 4),
+                        "TFLOP/s": round(2.0 * M * N * K / us / 1e6, 2), "launches": max(3, args.steps) * 16}
+        del launches, X, Y
+    res["kernel"] = "gemm_stream_kernel<NT, 3> (persistent, decoded W in tensor memory)"
+    res["note"] = "4 copies of 38.9 MB used in turn from one CUDA graph (156 MB > L2)"
+    del packs
+    torch.cuda.empty_cache()
     return res
 
 
@@ -1001,7 +1035,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
-    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv", "msweep", "ternary2", "w4", "traffic"],
+    ap.add_argument("--only", choices=["stream", "codec", "prefill", "gemv", "msweep", "smallm", "ternary2", "w4",
+                                       "traffic"],
                     default=None,
                     help="run one sub-benchmark alone and print its result (profiling aid)")
     args = ap.parse_args()
@@ -1018,7 +1053,8 @@ def main():
             torch.cuda.set_device(local)
             peaks = load_peaks()
             fn = {"stream": bench_gemv_stream, "codec": bench_bulk_codec, "prefill": bench_prefill,
-                  "gemv": bench_gemv_shapes, "msweep": bench_msweep, "ternary2": bench_ternary2, "w4": bench_w4,
+                  "gemv": bench_gemv_shapes, "msweep": bench_msweep, "smallm": bench_small_m_stack,
+                  "ternary2": bench_ternary2, "w4": bench_w4,
                   "traffic": decode_shapes_once}
             res = fn[args.only](tq, args, world, peaks)
             if rank == 0:
