@@ -49,6 +49,10 @@ template <int NT>
 constexpr int kAcc = NT < 32 ? 32 : NT;
 template <int NT>
 constexpr int kWSlots = (int)(kCols - kAcc<NT>) / 32;  // 7, 7, 6
+// W4A16 (FMT 4): a stage holds each weight as two bf16 terms, hi and lo, in a
+// pair of 32-column slots (3 pairs)
+template <int NT, int FMT>
+constexpr int kWSlotsF = (int)(kCols - kAcc<NT>) / (FMT == 4 ? 64 : 32);
 template <int NT>
 constexpr int kXStages = NT == 64 ? 4 : 8;
 constexpr int kCStages = 8;
@@ -80,6 +84,7 @@ struct Params {
     const uint8_t* codes;
     int64_t row_bytes;
     const uint16_t* scales;
+    const uint16_t* biases;  // W4A16 only
     void* Y;
     uint32_t* d_err;
     int64_t M, N;
@@ -91,13 +96,17 @@ struct Params {
 };
 
 // FMT 3: base-3 codes (five digits per byte); FMT 2: the 2-bit format (four
-// codes per byte, G a multiple of 64: a stage's 64 codes are 16 whole bytes).
+// codes per byte, G a multiple of 64: a stage's 64 codes are 16 whole bytes);
+// FMT 4: the W4A16 affine codes (two per byte, a stage's 64 codes are 32
+// bytes at a 32-byte boundary of the row), each weight w = q * s + b by one
+// fp32 FMA held as hi = RNE_bf16(w) and lo = RNE_bf16(w - hi), both MMAs
+// into the same accumulator.
 template <int NT, bool CODES_TMA, int FMT>
 __global__ void __launch_bounds__(kThreads, 2) gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_x,
                                                                  const __grid_constant__ CUtensorMap tmap_c,
                                                                  const Params p) {
-    constexpr int XS = kXStages<NT>, CST = kCStages, WSL = kWSlots<NT>;
-    constexpr uint32_t ACC = kAcc<NT>;
+    constexpr int XS = kXStages<NT>, CST = kCStages, WSL = kWSlotsF<NT, FMT>;
+    constexpr uint32_t ACC = kAcc<NT>, SLOT = FMT == 4 ? 64u : 32u;  // columns per stage slot
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem<NT>& sm = *reinterpret_cast<Smem<NT>*>(smem_raw + ((1024 - (s32(smem_raw) & 1023)) & 1023));
     cg::cluster_group cluster = cg::this_cluster();
@@ -150,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_small_kernel(const __grid_co
         const int k0 = kb * BK;
         g = k0 / p.G;
         c0 = k0 - g * p.G;
-        q_lo = FMT == 3 ? c0 / 5 : c0 / 4;
+        q_lo = FMT == 3 ? c0 / 5 : (FMT == 2 ? c0 / 4 : c0 / 2);
     };
 
     if (warp == 0) {
@@ -200,10 +209,13 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_small_kernel(const __grid_co
                 if (!mbar_wait(&sm.full_x[i % XS], (i / XS) & 1, abort_flag, lim)) break;
                 if (!mbar_wait(&sm.full_w[st], (i / WSL) & 1, abort_flag, lim)) break;
                 tc_fence_after();
-                const uint32_t a0 = tmem + ACC + 32u * (uint32_t)st, b0 = s32(sm.x[i % XS]);
+                const uint32_t a0 = tmem + ACC + SLOT * (uint32_t)st, b0 = s32(sm.x[i % XS]);
 #pragma unroll
-                for (int k = 0; k < BK / 16; ++k)
+                for (int k = 0; k < BK / 16; ++k) {
                     mma_bf16_ts(tmem, a0 + 8u * k, smem_desc_sw128(b0 + 32 * k), idesc, (i > 0 || k > 0) ? 1u : 0u);
+                    if (FMT == 4)  // the lo terms, 32 columns on
+                        mma_bf16_ts(tmem, a0 + 32u + 8u * k, smem_desc_sw128(b0 + 32 * k), idesc, 1u);
+                }
                 mma_commit(&sm.wempty[st]);
                 mma_commit(&sm.xempty[i % XS]);
             }
@@ -214,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_small_kernel(const __grid_co
         const uint32_t trow = tmem + ((uint32_t)(32 * (warp - kDecodeWarp0)) << 16) + ACC;
         const int64_t n = n0 + t;
         const uint16_t* srow = p.scales + (n < p.N ? n : 0) * p.ng;
+        const uint16_t* brow = FMT == 4 ? p.biases + (n < p.N ? n : 0) * p.ng : nullptr;
         const uint8_t* crow = p.codes + (n < p.N ? n : 0) * p.row_bytes;
         auto load_global = [&](int kb, uint32_t (&bytes)[14]) {
             int g, c0, q_lo;
@@ -225,12 +238,15 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_small_kernel(const __grid_co
         uint32_t cur[14], nxt[14];
         if (!CODES_TMA && FMT == 3 && nkl > 0) load_global(kb_lo, cur);
         uint32_t sc_nxt = nkl > 0 ? __ldg(srow + (kb_lo * BK) / p.G) : 0u;
+        uint32_t bi_nxt = FMT == 4 && nkl > 0 ? __ldg(brow + (kb_lo * BK) / p.G) : 0u;
         for (int i = 0; i < nkl; ++i) {
             const int kb = kb_lo + i, st = i % WSL, use = i / WSL;
             int g, c0, q_lo;
             stage_geom(kb, g, c0, q_lo);
             const uint32_t sc = sc_nxt;
             if (i + 1 < nkl) sc_nxt = __ldg(srow + ((kb + 1) * BK) / p.G);  // next stage's scale in flight
+            const uint32_t bi = bi_nxt;
+            if (FMT == 4 && i + 1 < nkl) bi_nxt = __ldg(brow + ((kb + 1) * BK) / p.G);
             uint32_t wv[32];
             auto put = [&](int k, uint4 v) {
                 wv[4 * k] = v.x;
@@ -243,7 +259,41 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_small_kernel(const __grid_co
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.cempty[i % CST]);
             };
-            if constexpr (FMT == 2) {
+            if constexpr (FMT == 4) {
+                // the stage's 32 code bytes (64 nibbles, low nibble first)
+                uint32_t wd[8];
+                if (CODES_TMA) {
+                    if (!mbar_wait(&sm.full_c[i % CST], (i / CST) & 1, abort_flag, lim)) break;
+                    const uint4* cw = reinterpret_cast<const uint4*>(sm.c[i % CST] + t * C_ROW);
+                    const uint4 v0 = cw[0], v1 = cw[1];
+                    wd[0] = v0.x, wd[1] = v0.y, wd[2] = v0.z, wd[3] = v0.w;
+                    wd[4] = v1.x, wd[5] = v1.y, wd[6] = v1.z, wd[7] = v1.w;
+                    release_window();
+                } else {
+                    const uint32_t* cw = reinterpret_cast<const uint32_t*>(crow + (int64_t)g * p.B + q_lo);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) wd[j] = __ldg(cw + j);
+                }
+                if (use > 0 && !mbar_wait(&sm.wempty[st], (use - 1) & 1, abort_flag, lim)) break;
+                const float s = __uint_as_float(sc << 16), b = __uint_as_float(bi << 16);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {  // columns 32 h .. 32 h + 31
+                    uint32_t hv[16], lv[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {  // columns 32 h + 2 j, + 1: byte j % 4 of word 4 h + j / 4
+                        const uint32_t by = wd[4 * h + (j >> 2)] >> (8 * (j & 3));
+                        const float w0 = fmaf((float)(by & 0xFu), s, b), w1 = fmaf((float)((by >> 4) & 0xFu), s, b);
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(w0, w1);
+                        const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h2);
+                        const __nv_bfloat162 l2 = __floats2bfloat162_rn(w0 - __uint_as_float(hb << 16),
+                                                                        w1 - __uint_as_float(hb & 0xFFFF0000u));
+                        hv[j] = hb;
+                        lv[j] = *reinterpret_cast<const uint32_t*>(&l2);
+                    }
+                    tmem_st16(trow + SLOT * (uint32_t)st + 16u * h, hv);
+                    tmem_st16(trow + SLOT * (uint32_t)st + 32u + 16u * h, lv);
+                }
+            } else if constexpr (FMT == 2) {
                 // the stage's 16 code bytes start on a 16-byte boundary of the row
                 uint32_t wd[4];
                 if (CODES_TMA) {
@@ -281,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_small_kernel(const __grid_co
                     for (int j = 0; j < 14; ++j) cur[j] = nxt[j];
                 }
             }
-            tmem_st32(trow + 32u * (uint32_t)st, wv);
+            if constexpr (FMT != 4) tmem_st32(trow + SLOT * (uint32_t)st, wv);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_w[st]);
@@ -339,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 2) gemm_small_kernel(const __grid_co
         const int64_t n = n0 + crank * RPQ + rr;
         if (n < p.N) {
             const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
-            if (mq == 0 && acc.x != acc.x)  // NaN output of the first token: rescan that W row
+            if (FMT != 4 && mq == 0 && acc.x != acc.x)  // NaN output of the first token: rescan that W row
                 err_acc |= FMT == 3 ? scan_row_errors(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G, p.B)
                                     : scan_row_errors2(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G);
 #pragma unroll
@@ -402,13 +452,15 @@ cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* code
                                cudaStream_t stream, int sm_count, bool* handled, int fmt);
 
 // Covered shapes: 1 <= M <= 64, K % 64 == 0, G % 64 == 0.  Otherwise *handled is
-// left false and nothing is launched.  fmt: 3 base-3 codes, 2 the 2-bit format.
+// left false and nothing is launched.  fmt: 3 base-3 codes, 2 the 2-bit format,
+// 4 the W4A16 affine codes with `biases` (the split-K kernel only: a shape
+// that would take the persistent kernel is left unhandled).
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                               int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                              cudaStream_t stream, int sm_count, bool* handled, int fmt) {
+                              cudaStream_t stream, int sm_count, bool* handled, int fmt, const uint16_t* biases) {
     using namespace small;
     *handled = false;
-    const int B = fmt == 3 ? bytes_per_group(G) : G / 4;
+    const int B = fmt == 3 ? bytes_per_group(G) : (fmt == 2 ? G / 4 : G / 2);
     const int64_t row_bytes = (int64_t)(K / G) * B;
     if (M < 1 || M > 64 || K % BK != 0 || G % 64 != 0 || N > (int64_t(1) << 31) || K > (1 << 30))
         return cudaSuccess;
@@ -433,13 +485,16 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     // every SM (16/32-token tiles fit twice) and decodes before its wait
     const int64_t slots = (int64_t)sm_count;
     while (CS < kMaxCS && tiles * CS * 2 <= slots && nk / (CS * 2) >= 2) CS *= 2;
-    if (CS == 1)  // no K split: the persistent kernel walks the tiles
+    if (CS == 1) {  // no K split: the persistent kernel walks the tiles
+        if (fmt == 4) return cudaSuccess;
         return launch_gemm_stream(X, M, codes, scales, N, K, G, Y, y_bf16, d_err, stream, sm_count, handled, fmt);
+    }
     Params p{};
     p.wc = tc::wait_cfg_from_env();
     p.codes = codes;
     p.row_bytes = row_bytes;
     p.scales = scales;
+    p.biases = biases;
     p.Y = Y;
     p.d_err = d_err;
     p.M = M;
@@ -452,7 +507,17 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     p.y_bf16 = y_bf16;
     padding_range(G, p.pad_base, p.pad_span);
     cudaError_t e;
-    if (fmt == 2) {
+    if (fmt == 4) {
+        if (codes_tma) {
+            if (NT == 16) e = launch_nt<16, true, 4>(tx, tcm, p, (int)tiles, stream);
+            else if (NT == 32) e = launch_nt<32, true, 4>(tx, tcm, p, (int)tiles, stream);
+            else e = launch_nt<64, true, 4>(tx, tcm, p, (int)tiles, stream);
+        } else {
+            if (NT == 16) e = launch_nt<16, false, 4>(tx, tcm, p, (int)tiles, stream);
+            else if (NT == 32) e = launch_nt<32, false, 4>(tx, tcm, p, (int)tiles, stream);
+            else e = launch_nt<64, false, 4>(tx, tcm, p, (int)tiles, stream);
+        }
+    } else if (fmt == 2) {
         if (codes_tma) {
             if (NT == 16) e = launch_nt<16, true, 2>(tx, tcm, p, (int)tiles, stream);
             else if (NT == 32) e = launch_nt<32, true, 2>(tx, tcm, p, (int)tiles, stream);

@@ -35,7 +35,7 @@ cudaError_t launch_gemv_predecode(const uint16_t* X, int64_t M, const uint8_t* c
                                   cudaStream_t stream, int sm_count, int fmt);
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                               int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                              cudaStream_t stream, int sm_count, bool* handled, int fmt);
+                              cudaStream_t stream, int sm_count, bool* handled, int fmt, const uint16_t* biases = nullptr);
 cudaError_t launch_quantize_pack2(const uint16_t* W, int64_t N, int64_t K, int G, uint8_t* codes,
                                   uint16_t* scales, uint32_t* d_err, cudaStream_t stream, int sm_count);
 cudaError_t launch_unpack2(const uint8_t* codes, const uint16_t* scales, int64_t N, int64_t K, int G, uint16_t* out,
@@ -477,6 +477,20 @@ tq_status tq_w4_gemv(const void* X, int64_t M, const uint32_t* codes, const void
         if (e != cudaErrorNotSupported) return from_cuda(e);  // NotSupported only from the first launch
         cudaGetLastError();
     }
+    // 5..64 tokens: the split-K tensor kernel, each weight as two bf16 terms
+    // in tensor memory, where it takes the shape (M-sweep projections 1536 x
+    // 1536 .. 4096 x 1536: 4.8-8.9 us at 16 tokens against 9.2-17.7 us for
+    // 8 tokens on the CUDA-core kernel)
+    if (M >= 5 && M <= 64) {
+        bool handled = false;
+        const cudaError_t e = launch_gemm_small(static_cast<const uint16_t*>(X), M,
+                                                reinterpret_cast<const uint8_t*>(codes),
+                                                static_cast<const uint16_t*>(scales), N, K, G, Y, yt == TQ_OUT_BF16,
+                                                nullptr, (cudaStream_t)stream, d->sm_count, &handled, 4,
+                                                static_cast<const uint16_t*>(biases));
+        if (e != cudaSuccess) return from_cuda(e);
+        if (handled) return TQ_OK;
+    }
     const cudaError_t e = launch_gemv_w4(static_cast<const uint16_t*>(X), M, codes, static_cast<const uint16_t*>(scales),
                                          static_cast<const uint16_t*>(biases), N, K, G, Y, yt == TQ_OUT_BF16,
                                          (cudaStream_t)stream, d->sm_count);
@@ -503,6 +517,15 @@ tq_status tq_w4_gemm(const void* X, int64_t M, const uint32_t* codes, const void
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
     bool handled = false;
+    if (M <= 64) {  // small M: the split-K tensor kernel (W in tensor memory) where it takes the shape
+        const cudaError_t e = launch_gemm_small(static_cast<const uint16_t*>(X), M,
+                                                reinterpret_cast<const uint8_t*>(codes),
+                                                static_cast<const uint16_t*>(scales), N, K, G, Y, yt == TQ_OUT_BF16,
+                                                nullptr, (cudaStream_t)stream, d->sm_count, &handled, 4,
+                                                static_cast<const uint16_t*>(biases));
+        if (e != cudaSuccess) return from_cuda(e);
+        if (handled) return TQ_OK;
+    }
     const cudaError_t e = launch_gemm_tc(static_cast<const uint16_t*>(X), M, reinterpret_cast<const uint8_t*>(codes),
                                          static_cast<const uint16_t*>(scales), N, K, G, Y, yt == TQ_OUT_BF16, nullptr,
                                          (cudaStream_t)stream, d->sm_count, &handled, 4,
