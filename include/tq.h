@@ -228,8 +228,9 @@ TQ_API size_t tq_w4_codes_bytes(int64_t N, int64_t K, int G);
  * thread-block cluster), one launch per token, for one token from 12 Mi
  * weights (6 Mi at K >= 2048) and for 2..4 tokens from 12 Mi weights at
  * K <= 512 or from 96 Mi weights at any K; 5..64 tokens with G % 64 == 0
- * and K % 64 == 0 on matrices of at most about 9,500 rows the split-K
- * tensor-core kernel (each weight as two bf16 terms, as tq_w4_gemm); other
+ * and K % 64 == 0 the small-M tensor-core kernels (each weight as two bf16
+ * terms, as tq_w4_gemm; above about 9,500 rows only with 16-byte-aligned
+ * codes); other
  * shapes with G % 32 == 0, K % 32 == 0 and K <= 4096 the CUDA-core streaming
  * kernel, eight tokens per launch, and the rest a plain one-warp-per-row
  * kernel.
@@ -243,10 +244,10 @@ TQ_API tq_status tq_w4_gemv(const void *X_bf16, int64_t M, const uint32_t *codes
  * fp32 accumulators in tensor memory): the same result definition as
  * tq_w4_gemv.  Each weight w = q * s + b is formed with one fp32 FMA and fed
  * to the MMA as two bf16 terms, RNE_bf16(w) and RNE_bf16 of the remainder,
- * so the products keep w to about 2^-17 relative.  Up to 64 tokens on
- * matrices of at most about 9,500 rows the split-K small-M kernel (the two
- * terms stored in tensor memory as the MMA's A operand), otherwise the
- * prefill kernel.  Needs K % 64 == 0 and G % 64 == 0, else
+ * so the products keep w to about 2^-17 relative.  Up to 64 tokens the
+ * small-M kernels (the two terms stored in tensor memory as the MMA's A
+ * operand; above about 9,500 rows only with 16-byte-aligned codes),
+ * otherwise the prefill kernel.  Needs K % 64 == 0 and G % 64 == 0, else
  * TQ_ERR_UNSUPPORTED; other arguments as tq_w4_gemv. */
 TQ_API tq_status tq_w4_gemm(const void *X_bf16, int64_t M, const uint32_t *codes, const void *scales_bf16,
                      const void *biases_bf16, int64_t N, int64_t K, int G, void *Y, tq_out_dtype y_dtype,

@@ -449,12 +449,12 @@ static cudaError_t launch_nt(const CUtensorMap& tx, const CUtensorMap& tc_, cons
 
 cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                               cudaStream_t stream, int sm_count, bool* handled, int fmt);
+                               cudaStream_t stream, int sm_count, bool* handled, int fmt, const uint16_t* biases);
 
 // Covered shapes: 1 <= M <= 64, K % 64 == 0, G % 64 == 0.  Otherwise *handled is
 // left false and nothing is launched.  fmt: 3 base-3 codes, 2 the 2-bit format,
-// 4 the W4A16 affine codes with `biases` (the split-K kernel only: a shape
-// that would take the persistent kernel is left unhandled).
+// 4 the W4A16 affine codes with `biases` (the persistent kernel needs
+// 16-byte-aligned codes for them, else the shape is left unhandled).
 cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                               int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
                               cudaStream_t stream, int sm_count, bool* handled, int fmt, const uint16_t* biases) {
@@ -485,10 +485,9 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t M, const uint8_t* codes
     // every SM (16/32-token tiles fit twice) and decodes before its wait
     const int64_t slots = (int64_t)sm_count;
     while (CS < kMaxCS && tiles * CS * 2 <= slots && nk / (CS * 2) >= 2) CS *= 2;
-    if (CS == 1) {  // no K split: the persistent kernel walks the tiles
-        if (fmt == 4) return cudaSuccess;
-        return launch_gemm_stream(X, M, codes, scales, N, K, G, Y, y_bf16, d_err, stream, sm_count, handled, fmt);
-    }
+    if (CS == 1)  // no K split: the persistent kernel walks the tiles
+        return launch_gemm_stream(X, M, codes, scales, N, K, G, Y, y_bf16, d_err, stream, sm_count, handled, fmt,
+                                  biases);
     Params p{};
     p.wc = tc::wait_cfg_from_env();
     p.codes = codes;

@@ -40,14 +40,17 @@ constexpr int CR = 4;      // code windows in flight per decoder thread
 constexpr int kThreads = 512;
 constexpr int kDecWarp0 = 4, kEpiWarp0 = 12;
 constexpr int kGroupWarps = 4;
-constexpr uint32_t WIN = 48;               // per row: 32 code bytes, the 4-byte word holding the scale, pad
+constexpr uint32_t WIN = 48;  // per row: 32 code bytes, the 4-byte words holding the scale and (W4A16) the bias
 
 // Tensor memory: two accumulators of NT columns, then one 32-column slot of
 // decoded W (128 x 64 bf16) per stage.
 template <int NT>
 constexpr uint32_t kAccCols = 2 * NT;
-template <int NT>
-constexpr uint32_t kTmemCols = kAccCols<NT> + 32 * STAGES <= 256 ? 256 : 512;
+// columns of a stage's W slot: 32 (64 bf16 of a row), 64 for W4A16 (hi and lo terms)
+template <int FMT>
+constexpr uint32_t kSlotCols = FMT == 4 ? 64 : 32;
+template <int NT, int FMT>
+constexpr uint32_t kTmemCols = kAccCols<NT> + kSlotCols<FMT> * STAGES <= 256 ? 256 : 512;
 
 template <int NT>
 struct Smem {
@@ -66,6 +69,8 @@ struct Params {
     int64_t row_bytes;
     const uint16_t* scales;
     const uint16_t* scales_end;
+    const uint16_t* biases;  // W4A16 only
+    const uint16_t* biases_end;
     void* Y;
     uint32_t* d_err;
     int64_t M, N;
@@ -124,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
     const int nk = p.K / BK;
     const int my_tiles = (p.tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const int total = my_tiles * nk;  // stages of this CTA
-    constexpr uint32_t kCols = kTmemCols<NT>, ACC = kAccCols<NT>;
+    constexpr uint32_t kCols = kTmemCols<NT, FMT>, ACC = kAccCols<NT>, SLOT = kSlotCols<FMT>;
     volatile int* abort_flag = &sm.abort_flag;
     const uint64_t lim = p.wc.limit_ns;
 
@@ -198,10 +203,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = tmem + ACC + 32u * (uint32_t)st, b0 = s32(sm.x[st]);
+                    const uint32_t a0 = tmem + ACC + SLOT * (uint32_t)st, b0 = s32(sm.x[st]);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
+                    for (int k = 0; k < BK / 16; ++k) {
                         mma_bf16_ts(d, a0 + 8u * k, smem_desc_sw128(b0 + 32 * k), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                        if (FMT == 4)  // the lo terms, 32 columns on
+                            mma_bf16_ts(d, a0 + 32u + 8u * k, smem_desc_sw128(b0 + 32 * k), idesc, 1u);
+                    }
                     mma_commit(&sm.empty[st]);
                 }
                 if (ok) mma_commit(&sm.tfull[buf]);
@@ -241,10 +249,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
         auto issue = [&](int s) {
             if (grp + 2 * s < total) {
                 const int64_t n = row_of(pi);
-                const int q_lo = FMT == 3 ? (BK * pi.sub) / 5 : (BK * pi.sub) / 4;
+                const int q_lo = FMT == 3 ? (BK * pi.sub) / 5 : (FMT == 2 ? (BK * pi.sub) / 4 : (BK * pi.sub) / 2);
                 uint8_t* slot = sm.win[grp][s % CR] + t * WIN;
                 fetch_window(slot, p.codes + n * p.row_bytes + (int64_t)pi.g * p.B + q_lo, p.codes, p.codes_end);
                 fetch_scale(slot + 32, p.scales + n * p.ng + pi.g, p.scales, p.scales_end);
+                if (FMT == 4) fetch_scale(slot + 36, p.biases + n * p.ng + pi.g, p.biases, p.biases_end);
                 advance(pi);
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
@@ -257,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
             const int i = grp + 2 * s, st = i % STAGES, use = i / STAGES;
             if (use > 0 && !mbar_wait(&sm.empty[st], (use - 1) & 1, abort_flag, lim)) break;
             const int64_t n = row_of(pd);
-            const int c0 = BK * pd.sub, q_lo = FMT == 3 ? c0 / 5 : c0 / 4;
+            const int c0 = BK * pd.sub, q_lo = FMT == 3 ? c0 / 5 : (FMT == 2 ? c0 / 4 : c0 / 2);
             const uintptr_t A = reinterpret_cast<uintptr_t>(p.codes + n * p.row_bytes + (int64_t)pd.g * p.B + q_lo);
             const uintptr_t S = reinterpret_cast<uintptr_t>(p.scales + n * p.ng + pd.g);
             const uint8_t* slot = sm.win[grp][s % CR] + t * WIN;
@@ -270,7 +279,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
                 wv[4 * k + 2] = v.z;
                 wv[4 * k + 3] = v.w;
             };
-            if constexpr (FMT == 2) {  // codes 4-byte aligned: cb is a word boundary of the window
+            if constexpr (FMT == 4) {  // codes 16-byte aligned: the window is the stage's 32 bytes
+                const uint4 v0 = *reinterpret_cast<const uint4*>(slot), v1 = *reinterpret_cast<const uint4*>(slot + 16);
+                const uint32_t wd[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                const uintptr_t Bi = reinterpret_cast<uintptr_t>(p.biases + n * p.ng + pd.g);
+                const uint32_t bi = *reinterpret_cast<const uint16_t*>(slot + 36 + (Bi & 2));
+                const float s_ = __uint_as_float(sc << 16), b_ = __uint_as_float(bi << 16);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {  // columns 32 h .. 32 h + 31
+                    uint32_t hv[16], lv[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {  // columns 32 h + 2 j, + 1: byte j % 4 of word 4 h + j / 4
+                        const uint32_t by = wd[4 * h + (j >> 2)] >> (8 * (j & 3));
+                        const float w0 = fmaf((float)(by & 0xFu), s_, b_), w1 = fmaf((float)((by >> 4) & 0xFu), s_, b_);
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(w0, w1);
+                        const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h2);
+                        const __nv_bfloat162 l2 = __floats2bfloat162_rn(w0 - __uint_as_float(hb << 16),
+                                                                        w1 - __uint_as_float(hb & 0xFFFF0000u));
+                        hv[j] = hb;
+                        lv[j] = *reinterpret_cast<const uint32_t*>(&l2);
+                    }
+                    tmem_st16(trow + SLOT * (uint32_t)st + 16u * h, hv);
+                    tmem_st16(trow + SLOT * (uint32_t)st + 32u + 16u * h, lv);
+                }
+            } else if constexpr (FMT == 2) {  // codes 4-byte aligned: cb is a word boundary of the window
                 const uint32_t* cw = reinterpret_cast<const uint32_t*>(cb);
                 const uint32_t wd[4] = {cw[0], cw[1], cw[2], cw[3]};
                 decode_stage64_2bit_to(wd, sc, put);
@@ -282,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
                 decode_stage64_to<32>(sm.lut + (t & 31), bytes, c0 - 5 * q_lo, ql < 14, ql < 14 ? cb[ql] : 0u,
                                       p.pad_base, p.pad_span, sc, put);
             }
-            tmem_st32(trow + 32u * (uint32_t)st, wv);
+            if constexpr (FMT != 4) tmem_st32(trow + SLOT * (uint32_t)st, wv);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.full_w[st]);
@@ -309,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_stream_kernel(const __grid_c
             if (lane == 0) mbar_arrive(&sm.tempty[buf]);
             const int64_t n = ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * WM + 32 * q + lane;
             if (n < p.N) {
-                if (__uint_as_float(v[0]) != __uint_as_float(v[0]))  // NaN for the first token: rescan the row
+                if (FMT != 4 && __uint_as_float(v[0]) != __uint_as_float(v[0]))  // NaN for the first token: rescan the row
                     err_acc |= FMT == 3 ? scan_row_errors(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G, p.B)
                                         : scan_row_errors2(p.codes + n * p.row_bytes, p.scales + n * p.ng, p.ng, p.G);
 #pragma unroll
@@ -365,13 +397,15 @@ static cudaError_t launch_nt(const CUtensorMap& tx, const Params& p, int grid, c
 // *handled is left false and nothing is launched.
 cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* codes, const uint16_t* scales,
                                int64_t N, int64_t K, int G, void* Y, int y_bf16, uint32_t* d_err,
-                               cudaStream_t stream, int sm_count, bool* handled, int fmt) {
+                               cudaStream_t stream, int sm_count, bool* handled, int fmt, const uint16_t* biases) {
     using namespace stream;
     *handled = false;
     if (M < 1 || M > 64 || K % BK != 0 || G % 64 != 0 || N < 1 || K > (1 << 30)) return cudaSuccess;
+    // W4A16: a stage's 32 code bytes must be one 16-byte-aligned window
+    if (fmt == 4 && (reinterpret_cast<uintptr_t>(codes) & 15)) return cudaSuccess;
     const int64_t tiles = (N + WM - 1) / WM;
     if (tiles > 0x7FFFFFFF / (K / BK)) return cudaSuccess;
-    const int B = fmt == 3 ? bytes_per_group(G) : G / 4;
+    const int B = fmt == 3 ? bytes_per_group(G) : (fmt == 2 ? G / 4 : G / 2);
     const int NT = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
     CUtensorMap tx;
     if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<uint16_t*>(X), (uint64_t)K, (uint64_t)M,
@@ -384,6 +418,8 @@ cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* code
     p.codes_end = codes + N * p.row_bytes;
     p.scales = scales;
     p.scales_end = scales + N * (K / G);
+    p.biases = biases;
+    p.biases_end = biases ? biases + N * (K / G) : nullptr;
     p.Y = Y;
     p.d_err = d_err;
     p.M = M;
@@ -397,7 +433,11 @@ cudaError_t launch_gemm_stream(const uint16_t* X, int64_t M, const uint8_t* code
     padding_range(G, p.pad_base, p.pad_span);
     const int grid = (int)(tiles < sm_count ? tiles : sm_count);
     cudaError_t e;
-    if (fmt == 2) {
+    if (fmt == 4) {
+        if (NT == 16) e = launch_nt<16, 4>(tx, p, grid, stream);
+        else if (NT == 32) e = launch_nt<32, 4>(tx, p, grid, stream);
+        else e = launch_nt<64, 4>(tx, p, grid, stream);
+    } else if (fmt == 2) {
         if (NT == 16) e = launch_nt<16, 2>(tx, p, grid, stream);
         else if (NT == 32) e = launch_nt<32, 2>(tx, p, grid, stream);
         else e = launch_nt<64, 2>(tx, p, grid, stream);

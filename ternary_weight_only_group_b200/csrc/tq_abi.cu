@@ -477,10 +477,11 @@ tq_status tq_w4_gemv(const void* X, int64_t M, const uint32_t* codes, const void
         if (e != cudaErrorNotSupported) return from_cuda(e);  // NotSupported only from the first launch
         cudaGetLastError();
     }
-    // 5..64 tokens: the split-K tensor kernel, each weight as two bf16 terms
-    // in tensor memory, where it takes the shape (M-sweep projections 1536 x
-    // 1536 .. 4096 x 1536: 4.8-8.9 us at 16 tokens against 9.2-17.7 us for
-    // 8 tokens on the CUDA-core kernel)
+    // 5..64 tokens: the small-M tensor kernels (split-K for few row tiles,
+    // persistent for many), each weight as two bf16 terms in tensor memory,
+    // where they take the shape (M-sweep projections 1536 x 1536 .. 4096 x
+    // 1536: 4.8-8.9 us at 16 tokens against 9.2-17.7 us for 8 tokens on the
+    // CUDA-core kernel)
     if (M >= 5 && M <= 64) {
         bool handled = false;
         const cudaError_t e = launch_gemm_small(static_cast<const uint16_t*>(X), M,
@@ -517,7 +518,7 @@ tq_status tq_w4_gemm(const void* X, int64_t M, const uint32_t* codes, const void
     const DeviceInfo* d = nullptr;
     if (tq_status st = device_info(&d)) return st;
     bool handled = false;
-    if (M <= 64) {  // small M: the split-K tensor kernel (W in tensor memory) where it takes the shape
+    if (M <= 64) {  // small M: the small-M tensor kernels (W in tensor memory) where they take the shape
         const cudaError_t e = launch_gemm_small(static_cast<const uint16_t*>(X), M,
                                                 reinterpret_cast<const uint8_t*>(codes),
                                                 static_cast<const uint16_t*>(scales), N, K, G, Y, yt == TQ_OUT_BF16,

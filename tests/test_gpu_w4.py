@@ -147,6 +147,30 @@ def test_w4_gemv_stream_unaligned_operands():
     assert_rows_close_f32(to_f64(Y), ref)
 
 
+@pytest.mark.parametrize("M", [5, 16, 40])
+@pytest.mark.parametrize("N,K,G", [(16411, 1024, 128), (12007, 2048, 64)])
+def test_w4_gemv_persistent_tensor_path(N, K, G, M):
+    """5..64 tokens on matrices with more 128-row tiles than half the SMs:
+    the persistent small-M tensor kernel (hi and lo bf16 terms of each weight
+    in tensor memory), token tiles of 16 and 64, ragged last tile."""
+    check(N, K, G, M, index=N + M, dtypes=(torch.float32,))
+
+
+def test_w4_gemv_persistent_unaligned_codes():
+    """Codes 4 bytes past a 16-byte boundary: the persistent tensor kernel
+    (16-byte code windows) declines and the CUDA-core kernel answers."""
+    N, K, G, M = 16411, 1024, 128, 8
+    codes, scales, biases = synthetic.w4_params(N, K, G, index=9)
+    X = synthetic.activations(M, K, offset=806)
+    ref = oracle.linear_w4(X, codes, scales, biases, N, K, G)
+    dc, ds, db = dev_params(codes, scales, biases)
+    flat = torch.empty(dc.numel() + 1, dtype=torch.int32, device="cuda")
+    flat[1:] = dc.reshape(-1)
+    Y = tq.w4_gemv(to_dev_bf16(X), flat[1:].view(N, K // 8), ds, db, N, K, G, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert_rows_close_f32(to_f64(Y), ref)
+
+
 @pytest.mark.parametrize("M", [1, 16, 256, 300])
 @pytest.mark.parametrize("N,K,G", [(512, 1024, 128), (1000, 4096, 64), (4096, 1024, 128), (130, 2048, 256)])
 def test_w4_gemm_tensor_cores(N, K, G, M):
